@@ -1,0 +1,331 @@
+"""Benchmark of the binary-weight decode GEMV (one JSON line on rank 0).
+
+Default workload: the Llama-7B attention projection, 4096x4096 with two binary
+bases and bf16 row/column scales, batch M=1. One step = one replay of a CUDA
+graph holding S back-to-back GEMVs over S distinct weight copies whose total
+size exceeds 3x the L2 cache, so every GEMV streams its weights from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bisco|reference]
+                    [--workload attn4096|mlp_gate_up|mlp_down|lowrank5120|cfg1] [--M m]
+
+Metric: effective HBM GB/s of the M=1 binary GEMV (algorithmic bytes: packed
+sign bits, scales, correction signs and coefficients, salient payload, X read
+and Y written, over device time); the microseconds per GEMV are reported too.
+Multi-GPU runs are weak-scaling replicas: every rank streams its own layers,
+there is no data-path collective, and the time is the max over ranks.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth.configs import build  # noqa: E402
+
+WORKLOADS = {
+    # name: (config, spec index, default M, description)
+    "attn4096": (2, 0, 1, "Llama-7B attention projection 4096x4096, 2 binary bases, bf16 scales"),
+    "mlp_gate_up": (3, 0, 1, "Llama-7B MLP gate/up 4096->11008, 2 bases, 1% salient int8 columns"),
+    "mlp_down": (3, 1, 1, "Llama-7B MLP down 11008->4096, 2 bases, 1% salient int8 columns"),
+    "lowrank5120": (4, 0, 1, "5120x5120, 2 bases + rank-512 binary correction, 0.1% outliers x20"),
+    "cfg1": (1, 0, 1, "256x512, 1 base, fp32 scales, rank-8 correction"),
+}
+
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def sources_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "binary_weight_decode_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(MEASURED_PEAKS) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_for(workload, M):
+    """dram bytes per launch of the dominant kernel from a committed ncu capture,
+    or None if there is none for this workload or the kernel sources changed."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        e = t.get(f"{workload}_M{M}")
+        if e and e.get("sources") == sources_digest():
+            return e["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_baseline(workload, M, budget_s=12.0):
+    """The fp64 oracle, as it stands, on this host's cores over a bounded sample."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    cfg, spec, _, _ = WORKLOADS[workload]
+    L, X = build(cfg, spec, M)
+    xdt = "f32" if cfg == 1 else "bf16"
+    nbytes = oracle.algorithmic_bytes(L, M, xdt, "bf16")
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.gemv(L, X, xdt)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 200:
+            break
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": round(n * nbytes / el / 1e9, 4), "unit": "GB/s", "cores": int(threads),
+            "kind": "oracle", "us_per_gemv": el / n * 1e6,
+            "sample": f"{n} full fp64 oracle GEMVs of the {workload} layer (M={M}) in {el:.1f} s on {os.cpu_count()} host cores"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    cb = cpu_baseline(args.workload, args.M, budget_s=max(5.0, 3.0 * args.steps))
+    cfg, spec, _, desc = WORKLOADS[args.workload]
+    line = {"metric": "M=1 binary-GEMV effective HBM GB/s", "value": cb["value"], "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": cb["us_per_gemv"] / 1000.0, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{args.workload}: {desc}", "M": args.M},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def algorithmic_bytes(L, M, x_bytes, y_bytes):
+    """Bytes one GEMV must move (same accounting as the oracle's, restated for the
+    product path so that the bench does not depend on the oracle)."""
+    sb = 2 if L.scale_dtype == "bf16" else 4
+    n = L.K * L.out * L.in_ / 8.0 + L.K * (L.out + L.in_) * sb
+    if L.rank:
+        n += L.rank * (L.out + L.in_) / 8.0 + 4 * L.rank
+    if L.n_sal:
+        n += L.out * L.n_sal + 8 * L.n_sal
+    n += M * L.in_ * x_bytes + M * L.out * y_bytes
+    return int(round(n))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="bisco", choices=["bisco", "reference"])
+    ap.add_argument("--workload", default="attn4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--M", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg, spec, m_default, desc = WORKLOADS[args.workload]
+    args.M = args.M or m_default
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import binary_weight_decode_b200 as bw
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    M = args.M
+    L, X = build(cfg, spec, M)
+    xdt = "f32" if cfg == 1 else "bf16"
+    x_bytes = 4 if xdt == "f32" else 2
+    y_dtype = torch.bfloat16
+    nbytes = algorithmic_bytes(L, M, x_bytes, 2)
+    props = torch.cuda.get_device_properties(local)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    S = max(4, math.ceil(3 * l2 / nbytes))
+
+    # S distinct weight copies: same values, separate HBM buffers
+    dls = [bw.DeviceLayer(L) for _ in range(S)]
+    Xh = torch.from_numpy(X.view(np.int16) if xdt == "bf16" else X)
+    Xd = Xh.to("cuda")
+    if xdt == "bf16":
+        Xd = Xd.view(torch.bfloat16)
+    Yd = torch.empty((S, M, L.out), dtype=y_dtype, device="cuda")
+    ws = bw.alloc_workspace(dls[:1], M)
+
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for i in range(S):  # eager warm-up run (also sets kernel attributes before capture)
+            bw.bisco_gemv(dls[i], Xd, Yd[i], ws, stream=stream)
+    stream.synchronize()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(S):
+            bw.bisco_gemv(dls[i], Xd, Yd[i], ws, stream=stream)
+    kernels_per_gemv = (2 if L.rank else 1) * math.ceil(M / 8)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # graph replays and events all go to `stream` (CUDAGraph.replay uses the current stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1)
+    clocks = sampler.stop()
+    if dist is not None:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    gemvs = args.steps * S
+    us_per_gemv = ms * 1000.0 / gemvs
+    value = world * gemvs * nbytes / (ms / 1000.0) / 1e9
+
+    # end to end through the public API: pinned host X in, host Y out, every step
+    Xpin = Xh.pin_memory()
+    Ypin = torch.empty((S, M, L.out), dtype=torch.int16).pin_memory()
+    Yd16 = Yd.view(torch.int16)
+    Xd_raw = Xd.view(torch.int16) if xdt == "bf16" else Xd
+    e2 = torch.cuda.Event(enable_timing=True)
+    e3 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps // 2)
+    barrier()
+    e2.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(e2e_steps):
+            Xd_raw.copy_(Xpin, non_blocking=True)
+            graph.replay()
+            Ypin.copy_(Yd16, non_blocking=True)
+    e3.record(stream)
+    barrier()
+    ms_e2e = e2.elapsed_time(e3)
+    if dist is not None:
+        t = torch.tensor([ms_e2e], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = world * e2e_steps * S * nbytes / (ms_e2e / 1000.0) / 1e9
+
+    peak, peak_kind = hbm_peak()
+    achieved = nbytes / (us_per_gemv * 1e-6) / 1e9
+    line = {
+        "metric": "M=1 binary-GEMV effective HBM GB/s", "value": round(value, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "bisco",
+        "config": {"workload": f"{args.workload}: {desc}", "M": M, "gemvs_per_step": S,
+                   "algorithmic_bytes_per_gemv": nbytes, "y_dtype": "bf16",
+                   "l2": f"inputs larger than L2: each step streams {S} distinct weight copies "
+                         f"({S * nbytes / 2 ** 20:.0f} MiB > 3x L2)",
+                   "parallelism": f"replicas x{world} (no collective)"},
+        "us_per_gemv": round(us_per_gemv, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
+                     "frac_of_8000": round(achieved / 8000.0, 4),
+                     "traffic": traffic_for(args.workload, M)},
+        "clocks": clocks,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
+                "d2h_bytes_per_step": int(Ypin.numel() * 2)},
+        "gpu_launches": int(args.steps * S * kernels_per_gemv),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, M)
+    del graph
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

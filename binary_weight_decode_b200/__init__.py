@@ -1,0 +1,236 @@
+"""Python binding of libbisco (binary-weight decode GEMV for B200).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library. PyTorch provides device memory and streams. Importing this package
+fails loudly if ``libbisco.so`` has not been built
+(``python -m binary_weight_decode_b200.build``).
+
+The functions carry the names of the C entry points in ``include/bisco.h``.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbisco.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m binary_weight_decode_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+BISCO_OK, BISCO_ERR_INVALID_ARG, BISCO_ERR_UNSUPPORTED, BISCO_ERR_CUDA, BISCO_ERR_TIMEOUT, BISCO_ERR_WORKSPACE = range(6)
+BISCO_F32, BISCO_BF16 = 0, 1
+
+EXPORTED = [
+    "bisco_packed_words", "bisco_pack", "bisco_unpack", "bisco_workspace_size", "bisco_workspace_init",
+    "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string",
+]
+
+
+class bisco_layer(ctypes.Structure):
+    _fields_ = [
+        ("out", ctypes.c_int32), ("in_", ctypes.c_int32), ("num_bases", ctypes.c_int32),
+        ("bits", ctypes.c_void_p), ("row_scale", ctypes.c_void_p), ("col_scale", ctypes.c_void_p),
+        ("scale_dtype", ctypes.c_int32), ("rank", ctypes.c_int32),
+        ("v_bits", ctypes.c_void_p), ("ut_bits", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+        ("n_sal", ctypes.c_int32), ("sal_stride", ctypes.c_int32),
+        ("sal_idx", ctypes.c_void_p), ("sal_q", ctypes.c_void_p), ("sal_scale", ctypes.c_void_p),
+    ]
+
+
+class bisco_bench_args(ctypes.Structure):
+    _fields_ = [
+        ("layers", ctypes.POINTER(bisco_layer)), ("n_layers", ctypes.c_int32),
+        ("X", ctypes.c_void_p), ("x_dtype", ctypes.c_int32), ("M", ctypes.c_int32),
+        ("Y", ctypes.c_void_p), ("y_dtype", ctypes.c_int32),
+        ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t),
+        ("warmup", ctypes.c_int32), ("reps", ctypes.c_int32), ("stream", ctypes.c_void_p),
+    ]
+
+
+class bisco_bench_result(ctypes.Structure):
+    _fields_ = [("us_per_gemv", ctypes.c_double), ("us_per_replay", ctypes.c_double),
+                ("kernels_per_gemv", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_lib.bisco_packed_words.argtypes = [ctypes.c_int64, ctypes.c_int64]
+_lib.bisco_packed_words.restype = ctypes.c_int64
+_lib.bisco_pack.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, _P]
+_lib.bisco_pack.restype = ctypes.c_int
+_lib.bisco_unpack.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, _P]
+_lib.bisco_unpack.restype = ctypes.c_int
+_lib.bisco_workspace_size.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+_lib.bisco_workspace_size.restype = ctypes.c_int
+_lib.bisco_workspace_init.argtypes = [_P, ctypes.c_size_t, _P]
+_lib.bisco_workspace_init.restype = ctypes.c_int
+_lib.bisco_gemv.argtypes = [ctypes.POINTER(bisco_layer), _P, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
+                            _P, ctypes.c_size_t, _P]
+_lib.bisco_gemv.restype = ctypes.c_int
+_lib.bisco_sync_status.argtypes = [_P, _P]
+_lib.bisco_sync_status.restype = ctypes.c_int
+_lib.bisco_bench.argtypes = [ctypes.POINTER(bisco_bench_args), ctypes.POINTER(bisco_bench_result)]
+_lib.bisco_bench.restype = ctypes.c_int
+_lib.bisco_status_string.argtypes = [ctypes.c_int]
+_lib.bisco_status_string.restype = ctypes.c_char_p
+
+
+class BiscoError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {bisco_status_string(status)}")
+
+
+def _check(st: int, where: str):
+    if st != BISCO_OK:
+        raise BiscoError(st, where)
+
+
+def bisco_status_string(status: int) -> str:
+    return _lib.bisco_status_string(int(status)).decode()
+
+
+def bisco_packed_words(rows: int, cols: int) -> int:
+    return int(_lib.bisco_packed_words(rows, cols))
+
+
+def bisco_pack(signs: np.ndarray) -> np.ndarray:
+    """Dense int8 +1/-1 matrix (host) -> packed uint32 words (host)."""
+    s = np.ascontiguousarray(signs, dtype=np.int8)
+    if s.ndim != 2:
+        raise ValueError("signs must be 2-D")
+    rows, cols = s.shape
+    out = np.empty(max(bisco_packed_words(rows, cols), 1), dtype=np.uint32)
+    _check(_lib.bisco_pack(s.ctypes.data, rows, cols, out.ctypes.data), "bisco_pack")
+    return out
+
+
+def bisco_unpack(words: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    if w.size < bisco_packed_words(rows, cols):
+        raise ValueError("packed buffer too small")
+    out = np.empty((rows, cols), dtype=np.int8)
+    _check(_lib.bisco_unpack(w.ctypes.data, rows, cols, out.ctypes.data), "bisco_unpack")
+    return out
+
+
+# --------------------------------------------------------------------------
+# device side (torch tensors for memory and streams)
+# --------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BISCO_BF16
+    if t.dtype == torch.float32:
+        return BISCO_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class DeviceLayer:
+    """Uploads a host layer (numpy arrays in the packed format) and holds its device
+    tensors alive together with the ``bisco_layer`` descriptor that points at them."""
+
+    def __init__(self, host, device="cuda"):
+        torch = _torch()
+
+        def up(a, dt=None):
+            if a is None:
+                return None
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:          # bf16 bit patterns
+                return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+            if a.dtype == np.uint32:
+                return torch.from_numpy(a.view(np.int32)).to(device)
+            return torch.from_numpy(a).to(device)
+
+        self.host = host
+        self.out, self.in_, self.K = host.out, host.in_, host.K
+        self.rank, self.n_sal = host.rank, host.n_sal
+        self.bits = up(host.bits) if host.K else None
+        self.row_scale = up(host.row_scale) if host.K else None
+        self.col_scale = up(host.col_scale) if host.K else None
+        self.v_bits = up(host.v_bits)
+        self.ut_bits = up(host.ut_bits)
+        self.alpha = up(host.alpha)
+        self.sal_idx = up(host.sal_idx)
+        self.sal_q = up(host.sal_q)
+        self.sal_scale = up(host.sal_scale)
+        ptr = lambda t: (t.data_ptr() if t is not None else None)  # noqa: E731
+        self.desc = bisco_layer(
+            out=host.out, in_=host.in_, num_bases=host.K,
+            bits=ptr(self.bits), row_scale=ptr(self.row_scale), col_scale=ptr(self.col_scale),
+            scale_dtype=BISCO_BF16 if host.scale_dtype == "bf16" else BISCO_F32,
+            rank=host.rank, v_bits=ptr(self.v_bits), ut_bits=ptr(self.ut_bits), alpha=ptr(self.alpha),
+            n_sal=host.n_sal, sal_stride=host.sal_stride if host.n_sal else 0,
+            sal_idx=ptr(self.sal_idx), sal_q=ptr(self.sal_q), sal_scale=ptr(self.sal_scale))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   [self.bits, self.row_scale, self.col_scale, self.v_bits, self.ut_bits, self.alpha,
+                    self.sal_idx, self.sal_q, self.sal_scale] if t is not None)
+
+
+def _desc(layer):
+    return layer.desc if isinstance(layer, DeviceLayer) else layer
+
+
+def bisco_workspace_size(layer, M: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.bisco_workspace_size(ctypes.byref(_desc(layer)), M, ctypes.byref(n)), "bisco_workspace_size")
+    return int(n.value)
+
+
+def bisco_workspace_init(ws, stream=None):
+    _check(_lib.bisco_workspace_init(ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                     _stream_ptr(stream)), "bisco_workspace_init")
+
+
+def alloc_workspace(layers, M: int, device="cuda"):
+    """Zero-initialised workspace large enough for every layer in `layers` at batch M."""
+    torch = _torch()
+    n = max(bisco_workspace_size(L, M) for L in layers)
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    bisco_workspace_init(ws)
+    return ws
+
+
+def bisco_gemv(layer, X, Y, ws, stream=None):
+    """Y[M, out] = X[M, in] @ W^T on the device (asynchronous on `stream`)."""
+    M = X.shape[0] if X.dim() == 2 else 1
+    st = _lib.bisco_gemv(ctypes.byref(_desc(layer)), ctypes.c_void_p(X.data_ptr()), _dtype_code(X), M,
+                         ctypes.c_void_p(Y.data_ptr()), _dtype_code(Y), ctypes.c_void_p(ws.data_ptr()),
+                         ws.numel() * ws.element_size(), _stream_ptr(stream))
+    _check(st, "bisco_gemv")
+    return Y
+
+
+def bisco_sync_status(ws, stream=None) -> int:
+    return int(_lib.bisco_sync_status(_stream_ptr(stream), ctypes.c_void_p(ws.data_ptr())))
+
+
+def bisco_bench(layers, X, Y, ws, warmup: int = 3, reps: int = 10, stream=None) -> dict:
+    arr = (bisco_layer * len(layers))(*[_desc(L) for L in layers])
+    M = X.shape[0]
+    args = bisco_bench_args(layers=arr, n_layers=len(layers), X=X.data_ptr(), x_dtype=_dtype_code(X), M=M,
+                            Y=Y.data_ptr(), y_dtype=_dtype_code(Y), ws=ws.data_ptr(),
+                            ws_bytes=ws.numel() * ws.element_size(), warmup=warmup, reps=reps,
+                            stream=_stream_ptr(stream).value)
+    res = bisco_bench_result()
+    _check(_lib.bisco_bench(ctypes.byref(args), ctypes.byref(res)), "bisco_bench")
+    return {"us_per_gemv": res.us_per_gemv, "us_per_replay": res.us_per_replay,
+            "kernels_per_gemv": res.kernels_per_gemv}

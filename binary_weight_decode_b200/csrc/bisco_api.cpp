@@ -1,0 +1,384 @@
+// C ABI front end: argument validation, host packing, workspace sizing and the
+// two-pass launch sequence of bisco_gemv.
+//
+// A layer with a binary low-rank correction ("BiLoCo", "The core idea": the
+// correction is applied as alpha * u * (v . x)) runs as two launches of the same
+// lookup-table kernel: pass Z computes z = alpha (.) (V x) into the workspace,
+// pass Y computes sum_k r_k (.) (B_k (c_k (.) x)) + U^T z + salient term into Y.
+// Pass Y reads z only after griddepcontrol.wait, i.e. after pass Z completed.
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "bisco_internal.h"
+
+using namespace bisco;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int cached_sms(int dev) {
+  static int sms[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return query_num_sms();
+  if (sms[dev] == 0) sms[dev] = query_num_sms();
+  return sms[dev];
+}
+
+size_t cached_smem_limit(int dev) {
+  static size_t lim[kMaxDevices] = {0};
+  if (dev < 0 || dev >= kMaxDevices) return query_smem_limit();
+  if (lim[dev] == 0) lim[dev] = query_smem_limit();
+  return lim[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(int32_t d) { return d == BISCO_F32 || d == BISCO_BF16; }
+size_t dtype_bytes(int32_t d) { return d == BISCO_BF16 ? 2 : 4; }
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
+int quads(int n) { return (n + 127) / 128; }
+
+bisco_status validate_layer(const bisco_layer* L) {
+  if (!L) return BISCO_ERR_INVALID_ARG;
+  if (L->out < 1 || L->in < 1 || L->num_bases < 0 || L->num_bases > kMaxBases) return BISCO_ERR_INVALID_ARG;
+  if (L->rank < 0 || L->rank > (1 << 20) || L->n_sal < 0 || L->n_sal > L->in) return BISCO_ERR_INVALID_ARG;
+  if (L->num_bases > 0) {
+    if (!L->bits || !L->row_scale || !L->col_scale || !aligned16(L->bits)) return BISCO_ERR_INVALID_ARG;
+    if (!dtype_ok(L->scale_dtype)) return BISCO_ERR_INVALID_ARG;
+  }
+  if (L->rank > 0) {
+    if (!L->v_bits || !L->ut_bits || !L->alpha) return BISCO_ERR_INVALID_ARG;
+    if (!aligned16(L->v_bits) || !aligned16(L->ut_bits)) return BISCO_ERR_INVALID_ARG;
+  }
+  if (L->n_sal > 0) {
+    if (!L->sal_idx || !L->sal_q || !L->sal_scale || !aligned16(L->sal_q)) return BISCO_ERR_INVALID_ARG;
+    if (L->sal_stride < L->n_sal || (L->sal_stride % 16) != 0) return BISCO_ERR_INVALID_ARG;
+  }
+  return BISCO_OK;
+}
+
+int batch_block(int Mc) { return Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8; }
+
+struct Layout {
+  Plan pz, py;
+  bool has_z;
+  size_t off_z, off_cz, off_cy, off_pz, off_py, total;
+};
+
+// Units (quads) of pass Y: one per 128 columns of each base, plus the U^T segment;
+// a layer with neither gets one empty unit so the salient term still has a home.
+int units_y(const bisco_layer* L) {
+  int u = L->num_bases * quads(L->in) + (L->rank > 0 ? quads(L->rank) : 0);
+  return u > 0 ? u : 1;
+}
+
+Layout layout_for(const bisco_layer* L, int MB, int dev) {
+  Layout lo{};
+  const int sms = cached_sms(dev);
+  const size_t lim = cached_smem_limit(dev);
+  lo.has_z = L->rank > 0;
+  lo.py = make_plan(L->out, units_y(L), MB, L->n_sal, sms, lim);
+  if (lo.has_z) lo.pz = make_plan(L->rank, quads(L->in), MB, 0, sms, lim);
+  size_t off = kStatusBytes;
+  lo.off_z = off;
+  off += align256(lo.has_z ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
+  lo.off_cz = off;
+  off += align256(lo.has_z ? lo.pz.cnt_ints * 4 : 0);
+  lo.off_cy = off;
+  off += align256(lo.py.cnt_ints * 4);
+  lo.off_pz = off;
+  off += align256(lo.has_z ? lo.pz.part_floats * 4 : 0);
+  lo.off_py = off;
+  off += align256(lo.py.part_floats * 4);
+  lo.total = off;
+  return lo;
+}
+
+// Largest workspace any batch chunk of this call needs.
+size_t ws_need(const bisco_layer* L, int32_t M, int dev) {
+  size_t need = 0;
+  const int full = std::min<int>(M, kMaxBatchChunk);
+  need = std::max(need, layout_for(L, batch_block(full), dev).total);
+  const int tail = M % kMaxBatchChunk;
+  if (M > kMaxBatchChunk && tail) need = std::max(need, layout_for(L, batch_block(tail), dev).total);
+  return need;
+}
+
+bool plans_fit(const Layout& lo, size_t lim) {
+  return lo.py.smem <= lim && (!lo.has_z || lo.pz.smem <= lim);
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t bisco_packed_words(int64_t rows, int64_t cols) {
+  if (rows <= 0 || cols <= 0) return 0;
+  return ((rows + 31) / 32) * ((cols + 127) / 128) * 128;
+}
+
+bisco_status bisco_pack(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* packed) {
+  if (!signs || !packed || rows <= 0 || cols <= 0) return BISCO_ERR_INVALID_ARG;
+  const int64_t n = rows * cols;
+  for (int64_t i = 0; i < n; ++i)
+    if (signs[i] != 1 && signs[i] != -1) return BISCO_ERR_INVALID_ARG;
+  const int64_t Q = (cols + 127) / 128;
+  std::memset(packed, 0, static_cast<size_t>(bisco_packed_words(rows, cols)) * 4);
+  for (int64_t i = 0; i < rows; ++i) {
+    const int64_t t = i / 32, r = i % 32;
+    const int8_t* row = signs + i * cols;
+    for (int64_t c = 0; c < cols; ++c) {
+      if (row[c] == 1) {
+        const int64_t q = c / 128, j = (c % 128) / 32, b = c % 32;
+        packed[((t * Q + q) * 32 + r) * 4 + j] |= (1u << b);
+      }
+    }
+  }
+  return BISCO_OK;
+}
+
+bisco_status bisco_unpack(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* signs) {
+  if (!signs || !packed || rows <= 0 || cols <= 0) return BISCO_ERR_INVALID_ARG;
+  const int64_t Q = (cols + 127) / 128;
+  for (int64_t i = 0; i < rows; ++i) {
+    const int64_t t = i / 32, r = i % 32;
+    for (int64_t c = 0; c < cols; ++c) {
+      const int64_t q = c / 128, j = (c % 128) / 32, b = c % 32;
+      const uint32_t w = packed[((t * Q + q) * 32 + r) * 4 + j];
+      signs[i * cols + c] = ((w >> b) & 1u) ? 1 : -1;
+    }
+  }
+  return BISCO_OK;
+}
+
+bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* bytes) {
+  if (!bytes || M < 1) return BISCO_ERR_INVALID_ARG;
+  const bisco_status st = validate_layer(layer);
+  if (st != BISCO_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
+  *bytes = ws_need(layer, M, dev);
+  return BISCO_OK;
+}
+
+bisco_status bisco_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < static_cast<size_t>(kStatusBytes) || !aligned16(ws)) return BISCO_ERR_INVALID_ARG;
+  return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? BISCO_OK
+                                                                                               : BISCO_ERR_CUDA;
+}
+
+bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, int32_t M, void* Y,
+                        int32_t y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  bisco_status st = validate_layer(L);
+  if (st != BISCO_OK) return st;
+  if (M < 0 || !dtype_ok(x_dtype) || !dtype_ok(y_dtype)) return BISCO_ERR_INVALID_ARG;
+  if (M == 0) return BISCO_OK;
+  if (!X || !Y || !aligned16(X) || !aligned16(Y)) return BISCO_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return BISCO_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
+  if (ws_bytes < ws_need(L, M, dev)) return BISCO_ERR_WORKSPACE;
+  const size_t lim = cached_smem_limit(dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  const size_t xb = dtype_bytes(x_dtype), yb = dtype_bytes(y_dtype);
+
+  // Every launch is planned before the first one is issued, so an unsupported
+  // request fails without touching any output.
+  std::vector<Layout> los;
+  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
+    const int Mc = std::min(kMaxBatchChunk, M - m0);
+    los.push_back(layout_for(L, batch_block(Mc), dev));
+    if (!plans_fit(los.back(), lim)) return BISCO_ERR_UNSUPPORTED;
+  }
+
+  int chunk = 0;
+  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk, ++chunk) {
+    const int Mc = std::min(kMaxBatchChunk, M - m0);
+    const Layout& lo = los[chunk];
+    int* status = reinterpret_cast<int*>(wsb);
+    float* zbuf = reinterpret_cast<float*>(wsb + lo.off_z);
+    const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(m0) * L->in * xb;
+    void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(m0) * L->out * yb;
+
+    if (lo.has_z) {
+      PassParam pz{};
+      pz.nseg = 1;
+      SegParam& V = pz.seg[0];
+      V.bits = reinterpret_cast<const uint4*>(L->v_bits);
+      V.nq = quads(L->in);
+      V.ncols = L->in;
+      V.unit0 = 0;
+      V.xsrc = 0;
+      V.cscale = nullptr;
+      V.cdt = BISCO_F32;
+      V.rscale = L->alpha;
+      V.rdt = BISCO_F32;
+      pz.rows = L->rank;
+      pz.tiles = (L->rank + 31) / 32;
+      pz.units = V.nq;
+      pz.G = lo.pz.G; pz.nblocks = lo.pz.nblocks; pz.L = lo.pz.L; pz.P = lo.pz.P;
+      pz.Mc = Mc; pz.max_cols = lo.pz.max_cols; pz.col_stride_bytes = lo.pz.col_stride_bytes;
+      pz.X = Xc; pz.xdt = x_dtype; pz.ldx = L->in; pz.xcols = L->in;
+      pz.Z = nullptr; pz.ldz = 0;
+      pz.Y = zbuf; pz.ydt = BISCO_F32; pz.ldy = L->rank;
+      pz.n_sal = 0; pz.sal_stride = 0;
+      pz.part = reinterpret_cast<float*>(wsb + lo.off_pz);
+      pz.cnt = reinterpret_cast<int*>(wsb + lo.off_cz);
+      pz.status = status;
+      if (launch_pass(pz, lo.pz, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
+    }
+
+    PassParam py{};
+    int nseg = 0, unit = 0;
+    for (int k = 0; k < L->num_bases; ++k) {
+      SegParam& B = py.seg[nseg++];
+      B.bits = reinterpret_cast<const uint4*>(L->bits + static_cast<size_t>(k) * bisco_packed_words(L->out, L->in));
+      B.nq = quads(L->in);
+      B.ncols = L->in;
+      B.unit0 = unit;
+      unit += B.nq;
+      B.xsrc = 0;
+      B.cscale = static_cast<const unsigned char*>(L->col_scale) + static_cast<size_t>(k) * L->in * dtype_bytes(L->scale_dtype);
+      B.cdt = L->scale_dtype;
+      B.rscale = static_cast<const unsigned char*>(L->row_scale) + static_cast<size_t>(k) * L->out * dtype_bytes(L->scale_dtype);
+      B.rdt = L->scale_dtype;
+    }
+    if (L->rank > 0) {
+      SegParam& U = py.seg[nseg++];
+      U.bits = reinterpret_cast<const uint4*>(L->ut_bits);
+      U.nq = quads(L->rank);
+      U.ncols = L->rank;
+      U.unit0 = unit;
+      unit += U.nq;
+      U.xsrc = 1;
+      U.cscale = nullptr;
+      U.cdt = BISCO_F32;
+      U.rscale = nullptr;
+      U.rdt = BISCO_F32;
+    }
+    if (nseg == 0) {  // salient-only (or empty) layer: one empty unit
+      SegParam& E = py.seg[nseg++];
+      E.bits = nullptr; E.nq = 1; E.ncols = 0; E.unit0 = 0; E.xsrc = 2;
+      E.cscale = nullptr; E.rscale = nullptr; E.cdt = E.rdt = BISCO_F32;
+      unit = 1;
+    }
+    py.nseg = nseg;
+    py.rows = L->out;
+    py.tiles = (L->out + 31) / 32;
+    py.units = unit;
+    py.G = lo.py.G; py.nblocks = lo.py.nblocks; py.L = lo.py.L; py.P = lo.py.P;
+    py.Mc = Mc; py.max_cols = lo.py.max_cols; py.col_stride_bytes = lo.py.col_stride_bytes;
+    py.X = Xc; py.xdt = x_dtype; py.ldx = L->in; py.xcols = L->in;
+    py.Z = zbuf; py.ldz = L->rank;
+    py.Y = Yc; py.ydt = y_dtype; py.ldy = L->out;
+    py.n_sal = L->n_sal; py.sal_stride = L->sal_stride;
+    py.sal_idx = L->sal_idx; py.sal_q = L->sal_q; py.sal_scale = L->sal_scale;
+    py.part = reinterpret_cast<float*>(wsb + lo.off_py);
+    py.cnt = reinterpret_cast<int*>(wsb + lo.off_cy);
+    py.status = status;
+    if (launch_pass(py, lo.py, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
+  }
+  return BISCO_OK;
+}
+
+bisco_status bisco_sync_status(void* stream, const void* ws) {
+  if (!ws) return BISCO_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BISCO_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return BISCO_ERR_CUDA;
+  return static_cast<bisco_status>(code);
+}
+
+bisco_status bisco_bench(const bisco_bench_args* a, bisco_bench_result* r) {
+  if (!a || !r || !a->layers || a->n_layers < 1 || a->M < 1 || a->reps < 1 || a->warmup < 0)
+    return BISCO_ERR_INVALID_ARG;
+  for (int i = 0; i < a->n_layers; ++i) {
+    const bisco_status st = validate_layer(&a->layers[i]);
+    if (st != BISCO_OK) return st;
+  }
+  if (!a->X || !a->Y || !a->ws || !dtype_ok(a->x_dtype) || !dtype_ok(a->y_dtype)) return BISCO_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
+  for (int i = 0; i < a->n_layers; ++i)
+    if (a->ws_bytes < ws_need(&a->layers[i], a->M, dev)) return BISCO_ERR_WORKSPACE;
+
+  if (ensure_kernel_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
+  cudaStream_t user = static_cast<cudaStream_t>(a->stream);
+  cudaStream_t cs = nullptr;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  cudaEvent_t e0 = nullptr, e1 = nullptr, join = nullptr;
+  bisco_status result = BISCO_OK;
+  const size_t yb = dtype_bytes(a->y_dtype);
+  auto fail = [&](bisco_status st) { if (result == BISCO_OK) result = st; };
+
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return BISCO_ERR_CUDA;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess ||
+      cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess)
+    fail(BISCO_ERR_CUDA);
+  if (result == BISCO_OK && (cudaEventRecord(join, user) != cudaSuccess || cudaStreamWaitEvent(cs, join, 0) != cudaSuccess))
+    fail(BISCO_ERR_CUDA);
+  if (result == BISCO_OK) {
+    if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+      fail(BISCO_ERR_CUDA);
+    } else {
+      size_t yoff = 0;
+      for (int i = 0; i < a->n_layers && result == BISCO_OK; ++i) {
+        const bisco_layer& L = a->layers[i];
+        const bisco_status st = bisco_gemv(&L, a->X, a->x_dtype, a->M, static_cast<unsigned char*>(a->Y) + yoff,
+                                           a->y_dtype, a->ws, a->ws_bytes, cs);
+        if (st != BISCO_OK) fail(st);
+        yoff += static_cast<size_t>(a->M) * L.out * yb;
+      }
+      if (cudaStreamEndCapture(cs, &graph) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    }
+  }
+  if (result == BISCO_OK && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) fail(BISCO_ERR_CUDA);
+  if (result == BISCO_OK) {
+    for (int i = 0; i < a->warmup && result == BISCO_OK; ++i)
+      if (cudaGraphLaunch(exec, cs) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    if (cudaEventRecord(e0, cs) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    for (int i = 0; i < a->reps && result == BISCO_OK; ++i)
+      if (cudaGraphLaunch(exec, cs) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    if (cudaEventRecord(e1, cs) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    if (cudaEventSynchronize(e1) != cudaSuccess) fail(BISCO_ERR_CUDA);
+    float ms = 0.f;
+    if (result == BISCO_OK && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess) {
+      r->us_per_replay = ms * 1000.0 / a->reps;
+      r->us_per_gemv = r->us_per_replay / a->n_layers;
+      const int chunks = (a->M + kMaxBatchChunk - 1) / kMaxBatchChunk;
+      r->kernels_per_gemv = chunks * (a->layers[0].rank > 0 ? 2 : 1);
+    } else {
+      fail(BISCO_ERR_CUDA);
+    }
+  }
+  if (exec) cudaGraphExecDestroy(exec);
+  if (graph) cudaGraphDestroy(graph);
+  if (join && cudaEventRecord(join, cs) == cudaSuccess) cudaStreamWaitEvent(user, join, 0);
+  if (cs) cudaStreamSynchronize(cs);
+  if (cs) cudaStreamDestroy(cs);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  if (join) cudaEventDestroy(join);
+  return result;
+}
+
+const char* bisco_status_string(bisco_status st) {
+  switch (st) {
+    case BISCO_OK: return "BISCO_OK";
+    case BISCO_ERR_INVALID_ARG: return "BISCO_ERR_INVALID_ARG";
+    case BISCO_ERR_UNSUPPORTED: return "BISCO_ERR_UNSUPPORTED";
+    case BISCO_ERR_CUDA: return "BISCO_ERR_CUDA";
+    case BISCO_ERR_TIMEOUT: return "BISCO_ERR_TIMEOUT";
+    case BISCO_ERR_WORKSPACE: return "BISCO_ERR_WORKSPACE";
+  }
+  return "BISCO_UNKNOWN_STATUS";
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+/*
+ * bisco.h -- C ABI of the binary-weight decode GEMV library (libbisco.so).
+ *
+ * The library computes the decode-time product Y = X * W^T for a weight that is
+ * stored as a sum of bit-packed sign matrices with decoupled row and column
+ * scales, plus an optional binary low-rank correction and an optional set of
+ * salient input columns kept in int8:
+ *
+ *   W[o][i] = sum_k r_k[o] * c_k[i] * B_k[o][i]                       (1)
+ *           + sum_j alpha_j * U[o][j] * V[j][i]                        (2)
+ *           + sum_t [i == idx_t] * s_t * q[o][t]                       (3)
+ *
+ *   (1) "FluxBin: Flexible LUT-based Ultra-low-bit LLM Inference by
+ *       Algorithm-Kernel Synergy", Sec. 3.1, decoupled row-column binary bases;
+ *       a stored bit b means the sign (2b - 1) (Sec. 3.2, Stage 1).
+ *   (2) "BiLoCo: Binary Low-Rank Corrections for Post-Training Quantization",
+ *       section "The core idea": U, V in {+1,-1}; applied as alpha * u * (v . x).
+ *   (3) "BiSCo-LLM" (gist.science summary), Methodology 3, Sensitivity
+ *       Protection: a ~1% set of channels in 8 bits; FluxBin Sec. 3.2, Virtual
+ *       Columnar Mapping: a dense block plus an index list gathered at run time.
+ *
+ * Conventions for every entry point:
+ *  - Host entry points (bisco_pack, bisco_unpack, sizes, strings) take host
+ *    pointers. bisco_gemv, bisco_workspace_init and bisco_bench take device
+ *    pointers and a CUDA stream (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream).
+ *  - The caller owns all memory. bisco_gemv allocates nothing; scratch space is
+ *    the caller's workspace buffer.
+ *  - Arguments are validated before anything is launched or written: a
+ *    validation failure returns BISCO_ERR_INVALID_ARG (or BISCO_ERR_WORKSPACE)
+ *    and leaves every output untouched. A CUDA launch failure returns
+ *    BISCO_ERR_CUDA. Device-side errors are recorded in the workspace status
+ *    word and read back with bisco_sync_status.
+ *  - Packed bit buffers, X, Y and the workspace must be 16-byte aligned.
+ *  - Calls are thread-safe; calls that share a workspace must be ordered on one
+ *    stream (two calls in flight on one workspace race).
+ */
+#ifndef BISCO_H
+#define BISCO_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BISCO_OK = 0,
+  BISCO_ERR_INVALID_ARG = 1,  /* bad pointer, size, dtype, index or alignment */
+  BISCO_ERR_UNSUPPORTED = 2,  /* valid request this build cannot run          */
+  BISCO_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed         */
+  BISCO_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up           */
+  BISCO_ERR_WORKSPACE = 5     /* workspace missing or too small               */
+} bisco_status;
+
+typedef enum { BISCO_F32 = 0, BISCO_BF16 = 1 } bisco_dtype;
+
+/*
+ * Packed sign-matrix layout (all bit matrices: B_k, V and U^T).
+ *
+ * A rows x cols matrix of signs is stored in row tiles of 32 rows and column
+ * quads of 128 columns: uint32 words [tiles][quads][32][4] with
+ * tiles = ceil(rows/32) and quads = ceil(cols/128). Entry (32t + r, 128q + 32j + b)
+ * is bit b of word [t][q][r][j]; bit 1 means +1 and bit 0 means -1. Padding
+ * entries (row >= rows or col >= cols) hold bit 0. With this layout the 32 lanes
+ * of a warp, one row each, read a (tile, quad) block as 512 contiguous bytes.
+ */
+
+/* Number of uint32 words of one packed rows x cols sign matrix (0 if either is <= 0). */
+int64_t bisco_packed_words(int64_t rows, int64_t cols);
+
+/*
+ * Pack a dense row-major int8 matrix of +1/-1 into the layout above.
+ * signs: host, rows*cols int8, each exactly +1 or -1.
+ * packed: host, bisco_packed_words(rows, cols) words, written in full (padding = 0).
+ * Returns BISCO_ERR_INVALID_ARG for null pointers, rows or cols <= 0, or any entry
+ * other than +1/-1; in that case nothing is written.
+ */
+bisco_status bisco_pack(const int8_t* signs, int64_t rows, int64_t cols, uint32_t* packed);
+
+/*
+ * Inverse of bisco_pack: signs (host, rows*cols int8) receives +1/-1.
+ * Padding bits are ignored. BISCO_ERR_INVALID_ARG for null pointers or sizes <= 0.
+ */
+bisco_status bisco_unpack(const uint32_t* packed, int64_t rows, int64_t cols, int8_t* signs);
+
+/* One layer. All pointers are device pointers owned by the caller. */
+typedef struct {
+  int32_t out;              /* output features (rows of W), >= 1                      */
+  int32_t in;               /* input features (columns of W), >= 1                    */
+  int32_t num_bases;        /* K >= 0 binary bases                                    */
+  const uint32_t* bits;     /* [K][bisco_packed_words(out, in)] sign matrices B_k     */
+  const void* row_scale;    /* [K][out] r_k, dtype scale_dtype                        */
+  const void* col_scale;    /* [K][in]  c_k, dtype scale_dtype                        */
+  int32_t scale_dtype;      /* BISCO_F32 or BISCO_BF16                                */
+  int32_t rank;             /* R >= 0; 0 = no low-rank correction                     */
+  const uint32_t* v_bits;   /* [bisco_packed_words(R, in)]  V, row j = v_j            */
+  const uint32_t* ut_bits;  /* [bisco_packed_words(out, R)] U^T: entry (o, j) = u_j[o] */
+  const float* alpha;       /* [R] coefficients alpha_j                               */
+  int32_t n_sal;            /* n_s >= 0 salient input columns; 0 = none               */
+  int32_t sal_stride;       /* bytes per row of sal_q: multiple of 16, >= n_sal       */
+  const int32_t* sal_idx;   /* [n_s] strictly ascending column indices in [0, in)     */
+  const int8_t* sal_q;      /* [out][sal_stride] int8 values q[o][t]                  */
+  const float* sal_scale;   /* [n_s] per-column scales s_t                            */
+} bisco_layer;
+
+/*
+ * Bytes of workspace bisco_gemv needs for this layer and batch M (>= 1).
+ * BISCO_ERR_INVALID_ARG for a null pointer or a layer whose sizes are invalid.
+ */
+bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* bytes);
+
+/*
+ * Prepare a workspace for first use: zero-fills ws_bytes bytes on `stream`.
+ * Every bisco_gemv call leaves the workspace ready for the next call, so this is
+ * needed once per buffer (and again after a call reported an error).
+ */
+bisco_status bisco_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Y = X * W^T with W as in (1)-(3) above; asynchronous on `stream`.
+ *  X:  device, [M][in] row-major, x_dtype (BISCO_BF16 or BISCO_F32).
+ *  Y:  device, [M][out] row-major, y_dtype; fully overwritten.
+ *  M:  batch rows; M == 0 is a no-op that returns BISCO_OK.
+ *  ws: device workspace of at least bisco_workspace_size bytes, prepared once by
+ *      bisco_workspace_init.
+ * The sign-times-activation sums use fp32 accumulation. Results are deterministic:
+ * the reduction order is fixed, so repeated calls give bit-identical Y.
+ * Kernels are launched with programmatic dependent launch: they prefetch weights
+ * while the previous kernel on the stream finishes, and read X only after it
+ * has completed. The calls can be captured in a CUDA graph.
+ */
+bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype, int32_t M,
+                        void* Y, int32_t y_dtype, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronise `stream` and return the device-side status recorded in workspace
+ * `ws` by earlier bisco_gemv calls (BISCO_OK if none). A recorded error stays
+ * until bisco_workspace_init clears it.
+ */
+bisco_status bisco_sync_status(void* stream, const void* ws);
+
+/* Benchmark request: a stream of n_layers GEMVs (distinct weight copies) captured
+ * in one CUDA graph and replayed. */
+typedef struct {
+  const bisco_layer* layers;  /* host array of n_layers layer descriptors (device data) */
+  int32_t n_layers;
+  const void* X;              /* device [M][in] shared by all layers                     */
+  int32_t x_dtype;
+  int32_t M;
+  void* Y;                    /* device [n_layers][M][out]                               */
+  int32_t y_dtype;
+  void* ws;                   /* device workspace, >= max over layers of the size        */
+  size_t ws_bytes;
+  int32_t warmup;             /* untimed graph replays                                   */
+  int32_t reps;               /* timed graph replays                                     */
+  void* stream;
+} bisco_bench_args;
+
+typedef struct {
+  double us_per_gemv;         /* mean device time per GEMV over the timed replays  */
+  double us_per_replay;       /* mean device time of one replay of the whole graph */
+  int32_t kernels_per_gemv;   /* kernel launches per GEMV                         */
+} bisco_bench_result;
+
+/*
+ * Time the GEMV stream with CUDA events on args->stream (warm-up replays are not
+ * timed). Returns BISCO_ERR_INVALID_ARG for bad arguments, BISCO_ERR_CUDA on a
+ * CUDA failure; the graph is released before returning.
+ */
+bisco_status bisco_bench(const bisco_bench_args* args, bisco_bench_result* result);
+
+/* Static string naming a status code. */
+const char* bisco_status_string(bisco_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BISCO_H */

@@ -17,4 +17,5 @@ from .bisco_oracle import (  # noqa: F401
     pack_bit_matrix,
     reconstruct,
     unpack_bit_matrix,
+    unpack_bit_rows,
 )

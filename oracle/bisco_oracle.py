@@ -68,6 +68,20 @@ def unpack_bit_matrix(words, rows, cols):
     return out
 
 
+def unpack_bit_rows(words, rows, cols, row_idx):
+    """Signs of the selected rows only, int8 [len(row_idx), cols]; decodes just their tiles."""
+    row_idx = np.asarray(row_idx, dtype=np.int64)
+    T, Q = _grid(rows, cols)
+    w = np.asarray(words, dtype=np.uint32).reshape(T, Q, TILE_ROWS, 4)
+    shifts = np.arange(32, dtype=np.uint32)
+    out = np.empty((len(row_idx), cols), dtype=np.int8)
+    for n, i in enumerate(row_idx):
+        t, r = divmod(int(i), TILE_ROWS)
+        bits = ((w[t, :, r, :][..., None] >> shifts) & 1).astype(np.int8)   # [q][j][b]
+        out[n] = bits.reshape(Q * QUAD_COLS)[:cols] * 2 - 1
+    return out
+
+
 def pack_bit_matrix(signs):
     """int8 matrix of +1/-1 -> packed words (+1 -> bit 1). Rejects other values."""
     s = np.asarray(signs)
@@ -113,7 +127,7 @@ def _binary_part_rows(layer, rows):
     C = decode_values(layer.col_scale, layer.scale_dtype).reshape(layer.K, layer.in_)
     bits = np.asarray(layer.bits).reshape(layer.K, -1)
     for k in range(layer.K):
-        S = unpack_bit_matrix(bits[k], layer.out, layer.in_)[rows]
+        S = unpack_bit_rows(bits[k], layer.out, layer.in_, rows)
         W += R[k, rows][:, None] * S * C[k][None, :]
     return W
 
@@ -122,10 +136,10 @@ def _correction_part_rows(layer, rows):
     """sum_j alpha_j u_j v_j^T restricted to output rows `rows`."""
     if not layer.rank:
         return 0.0
-    V = unpack_bit_matrix(layer.v_bits, layer.rank, layer.in_).astype(np.float64)   # [R, in]
-    U = unpack_bit_matrix(layer.ut_bits, layer.out, layer.rank).astype(np.float64)  # [out, R]
+    V = unpack_bit_matrix(layer.v_bits, layer.rank, layer.in_).astype(np.float64)        # [R, in]
+    U = unpack_bit_rows(layer.ut_bits, layer.out, layer.rank, rows).astype(np.float64)  # [rows, R]
     a = np.asarray(layer.alpha, dtype=np.float32).astype(np.float64)
-    return (U[rows] * a[None, :]) @ V
+    return (U * a[None, :]) @ V
 
 
 def _salient_part_rows(layer, rows):

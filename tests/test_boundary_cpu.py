@@ -1,0 +1,80 @@
+"""The C ABI library on the host: it loads, exports every declared entry point,
+packs bit-exactly like the oracle's packer, and rejects bad arguments.
+No GPU is needed; no device computation is called."""
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import binary_weight_decode_b200 as bw
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "bisco.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bisco_[a-z_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_entry_points()
+    assert "bisco_gemv" in names and "bisco_pack" in names and "bisco_bench" in names
+    for n in names:
+        assert hasattr(bw._lib, n), f"libbisco.so does not export {n}"
+    assert sorted(bw.EXPORTED) == names
+
+
+def test_packed_words():
+    assert bw.bisco_packed_words(4096, 4096) == 4096 * 4096 // 32
+    assert bw.bisco_packed_words(33, 129) == 512
+    assert bw.bisco_packed_words(0, 5) == 0
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 1), (5, 7), (32, 128), (33, 129), (100, 1000), (257, 4096)])
+def test_pack_matches_oracle_bit_exact(rows, cols):
+    S = np.random.default_rng(rows * 7 + cols).choice(np.array([-1, 1], np.int8), size=(rows, cols))
+    w = bw.bisco_pack(S)
+    assert np.array_equal(w, oracle.pack_bit_matrix(S))
+    assert np.array_equal(bw.bisco_unpack(w, rows, cols), S)
+    assert np.array_equal(oracle.unpack_bit_matrix(w, rows, cols), S)
+
+
+def test_pack_single_bits():
+    for (i, c) in [(0, 0), (31, 127), (32, 128), (40, 300), (40, 31), (40, 32)]:
+        S = -np.ones((41, 301), np.int8)
+        S[i, c] = 1
+        w = bw.bisco_pack(S)
+        assert sum(bin(int(x)).count("1") for x in w) == 1
+        U = oracle.unpack_bit_matrix(w, 41, 301)
+        assert U[i, c] == 1 and (U == 1).sum() == 1
+
+
+def test_pack_rejects_non_signs_and_writes_nothing():
+    bad = np.ones((3, 40), np.int8)
+    bad[2, 39] = 0
+    out = np.full(bw.bisco_packed_words(3, 40), 0xDEADBEEF, np.uint32)
+    st = bw._lib.bisco_pack(bad.ctypes.data, 3, 40, out.ctypes.data)
+    assert st == bw.BISCO_ERR_INVALID_ARG
+    assert np.all(out == 0xDEADBEEF)
+    assert bw._lib.bisco_pack(None, 3, 40, out.ctypes.data) == bw.BISCO_ERR_INVALID_ARG
+    assert bw._lib.bisco_pack(bad.ctypes.data, 0, 40, out.ctypes.data) == bw.BISCO_ERR_INVALID_ARG
+
+
+def test_gemv_rejects_bad_arguments_before_touching_the_device():
+    L = bw.bisco_layer(out=0, in_=10, num_bases=0)
+    assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    L = bw.bisco_layer(out=10, in_=10, num_bases=5)
+    assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    L = bw.bisco_layer(out=10, in_=10, num_bases=1)          # null bits
+    assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    L = bw.bisco_layer(out=10, in_=10, num_bases=0, n_sal=3, sal_stride=8)
+    assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    L = bw.bisco_layer(out=10, in_=10, num_bases=0)
+    assert bw._lib.bisco_gemv(L, None, 7, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG   # dtype
+    assert bw._lib.bisco_gemv(L, None, 0, -1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG  # M < 0
+    assert bw._lib.bisco_gemv(L, None, 0, 0, None, 0, None, 0, None) == bw.BISCO_OK                # M == 0
+    assert bw.bisco_status_string(bw.BISCO_ERR_WORKSPACE) == "BISCO_ERR_WORKSPACE"

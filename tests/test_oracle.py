@@ -328,3 +328,11 @@ def test_algorithmic_bytes_counts_each_payload():
     L.rank = 512
     extra = 512 * (4096 + 4096) // 8 + 4 * 512
     assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 4_243_456 + extra
+
+
+@pytest.mark.parametrize("rows,cols", [(70, 300), (33, 129), (1, 5)])
+def test_row_decoder_matches_independent_packer(rows, cols):
+    S = np.random.default_rng(7 * rows + cols).choice(np.array([-1, 1], np.int8), size=(rows, cols))
+    w = py_pack(S.tolist())
+    sel = sorted({0, rows - 1, rows // 2, min(31, rows - 1), min(32, rows - 1)})
+    assert np.array_equal(oracle.unpack_bit_rows(w, rows, cols, sel), S[sel])
