@@ -189,6 +189,8 @@ def main():
     ap.add_argument("--workload", default="attn4096", choices=sorted(WORKLOADS))
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--calls", type=int, default=0,
+                    help="profiling case: run this many plain bisco_gemv calls on one weight copy and exit")
     args = ap.parse_args()
     cfg, spec, m_default, desc = WORKLOADS[args.workload]
     args.M = args.M or m_default
@@ -212,6 +214,19 @@ def main():
     M = args.M
     L, X = build(cfg, spec, M)
     xdt = "f32" if cfg == 1 else "bf16"
+    if args.calls:  # small case for ncu captures: no graph, no timing
+        dl = bw.DeviceLayer(L)
+        Xd = torch.from_numpy(X.view(np.int16) if xdt == "bf16" else X).cuda()
+        Xd = Xd.view(torch.bfloat16) if xdt == "bf16" else Xd
+        Yd = torch.empty((M, L.out), dtype=torch.bfloat16, device="cuda")
+        ws = bw.alloc_workspace([dl], M)
+        for _ in range(args.calls):
+            bw.bisco_gemv(dl, Xd, Yd, ws)
+            torch.cuda.synchronize()
+        st = bw.bisco_sync_status(ws)
+        if st != bw.BISCO_OK:
+            raise SystemExit(f"device status {bw.bisco_status_string(st)}")
+        return
     x_bytes = 4 if xdt == "f32" else 2
     y_dtype = torch.bfloat16
     nbytes = algorithmic_bytes(L, M, x_bytes, 2)

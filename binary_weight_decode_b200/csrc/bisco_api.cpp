@@ -63,53 +63,76 @@ bisco_status validate_layer(const bisco_layer* L) {
 
 int batch_block(int Mc) { return Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8; }
 
+// Segment list of pass Y: K binary bases, then U^T if the layer has a correction;
+// a layer with neither gets one empty unit so the salient term still has a home.
+struct SegList {
+  int unit0[kMaxSeg];
+  int nseg, units;
+};
+
+SegList segs_y(const bisco_layer* L) {
+  SegList s{};
+  for (int k = 0; k < L->num_bases; ++k) { s.unit0[s.nseg++] = s.units; s.units += quads(L->in); }
+  if (L->rank > 0) { s.unit0[s.nseg++] = s.units; s.units += quads(L->rank); }
+  if (s.nseg == 0) { s.unit0[s.nseg++] = 0; s.units = 1; }
+  return s;
+}
+
 struct Layout {
   Plan pz, py;
   bool has_z;
-  size_t off_z, off_cz, off_cy, off_pz, off_py, total;
+  size_t off_z, total;
 };
-
-// Units (quads) of pass Y: one per 128 columns of each base, plus the U^T segment;
-// a layer with neither gets one empty unit so the salient term still has a home.
-int units_y(const bisco_layer* L) {
-  int u = L->num_bases * quads(L->in) + (L->rank > 0 ? quads(L->rank) : 0);
-  return u > 0 ? u : 1;
-}
 
 Layout layout_for(const bisco_layer* L, int MB, int dev) {
   Layout lo{};
   const int sms = cached_sms(dev);
   const size_t lim = cached_smem_limit(dev);
   lo.has_z = L->rank > 0;
-  lo.py = make_plan(L->out, units_y(L), MB, L->n_sal, sms, lim);
-  if (lo.has_z) lo.pz = make_plan(L->rank, quads(L->in), MB, 0, sms, lim);
-  size_t off = kStatusBytes;
-  lo.off_z = off;
-  off += align256(lo.has_z ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
-  lo.off_cz = off;
-  off += align256(lo.has_z ? lo.pz.cnt_ints * 4 : 0);
-  lo.off_cy = off;
-  off += align256(lo.py.cnt_ints * 4);
-  lo.off_pz = off;
-  off += align256(lo.has_z ? lo.pz.part_floats * 4 : 0);
-  lo.off_py = off;
-  off += align256(lo.py.part_floats * 4);
-  lo.total = off;
+  const SegList sy = segs_y(L);
+  lo.py = make_plan(L->out, sy.units, sy.unit0, sy.nseg, MB, L->n_sal, sms, lim);
+  if (lo.has_z) {
+    const int z0 = 0;
+    lo.pz = make_plan(L->rank, quads(L->in), &z0, 1, MB, 0, sms, lim);
+  }
+  lo.off_z = kStatusBytes;
+  lo.total = lo.off_z + align256(lo.has_z ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
   return lo;
 }
 
-// Largest workspace any batch chunk of this call needs.
-size_t ws_need(const bisco_layer* L, int32_t M, int dev) {
-  size_t need = 0;
-  const int full = std::min<int>(M, kMaxBatchChunk);
-  need = std::max(need, layout_for(L, batch_block(full), dev).total);
-  const int tail = M % kMaxBatchChunk;
-  if (M > kMaxBatchChunk && tail) need = std::max(need, layout_for(L, batch_block(tail), dev).total);
-  return need;
+// Plans depend only on shapes and the device: cache them so that a call does not
+// re-run the occupancy queries.
+Layout cached_layout(const bisco_layer* L, int MB, int dev) {
+  struct Key {
+    int dev, out, in, K, rank, n_sal, MB;
+    bool operator==(const Key& o) const {
+      return dev == o.dev && out == o.out && in == o.in && K == o.K && rank == o.rank && n_sal == o.n_sal && MB == o.MB;
+    }
+  };
+  struct Entry { Key k; Layout lo; };
+  static std::mutex mu;
+  static std::vector<Entry>* cache = new std::vector<Entry>();
+  const Key k{dev, L->out, L->in, L->num_bases, L->rank, L->n_sal, MB};
+  std::lock_guard<std::mutex> g(mu);
+  for (const Entry& e : *cache)
+    if (e.k == k) return e.lo;
+  if (cache->size() > 4096) cache->clear();
+  cache->push_back(Entry{k, layout_for(L, MB, dev)});
+  return cache->back().lo;
+}
+
+// Workspace bytes: the status word and, with a correction, z for one batch chunk.
+size_t ws_need(const bisco_layer* L, int32_t) {
+  return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
 }
 
 bool plans_fit(const Layout& lo, size_t lim) {
   return lo.py.smem <= lim && (!lo.has_z || lo.pz.smem <= lim);
+}
+
+void fill_plan(PassParam& P, const Plan& pl) {
+  P.C = pl.C; P.ncl = pl.ncl; P.max_tiles = pl.max_tiles; P.max_units = pl.max_units;
+  P.max_lseg = pl.max_lseg; P.col_stride_bytes = pl.col_stride_bytes;
 }
 
 }  // namespace
@@ -161,7 +184,8 @@ bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* b
   if (st != BISCO_OK) return st;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
-  *bytes = ws_need(layer, M, dev);
+  (void)dev;
+  *bytes = ws_need(layer, M);
   return BISCO_OK;
 }
 
@@ -181,7 +205,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
   if (!ws || !aligned16(ws)) return BISCO_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
-  if (ws_bytes < ws_need(L, M, dev)) return BISCO_ERR_WORKSPACE;
+  if (ws_bytes < ws_need(L, M)) return BISCO_ERR_WORKSPACE;
   const size_t lim = cached_smem_limit(dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* wsb = static_cast<unsigned char*>(ws);
@@ -192,7 +216,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
   std::vector<Layout> los;
   for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
     const int Mc = std::min(kMaxBatchChunk, M - m0);
-    los.push_back(layout_for(L, batch_block(Mc), dev));
+    los.push_back(cached_layout(L, batch_block(Mc), dev));
     if (!plans_fit(los.back(), lim)) return BISCO_ERR_UNSUPPORTED;
   }
 
@@ -218,17 +242,19 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       V.cdt = BISCO_F32;
       V.rscale = L->alpha;
       V.rdt = BISCO_F32;
+      V.cvec = 0;
+      V.rvec = aligned16(L->alpha);
       pz.rows = L->rank;
       pz.tiles = (L->rank + 31) / 32;
       pz.units = V.nq;
-      pz.G = lo.pz.G; pz.nblocks = lo.pz.nblocks; pz.L = lo.pz.L; pz.P = lo.pz.P;
-      pz.Mc = Mc; pz.max_cols = lo.pz.max_cols; pz.col_stride_bytes = lo.pz.col_stride_bytes;
+      fill_plan(pz, lo.pz);
+      pz.Mc = Mc;
       pz.X = Xc; pz.xdt = x_dtype; pz.ldx = L->in; pz.xcols = L->in;
       pz.Z = nullptr; pz.ldz = 0;
+      pz.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
+      pz.z_vec = 0;
       pz.Y = zbuf; pz.ydt = BISCO_F32; pz.ldy = L->rank;
       pz.n_sal = 0; pz.sal_stride = 0;
-      pz.part = reinterpret_cast<float*>(wsb + lo.off_pz);
-      pz.cnt = reinterpret_cast<int*>(wsb + lo.off_cz);
       pz.status = status;
       if (launch_pass(pz, lo.pz, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
     }
@@ -247,6 +273,8 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       B.cdt = L->scale_dtype;
       B.rscale = static_cast<const unsigned char*>(L->row_scale) + static_cast<size_t>(k) * L->out * dtype_bytes(L->scale_dtype);
       B.rdt = L->scale_dtype;
+      B.cvec = aligned16(B.cscale);
+      B.rvec = aligned16(B.rscale);
     }
     if (L->rank > 0) {
       SegParam& U = py.seg[nseg++];
@@ -260,26 +288,28 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       U.cdt = BISCO_F32;
       U.rscale = nullptr;
       U.rdt = BISCO_F32;
+      U.cvec = U.rvec = 0;
     }
     if (nseg == 0) {  // salient-only (or empty) layer: one empty unit
       SegParam& E = py.seg[nseg++];
       E.bits = nullptr; E.nq = 1; E.ncols = 0; E.unit0 = 0; E.xsrc = 2;
       E.cscale = nullptr; E.rscale = nullptr; E.cdt = E.rdt = BISCO_F32;
+      E.cvec = E.rvec = 0;
       unit = 1;
     }
     py.nseg = nseg;
     py.rows = L->out;
     py.tiles = (L->out + 31) / 32;
     py.units = unit;
-    py.G = lo.py.G; py.nblocks = lo.py.nblocks; py.L = lo.py.L; py.P = lo.py.P;
-    py.Mc = Mc; py.max_cols = lo.py.max_cols; py.col_stride_bytes = lo.py.col_stride_bytes;
+    fill_plan(py, lo.py);
+    py.Mc = Mc;
     py.X = Xc; py.xdt = x_dtype; py.ldx = L->in; py.xcols = L->in;
     py.Z = zbuf; py.ldz = L->rank;
+    py.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
+    py.z_vec = (L->rank % 4) == 0;
     py.Y = Yc; py.ydt = y_dtype; py.ldy = L->out;
     py.n_sal = L->n_sal; py.sal_stride = L->sal_stride;
     py.sal_idx = L->sal_idx; py.sal_q = L->sal_q; py.sal_scale = L->sal_scale;
-    py.part = reinterpret_cast<float*>(wsb + lo.off_py);
-    py.cnt = reinterpret_cast<int*>(wsb + lo.off_cy);
     py.status = status;
     if (launch_pass(py, lo.py, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
   }
@@ -306,7 +336,7 @@ bisco_status bisco_bench(const bisco_bench_args* a, bisco_bench_result* r) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
   for (int i = 0; i < a->n_layers; ++i)
-    if (a->ws_bytes < ws_need(&a->layers[i], a->M, dev)) return BISCO_ERR_WORKSPACE;
+    if (a->ws_bytes < ws_need(&a->layers[i], a->M)) return BISCO_ERR_WORKSPACE;
 
   if (ensure_kernel_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
   cudaStream_t user = static_cast<cudaStream_t>(a->stream);

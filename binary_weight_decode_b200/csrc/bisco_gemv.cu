@@ -4,35 +4,40 @@
 //   y[m][o] = sum_seg rs_seg[o] * sum_i sign_seg[o][i] * xin_seg[m][i]  (+ salient term)
 // where each "segment" is one packed sign matrix: a binary base B_k with
 // xin = c_k (.) x and rs = r_k ("FluxBin", Sec. 3.1, decoupled row-column binary
-// bases, column scale folded into the activation as in Sec. 3.2 Stage 1, "LUT
-// Building with Scale Fusion"), the correction's V with xin = x and rs = alpha
-// (z = alpha (.) (V x)), or the correction's U^T with xin = z ("BiLoCo", "The
-// core idea": alpha * u * (v . x)).
+// bases; the column scale is folded into the activation as in Sec. 3.2 Stage 1,
+// "LUT Building with Scale Fusion"), the correction's V with xin = x and
+// rs = alpha (z = alpha (.) (V x)), or the correction's U^T with xin = z
+// ("BiLoCo", "The core idea": alpha * u * (v . x)).
 //
 // Sign-times-activation sums use 5-bit lookup tables in shared memory: for every
 // 5 consecutive columns the CTA stores the 32 signed sums of their scaled
-// activations, so one table read replaces five signed adds (the LUT idea of
-// FluxBin Sec. 3.2, Stage 1/2, re-shaped for B200). A 128-column quad splits into
-// 25 five-bit fields and one three-bit field. All lanes of a warp read the same
-// 32-entry table in one instruction, one entry per bank, so reads never conflict.
+// activations, so one table read replaces five signed adds (the lookup-table idea
+// of FluxBin Sec. 3.2, re-shaped for B200: 32-entry tables, one entry per bank, so
+// the 32 lanes of a warp never conflict). A 128-column quad splits into 25
+// five-bit fields and one three-bit field.
 //
-// Work: item = (block of G row tiles, quad, tile). Items are split evenly over
-// the CTAs. Each lane owns one row of a 32-row tile and reads its 16 bytes of the
-// (tile, quad) block; the 32 lanes read 512 contiguous bytes. Partial sums of a
-// block from different CTAs (split-K) meet in the workspace; the last CTA to
-// finish a block adds them in CTA order (deterministic) and writes Y.
+// Work decomposition: clusters of C CTAs. A cluster owns a range of 32-row tiles;
+// CTA r of the cluster owns 1/C of the columns (units of 128 columns across all
+// segments) and builds tables for those columns only. Warp w owns the tiles
+// w, w + 8, ... of its cluster; each lane owns one row of a tile and reads its 16
+// bytes of a (tile, unit) block, so a warp reads 512 contiguous bytes per load.
+// The C partial sums of a row meet in distributed shared memory and are added
+// in CTA-rank order, so results are deterministic.
 //
-// Launch protocol (programmatic dependent launch): sign words and row scales are
-// loaded before griddepcontrol.wait, activations and the workspace only after it.
+// Launch protocol (programmatic dependent launch): sign words, row and column
+// scales are loaded before griddepcontrol.wait; activations only after it.
 
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "bisco_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace bisco {
 
@@ -48,15 +53,74 @@ __device__ __forceinline__ float ld_val(const void* p, long long i, int dt) {
   return __ldg(reinterpret_cast<const float*>(p) + i);
 }
 
+// Eight consecutive values v[j] = a[off + j] (bf16 or fp32) as fp32, zero where
+// j >= valid. One 16-byte load (two for fp32) when `vec` says the run is aligned.
+__device__ __forceinline__ void load8(const void* a, long long off, int dt, int valid, bool vec, float v[8]) {
+  if (dt == BISCO_BF16) {
+    const unsigned short* h = reinterpret_cast<const unsigned short*>(a) + off;
+    if (vec && valid >= 8) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(h));
+      const unsigned w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = j < valid ? __uint_as_float(static_cast<unsigned>(__ldg(h + j)) << 16) : 0.f;
+    }
+  } else {
+    const float* f = reinterpret_cast<const float*>(a) + off;
+    if (vec && valid >= 8) {
+      const float4 q0 = __ldg(reinterpret_cast<const float4*>(f));
+      const float4 q1 = __ldg(reinterpret_cast<const float4*>(f) + 1);
+      v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+      v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = j < valid ? __ldg(f + j) : 0.f;
+    }
+  }
+}
+
+// load8 for activations: coherent loads through L2 (the previous kernel may have written them).
+__device__ __forceinline__ void load8_l2(const void* a, long long off, int dt, int valid, bool vec, float v[8]) {
+  if (dt == BISCO_BF16) {
+    const unsigned short* h = reinterpret_cast<const unsigned short*>(a) + off;
+    if (vec && valid >= 8) {
+      const uint4 q = __ldcg(reinterpret_cast<const uint4*>(h));
+      const unsigned w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[2 * j] = __uint_as_float(w[j] << 16);
+        v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = j < valid ? __uint_as_float(static_cast<unsigned>(__ldcg(h + j)) << 16) : 0.f;
+    }
+  } else {
+    const float* f = reinterpret_cast<const float*>(a) + off;
+    if (vec && valid >= 8) {
+      const float4 q0 = __ldcg(reinterpret_cast<const float4*>(f));
+      const float4 q1 = __ldcg(reinterpret_cast<const float4*>(f) + 1);
+      v[0] = q0.x; v[1] = q0.y; v[2] = q0.z; v[3] = q0.w;
+      v[4] = q1.x; v[5] = q1.y; v[6] = q1.z; v[7] = q1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = j < valid ? __ldcg(f + j) : 0.f;
+    }
+  }
+}
+
 // Byte offset 4*p of the table entry selected by field F of a 128-bit quad.
 // Fields 0..24 are 5 bits at bit 5F; field 25 is 3 bits at bits 125..127.
 __device__ __forceinline__ unsigned field_off(const uint4& w, const int F) {
   const unsigned ws[4] = {w.x, w.y, w.z, w.w};
   if (F == 25) return (w.w >> 27) & 0x1Cu;
   const int s = 5 * F, wi = s >> 5, b = s & 31;
-  if (b + 5 <= 32) {
-    return (b >= 2 ? (ws[wi] >> (b - 2)) : (ws[wi] << (2 - b))) & 0x7Cu;
-  }
+  if (b + 5 <= 32) return (b >= 2 ? (ws[wi] >> (b - 2)) : (ws[wi] << (2 - b))) & 0x7Cu;
   return __funnelshift_r(ws[wi], ws[wi + 1], b - 2) & 0x7Cu;
 }
 
@@ -78,138 +142,272 @@ __device__ __forceinline__ int find_seg(const PassParam& p, int u) {
   return s;
 }
 
-// CTA that owns work item `it` under the even split [c*L/P, (c+1)*L/P).
-__device__ __forceinline__ int cta_of(long long it, long long L, int P) {
-  return static_cast<int>(((it + 1) * P - 1) / L);
-}
-
 // Index of the lowest set bit of e (1 <= e < 32); folds to a constant when e is.
 __host__ __device__ constexpr int low_bit(int e) {
   return (e & 1) ? 0 : (e & 2) ? 1 : (e & 4) ? 2 : (e & 8) ? 3 : 4;
 }
 
-template <int MB>
-__global__ void __launch_bounds__(kThreads) lut_gemv_kernel(const __grid_constant__ PassParam p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int c = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long pbeg = static_cast<long long>(c) * p.L / p.P;
-  const long long pend = static_cast<long long>(c + 1) * p.L / p.P;
-  const int G = p.G;
-  const long long col0 = pbeg / G, col1 = (pend - 1) / G;
-  const int ncol = static_cast<int>(col1 - col0 + 1);
-  const int blk0 = static_cast<int>(col0 / p.units);
-  const int blk1 = static_cast<int>(col1 / p.units);
+// Per-unit metadata staged in shared memory.
+struct UnitInfo {
+  const uint4* base;   // this unit's quad in row tile 0, lane 0 (nullptr: no bits)
+  int tstride;         // uint4 stride between row tiles (= 32 * nq)
+  int ls;              // local segment index (row-scale slot)
+  int flush;           // 1 if the unit ends its segment within the CTA range or ends a chunk
+  int pad;
+};
+
+struct Smem {
+  float* tables;   // [CU][MB][26 fields][36]   32-entry tables
+  float* cs;       // [max_units][128]          column scales (0 past the segment's columns)
+  float* rsc;      // [max_lseg][max_tiles*32]  row scales
+  float* part;     // [max_tiles][MB][32]       this CTA's partial sums per owned row
+  float* recv;     // [C][MB][max_share]        partial sums pushed by every CTA of the cluster
+  float* xs;       // [MB][nsp]                 salient activations x[idx_t] * s_t
+  UnitInfo* ui;    // [max_units]
+};
+
+__device__ __forceinline__ int max_share(const PassParam& p) { return (p.max_tiles * 32 + p.C - 1) / p.C; }
+
+__device__ __forceinline__ Smem carve(unsigned char* smem, const PassParam& p, int MB, int CU) {
+  Smem s;
   const int nsp = (p.n_sal + 3) & ~3;
+  unsigned char* q = smem;
+  s.tables = reinterpret_cast<float*>(q); q += static_cast<size_t>(CU) * p.col_stride_bytes;
+  s.cs = reinterpret_cast<float*>(q);     q += static_cast<size_t>(p.max_units) * 128 * 4;
+  s.rsc = reinterpret_cast<float*>(q);    q += static_cast<size_t>(p.max_lseg) * p.max_tiles * 32 * 4;
+  s.part = reinterpret_cast<float*>(q);   q += static_cast<size_t>(p.max_tiles) * MB * 32 * 4;
+  s.recv = reinterpret_cast<float*>(q);   q += static_cast<size_t>(p.C) * MB * ((max_share(p) + 3) & ~3) * 4;
+  s.xs = reinterpret_cast<float*>(q);     q += static_cast<size_t>(MB) * nsp * 4;
+  s.ui = reinterpret_cast<UnitInfo*>(q);
+  return s;
+}
 
-  float* tables = reinterpret_cast<float*>(smem);
-  float* xt = reinterpret_cast<float*>(smem + static_cast<size_t>(p.max_cols) * p.col_stride_bytes);
-  float* xs = xt + static_cast<size_t>(p.max_cols) * MB * 128;
-  float* part = xs + MB * nsp;
-  __shared__ int last_flag[2];
+// First row of CTA d's share when R rows are split over C CTAs, and the owner of row r.
+__device__ __forceinline__ int share_begin(int d, int R, int C) { return d * R / C; }
+__device__ __forceinline__ int share_owner(int r, int R, int C) { return ((r + 1) * C - 1) / R; }
 
-  // ---- prefetch this warp's first kDepth items (weights only) ----
-  uint4 buf[kDepth];
-  float rsb[kDepth];
-  auto load_item = [&](long long it, uint4& w, float& rs) {
-    const long long col = it / G;
-    const int g = static_cast<int>(it - col * G);
-    const int b = static_cast<int>(col / p.units);
-    const int u = static_cast<int>(col - static_cast<long long>(b) * p.units);
-    const int t = b * G + g;
-    w = make_uint4(0u, 0u, 0u, 0u);
-    rs = 0.f;
-    if (t >= p.tiles) return;
-    const int sg = find_seg(p, u);
-    const SegParam& S = p.seg[sg];
-    const int q = u - S.unit0;
-    if (S.bits != nullptr)
-      w = __ldcs(S.bits + (static_cast<long long>(t) * S.nq + q) * 32 + lane);
-    const int o = t * 32 + lane;
-    if (o < p.rows) rs = S.rscale ? ld_val(S.rscale, o, S.rdt) : 1.f;
-  };
-#pragma unroll
-  for (int d = 0; d < kDepth; ++d) {
-    const long long it = pbeg + warp + static_cast<long long>(kWarps) * d;
-    if (it < pend) load_item(it, buf[d], rsb[d]);
+// Input value xin[m][cc] of a segment (0 past its columns).
+// Input value xin[m][cc] of a segment (0 past its columns). Activations may have been
+// written by the previous kernel on the stream, so they are read through L2.
+__device__ __forceinline__ float seg_input(const PassParam& p, const SegParam& G, int m, int cc) {
+  if (m >= p.Mc || cc >= G.ncols || G.xsrc == 2) return 0.f;
+  if (G.xsrc == 0) {
+    const long long i = static_cast<long long>(m) * p.ldx + cc;
+    if (p.xdt == BISCO_BF16)
+      return __uint_as_float(static_cast<unsigned>(__ldcg(reinterpret_cast<const unsigned short*>(p.X) + i)) << 16);
+    return __ldcg(reinterpret_cast<const float*>(p.X) + i);
   }
+  return __ldcg(p.Z + static_cast<long long>(m) * p.ldz + cc);
+}
+
+// Shared-memory accesses to the partial-sum buffer through inline PTX without a
+// memory clobber: they never alias the lookup tables, and this lets the compiler
+// keep the next item's table reads ahead of these updates.
+__device__ __forceinline__ float lds_part(const float* a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(static_cast<unsigned>(__cvta_generic_to_shared(a))));
+  return v;
+}
+__device__ __forceinline__ void sts_part(float* a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(a))), "f"(v));
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kThreads, 2) lut_gemv_kernel(const __grid_constant__ PassParam p, const int CU) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int ci = blockIdx.x / p.C;
+  const int t0 = ci * p.tiles / p.ncl, t1 = (ci + 1) * p.tiles / p.ncl, nt = t1 - t0;
+  const int u0 = rank * p.units / p.C, u1 = (rank + 1) * p.units / p.C, nu = u1 - u0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nsp = (p.n_sal + 3) & ~3;
+  const int seg_first = find_seg(p, u0);
+  const Smem S = carve(smem, p, MB, CU);
+  const int rows_c = nt * 32;           // rows of this cluster (incl. padding of the last tile)
+  const int msh = (max_share(p) + 3) & ~3;
+  // Peers write into this CTA's shared memory later on; the split barrier below tells
+  // them that every CTA of the cluster is running before any such write happens.
+  auto started = cluster.barrier_arrive();
+
+  // ---- weights-only staging (before the dependency wait) ----
+  // (a) weight prefetch into the register ring: items of this warp, per chunk of CU
+  //     units, are (owned tile k = tile warp + 8k, unit in chunk)
+  const int my_tiles = warp < nt ? (nt - warp + kWarps - 1) / kWarps : 0;
+  const int nchunks = (nu + CU - 1) / CU;
+  uint4 buf[kDepth];
+  int lk = 0, lu = 0;  // load cursor (tile slot, unit in chunk)
+  auto load_next = [&](int cu0, int cn, uint4& dst) {
+    const int u = u0 + cu0 + lu;
+    const SegParam& G = p.seg[find_seg(p, u)];
+    const int t = t0 + warp + lk * kWarps;
+    dst = G.bits ? __ldcs(G.bits + (static_cast<long long>(t) * G.nq + (u - G.unit0)) * 32 + lane)
+                 : make_uint4(0u, 0u, 0u, 0u);
+    if (++lu == cn) { lu = 0; ++lk; }
+  };
+  auto prefetch_chunk = [&](int c) {
+    const int cu0 = c * CU, cn = min(CU, nu - cu0), n = my_tiles * cn;
+    lk = 0; lu = 0;
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d)
+      if (d < n) load_next(cu0, cn, buf[d]);
+  };
+  prefetch_chunk(0);
+  // (b) unit metadata
+  for (int ul = threadIdx.x; ul < nu; ul += kThreads) {
+    const int u = u0 + ul;
+    const int sg = find_seg(p, u);
+    const SegParam& G = p.seg[sg];
+    UnitInfo I;
+    I.base = G.bits ? G.bits + static_cast<long long>(u - G.unit0) * 32 : nullptr;
+    I.tstride = 32 * G.nq;
+    I.ls = sg - seg_first;
+    I.flush = (ul + 1 == nu) || ((ul + 1) % CU == 0) || (find_seg(p, u + 1) != sg);
+    I.pad = 0;
+    S.ui[ul] = I;
+  }
+  // (c) column and row scales, staged in rounds; every load of a round is issued
+  //     before any of them is used
+  const int nls = find_seg(p, u1 - 1) - seg_first + 1;
+  const int n_cs = nu * 16, n_rs = nls * nt * 4;
+  for (int base = 0; base < n_cs + n_rs; base += 2 * kThreads) {
+    float v[2][8];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int ch = base + threadIdx.x + k * kThreads;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[k][j] = 0.f;
+      if (ch < n_cs) {  // column scales of unit ch/16, columns 8*(ch%16) ..
+        const int ul = ch >> 4, j0 = (ch & 15) * 8;
+        const int u = u0 + ul;
+        const SegParam& G = p.seg[find_seg(p, u)];
+        const int cc = (u - G.unit0) * 128 + j0;
+        const int valid = G.xsrc == 2 ? 0 : max(0, min(8, G.ncols - cc));
+        if (G.cscale == nullptr) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[k][j] = j < valid ? 1.f : 0.f;
+        } else if (valid > 0) {
+          load8(G.cscale, cc, G.cdt, valid, G.cvec != 0, v[k]);
+        }
+      } else if (ch < n_cs + n_rs) {  // row scales of local segment ls, rows 8*(...) ..
+        const int rc = ch - n_cs;
+        const int ls = rc / (nt * 4), r8 = (rc - ls * nt * 4) * 8;
+        const SegParam& G = p.seg[seg_first + ls];
+        const int o = t0 * 32 + r8;
+        const int valid = max(0, min(8, p.rows - o));
+        if (G.rscale == nullptr) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[k][j] = j < valid ? 1.f : 0.f;
+        } else if (valid > 0) {
+          load8(G.rscale, o, G.rdt, valid, G.rvec != 0, v[k]);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int ch = base + threadIdx.x + k * kThreads;
+      float* d = nullptr;
+      if (ch < n_cs) {
+        d = S.cs + ch * 8;
+      } else if (ch < n_cs + n_rs) {
+        const int rc = ch - n_cs;
+        const int ls = rc / (nt * 4), r8 = (rc - ls * nt * 4) * 8;
+        d = S.rsc + ls * p.max_tiles * 32 + r8;
+      }
+      if (d) {
+        reinterpret_cast<float4*>(d)[0] = make_float4(v[k][0], v[k][1], v[k][2], v[k][3]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(v[k][4], v[k][5], v[k][6], v[k][7]);
+      }
+    }
+  }
+  for (int idx = threadIdx.x; idx < nt * MB * 32; idx += kThreads) S.part[idx] = 0.f;
+  __syncthreads();  // unit metadata and scales visible
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
 
-  // ---- stage scaled activations x~ for this CTA's quads ----
-  for (int idx = threadIdx.x; idx < ncol * MB * 128; idx += kThreads) {
-    const int s = idx / (MB * 128);
-    const int rem = idx - s * (MB * 128);
-    const int m = rem >> 7, j = rem & 127;
-    const long long col = col0 + s;
-    const int u = static_cast<int>(col % p.units);
-    const SegParam& S = p.seg[find_seg(p, u)];
-    const int ci = (u - S.unit0) * 128 + j;
-    float v = 0.f;
-    if (m < p.Mc && ci < S.ncols) {
-      if (S.xsrc == 0) v = ld_val(p.X, m * p.ldx + ci, p.xdt);
-      else if (S.xsrc == 1) v = __ldcg(p.Z + m * p.ldz + ci);
-      if (S.cscale) v *= ld_val(S.cscale, ci, S.cdt);
-    }
-    xt[(s * MB + m) * 128 + j] = v;
-  }
+  // ---- salient activations (gathered and scaled) ----
   for (int idx = threadIdx.x; idx < MB * p.n_sal; idx += kThreads) {
     const int m = idx / p.n_sal, t = idx - m * p.n_sal;
     float v = 0.f;
-    const int ci = __ldg(p.sal_idx + t);
-    if (ci < 0 || ci >= p.xcols) {
-      atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));  // index out of range: term skipped
-    } else if (m < p.Mc) {
-      v = ld_val(p.X, m * p.ldx + ci, p.xdt) * __ldg(p.sal_scale + t);
+    const int cc = __ldg(p.sal_idx + t);
+    if (cc < 0 || cc >= p.xcols) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+    else if (m < p.Mc) {
+      const long long i = static_cast<long long>(m) * p.ldx + cc;
+      const float xv = p.xdt == BISCO_BF16
+                           ? __uint_as_float(static_cast<unsigned>(__ldcg(reinterpret_cast<const unsigned short*>(p.X) + i)) << 16)
+                           : __ldcg(reinterpret_cast<const float*>(p.X) + i);
+      v = xv * __ldg(p.sal_scale + t);
     }
-    xs[m * nsp + t] = v;
+    S.xs[m * nsp + t] = v;
   }
-  for (int idx = threadIdx.x; idx < 2 * MB * G * 32; idx += kThreads) part[idx] = 0.f;
-  __syncthreads();
 
-  // ---- build the 32-entry tables: lane f computes all entries of field f ----
-  for (int task = warp; task < ncol * MB; task += kWarps) {
-    const int s = task / MB, m = task - s * MB;
-    if (lane < kFields) {
-      const float* x = xt + (s * MB + m) * 128 + 5 * lane;
-      const float x0 = x[0], x1 = x[1], x2 = x[2];
-      const float x3 = lane < 25 ? x[3] : 0.f, x4 = lane < 25 ? x[4] : 0.f;
-      const float d[5] = {2.f * x0, 2.f * x1, 2.f * x2, 2.f * x3, 2.f * x4};
-      float T[32];
-      T[0] = -((x0 + x1) + (x2 + x3) + x4);
+  constexpr int NA = MB > 1 ? MB : 2;
+  float acc[NA], tot[MB];
 #pragma unroll
-      for (int e = 1; e < 32; ++e) T[e] = T[e & (e - 1)] + d[low_bit(e)];
-      float* dst = tables + static_cast<size_t>(s) * (p.col_stride_bytes / 4) + (m * kFields + lane) * kFieldStride;
+  for (int m = 0; m < NA; ++m) acc[m] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        reinterpret_cast<float4*>(dst)[j] = make_float4(T[4 * j], T[4 * j + 1], T[4 * j + 2], T[4 * j + 3]);
+  for (int m = 0; m < MB; ++m) tot[m] = 0.f;
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(S.tables);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int cu0 = c * CU, cn = min(CU, nu - cu0);
+    // tables straight from the activations: task (unit, batch row) per warp; lane f
+    // loads the 5 inputs of field f (3 for field 25), scales them by c and writes
+    // all 32 signed sums. Two tasks' loads are in flight together.
+    for (int task = warp; task < cn * MB; task += 2 * kWarps) {
+      float xin[2][5];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int tk = task + h * kWarps;
+#pragma unroll
+        for (int n = 0; n < 5; ++n) xin[h][n] = 0.f;
+        if (tk < cn * MB && lane < kFields) {
+          const int ulc = tk / MB, m = tk - ulc * MB;
+          const int u = u0 + cu0 + ulc;
+          const SegParam& G = p.seg[find_seg(p, u)];
+          const int cb = (u - G.unit0) * 128 + 5 * lane;
+          const int len = lane < 25 ? 5 : 3;
+#pragma unroll
+          for (int n = 0; n < 5; ++n)
+            if (n < len) xin[h][n] = seg_input(p, G, m, cb + n);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int tk = task + h * kWarps;
+        if (tk < cn * MB && lane < kFields) {
+          const int ulc = tk / MB, m = tk - ulc * MB;
+          const float* cv = S.cs + (cu0 + ulc) * 128 + 5 * lane;
+          const int len = lane < 25 ? 5 : 3;
+          float x[5];
+#pragma unroll
+          for (int n = 0; n < 5; ++n) x[n] = n < len ? xin[h][n] * cv[n] : 0.f;
+          const float d[5] = {2.f * x[0], 2.f * x[1], 2.f * x[2], 2.f * x[3], 2.f * x[4]};
+          float T[32];
+          T[0] = -((x[0] + x[1]) + (x[2] + x[3]) + x[4]);
+#pragma unroll
+          for (int e = 1; e < 32; ++e) T[e] = T[e & (e - 1)] + d[low_bit(e)];
+          float* dst = S.tables + static_cast<size_t>(ulc) * (p.col_stride_bytes / 4) + (m * kFields + lane) * kFieldStride;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            reinterpret_cast<float4*>(dst)[j] = make_float4(T[4 * j], T[4 * j + 1], T[4 * j + 2], T[4 * j + 3]);
+        }
+      }
     }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // ---- main loop: one table read per field per batch row ----
-  const unsigned char* tb = reinterpret_cast<const unsigned char*>(tables);
-  for (long long base = 0;; base += kDepth) {
-    const long long first = pbeg + warp + static_cast<long long>(kWarps) * base;
-    if (first >= pend) break;
+    // lookups: item i of this chunk sits in ring slot i % kDepth
+    const int n_ci = my_tiles * cn;
+    int pk = 0, pu = 0;  // processing cursor
+    for (int base = 0; base < n_ci; base += kDepth) {
 #pragma unroll
-    for (int d = 0; d < kDepth; ++d) {
-      const long long it = first + static_cast<long long>(kWarps) * d;
-      if (it < pend) {
-        const long long col = it / G;
-        const int g = static_cast<int>(it - col * G);
-        const int b = static_cast<int>(col / p.units);
-        const int u = static_cast<int>(col - static_cast<long long>(b) * p.units);
-        const int t = b * G + g;
-        if (t < p.tiles) {
+      for (int d = 0; d < kDepth; ++d) {
+        if (base + d < n_ci) {
           const uint4 w = buf[d];
-          const unsigned uoff = static_cast<unsigned>(col - col0) * static_cast<unsigned>(p.col_stride_bytes);
-          float acc[MB > 1 ? MB : 2];
-#pragma unroll
-          for (int m = 0; m < (MB > 1 ? MB : 2); ++m) acc[m] = 0.f;
+          if (base + d + kDepth < n_ci) load_next(cu0, cn, buf[d]);
+          const unsigned uoff = static_cast<unsigned>(pu) * static_cast<unsigned>(p.col_stride_bytes);
           if (MB == 1) {
-            // fields in pairs: one packed fp32x2 add per two table reads
 #pragma unroll
             for (int F = 0; F < kFields; F += 2) {
               const float v0 = *reinterpret_cast<const float*>(tb + (field_off(w, F) | uoff) + F * kFieldStride * 4);
@@ -229,110 +427,499 @@ __global__ void __launch_bounds__(kThreads) lut_gemv_kernel(const __grid_constan
               }
             }
           }
-          float val[MB];
-          if (MB == 1) val[0] = (acc[0] + acc[1]) * rsb[d];
-          else {
+          const int tl = warp + pk * kWarps;
+          const UnitInfo& I = S.ui[cu0 + pu];
+          if (I.flush) {  // the unit ends a segment (or the chunk): apply that segment's row scale
+            const float rs = S.rsc[I.ls * p.max_tiles * 32 + tl * 32 + lane];
+            if (MB == 1) {
+              tot[0] = fmaf(acc[0] + acc[1], rs, tot[0]);
+              acc[0] = acc[1] = 0.f;
+            } else {
 #pragma unroll
-            for (int m = 0; m < MB; ++m) val[m] = acc[m] * rsb[d];
-          }
-          const int o = t * 32 + lane;
-          if (u == 0 && p.n_sal > 0 && o < p.rows) {
-            // salient columns: y += sum_t q[o][t] * (x[idx_t] * s_t), added once per row
-            const int8_t* qrow = p.sal_q + static_cast<long long>(o) * p.sal_stride;
-            for (int t0 = 0; t0 < p.n_sal; t0 += 16) {
-              const uint4 qq = __ldg(reinterpret_cast<const uint4*>(qrow + t0));
-              const unsigned qw[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                const int tt = t0 + k;
-                if (tt < p.n_sal) {
-                  const float qv = static_cast<float>(static_cast<int8_t>((qw[k >> 2] >> (8 * (k & 3))) & 0xFF));
-#pragma unroll
-                  for (int m = 0; m < MB; ++m) val[m] = fmaf(qv, xs[m * nsp + tt], val[m]);
-                }
-              }
+              for (int m = 0; m < MB; ++m) { tot[m] = fmaf(acc[m], rs, tot[m]); acc[m] = 0.f; }
             }
           }
-          const int slot = b - blk0;
-          if (slot < 0 || slot > 1) {  // cannot happen under make_plan; record instead of writing out of range
-            atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
-          } else {
+          if (++pu == cn) {  // this tile's units of the chunk are done
 #pragma unroll
-            for (int m = 0; m < MB; ++m) part[(slot * MB + m) * G * 32 + g * 32 + lane] += val[m];
+            for (int m = 0; m < MB; ++m) { S.part[(tl * MB + m) * 32 + lane] += tot[m]; tot[m] = 0.f; }
+            pu = 0;
+            ++pk;
           }
         }
-        const long long nxt = it + static_cast<long long>(kWarps) * kDepth;
-        if (nxt < pend) load_item(nxt, buf[d], rsb[d]);
       }
     }
+    if (c + 1 < nchunks) {
+      prefetch_chunk(c + 1);
+      __syncthreads();  // all warps are done with this chunk's tables before they are rebuilt
+    }
   }
-  __syncthreads();
 
-  // ---- publish partial sums, then the last CTA of each block reduces it ----
-  const int nslots = blk1 - blk0 + 1;
-  float* gpart = p.part + static_cast<long long>(c) * 2 * MB * G * 32;
-  for (int idx = threadIdx.x; idx < nslots * MB * G * 32; idx += kThreads) gpart[idx] = part[idx];
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int sl = 0; sl < 2; ++sl) {
-      last_flag[sl] = 0;
-      if (sl < nslots) {
-        const int b = blk0 + sl;
-        const long long f0 = static_cast<long long>(b) * p.units * G;
-        const long long f1 = f0 + static_cast<long long>(p.units) * G - 1;
-        const int need = cta_of(f1, p.L, p.P) - cta_of(f0, p.L, p.P) + 1;
-        const int old = atomicAdd(p.cnt + b, 1);
-        last_flag[sl] = (old == need - 1);
+  // ---- push partial sums to the CTA that reduces each row (distributed shared memory) ----
+  cluster.barrier_wait(std::move(started));
+  for (int k = 0; k < my_tiles; ++k) {
+    const int tl = warp + k * kWarps;
+    const int lr = tl * 32 + lane;
+    const int dst = share_owner(lr, rows_c, p.C);
+    float* rp = cluster.map_shared_rank(S.recv, dst);
+    const int sr = lr - share_begin(dst, rows_c, p.C);
+#pragma unroll
+    for (int m = 0; m < MB; ++m) rp[(rank * MB + m) * msh + sr] = S.part[(tl * MB + m) * 32 + lane];
+  }
+  cluster.sync();  // all partial sums have landed
+
+  // ---- reduce this CTA's share of rows in CTA-rank order, add salient columns, store ----
+  const int r0 = share_begin(rank, rows_c, p.C), r1 = share_begin(rank + 1, rows_c, p.C);
+  for (int lr = r0 + threadIdx.x; lr < r1; lr += kThreads) {
+    const int o = t0 * 32 + lr;
+    if (o >= p.rows) continue;
+    const int sr = lr - r0;
+    float sum[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) sum[m] = 0.f;
+    for (int src = 0; src < p.C; ++src) {
+#pragma unroll
+      for (int m = 0; m < MB; ++m) sum[m] += S.recv[(src * MB + m) * msh + sr];
+    }
+    if (p.n_sal > 0) {
+      // salient columns: y += sum_t q[o][t] * (x[idx_t] * s_t)
+      const int8_t* qrow = p.sal_q + static_cast<long long>(o) * p.sal_stride;
+      for (int tq = 0; tq < p.n_sal; tq += 16) {
+        const uint4 qq = __ldg(reinterpret_cast<const uint4*>(qrow + tq));
+        const unsigned qw[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int tt = tq + k;
+          if (tt < p.n_sal) {
+            const float qv = static_cast<float>(static_cast<int8_t>((qw[k >> 2] >> (8 * (k & 3))) & 0xFF));
+#pragma unroll
+            for (int m = 0; m < MB; ++m) sum[m] = fmaf(qv, S.xs[m * nsp + tt], sum[m]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      if (m < p.Mc) {
+        if (p.ydt == BISCO_BF16)
+          reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(sum[m]);
+        else
+          reinterpret_cast<float*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = sum[m];
       }
     }
   }
-  __syncthreads();
-  for (int sl = 0; sl < nslots; ++sl) {
-    if (!last_flag[sl]) continue;
-    __threadfence();
-    const int b = blk0 + sl;
-    const long long f0 = static_cast<long long>(b) * p.units * G;
-    const long long f1 = f0 + static_cast<long long>(p.units) * G - 1;
-    const int cf = cta_of(f0, p.L, p.P), cl = cta_of(f1, p.L, p.P);
-    for (int idx = threadIdx.x; idx < p.Mc * G * 32; idx += kThreads) {
-      const int m = idx / (G * 32), r = idx - m * (G * 32);
-      const int o = (b * G) * 32 + r;
-      if (o >= p.rows) continue;
-      float sum = 0.f;
-      for (int cc = cf; cc <= cl; ++cc) {
-        const long long cb = static_cast<long long>(cc) * p.L / p.P;
-        const int cblk0 = static_cast<int>((cb / G) / p.units);
-        sum += __ldcg(p.part + static_cast<long long>(cc) * 2 * MB * G * 32 + ((b - cblk0) * MB + m) * G * 32 + r);
+}
+
+// ----------------------------------------------------------------------------
+// Batch rows <= 2: a wider CTA (16 warps, 64 registers a thread) that stages the
+// packed sign words with cp.async into a per-warp shared-memory ring, so the loop
+// over work items stays compact. Items (unit, row tile) of the CTA are dealt to
+// the warps round-robin; every warp keeps its own partial sum per row tile, and
+// the warps' partial sums are added in warp order at the end.
+// ----------------------------------------------------------------------------
+constexpr int kWW = 16;          // warps per CTA
+constexpr int kTW = kWW * 32;    // threads per CTA
+constexpr int kRing = 6;         // items per warp in flight
+
+struct WUnit {           // per-unit metadata of the current chunk
+  const uint4* base;    // sign words of this unit's quad, row tile 0, lane 0 (nullptr: none)
+  int tstride;          // uint4 stride between row tiles
+  int ls;               // local segment (row-scale slot)
+};
+
+struct WSmem {
+  float* tables;   // [CU][MB][26][36]          tables of the current chunk of units
+  float* xt;       // [CU][MB][128]             scaled activations of the chunk
+  float* cs;       // [max_units][128]          column scales
+  float* rsc;      // [max_lseg][max_tiles*32]  row scales
+  float* part;     // [kWW][max_tiles][MB][32]  per-warp partial sums
+  float* recv;     // [C][MB][msh]              partial sums pushed by the cluster
+  float* xs;       // [MB][nsp]                 salient activations
+  WUnit* ui;       // [max_units]
+  uint4* ring;     // [kWW][kRing][32]          staged sign words
+};
+
+__host__ __device__ __forceinline__ size_t wsmem_bytes(int CU, int col_stride, int max_units, int max_lseg,
+                                                       int max_tiles, int MB, int C, int n_sal) {
+  const int nsp = (n_sal + 3) & ~3;
+  const int msh = ((max_tiles * 32 + C - 1) / C + 3) & ~3;
+  return static_cast<size_t>(CU) * col_stride + static_cast<size_t>(CU) * MB * 128 * 4 +
+         static_cast<size_t>(max_units) * 128 * 4 + static_cast<size_t>(max_lseg) * max_tiles * 32 * 4 +
+         static_cast<size_t>(kWW) * max_tiles * MB * 32 * 4 + static_cast<size_t>(C) * MB * msh * 4 +
+         static_cast<size_t>(MB) * nsp * 4 + static_cast<size_t>(max_units) * sizeof(WUnit) +
+         static_cast<size_t>(kWW) * kRing * 32 * 16 + 16;
+}
+
+__device__ __forceinline__ WSmem wcarve(unsigned char* smem, const PassParam& p, int MB, int CU) {
+  WSmem s;
+  const int nsp = (p.n_sal + 3) & ~3;
+  unsigned char* q = smem;
+  s.tables = reinterpret_cast<float*>(q); q += static_cast<size_t>(CU) * p.col_stride_bytes;
+  s.xt = reinterpret_cast<float*>(q);     q += static_cast<size_t>(CU) * MB * 128 * 4;
+  s.cs = reinterpret_cast<float*>(q);     q += static_cast<size_t>(p.max_units) * 128 * 4;
+  s.rsc = reinterpret_cast<float*>(q);    q += static_cast<size_t>(p.max_lseg) * p.max_tiles * 32 * 4;
+  s.part = reinterpret_cast<float*>(q);   q += static_cast<size_t>(kWW) * p.max_tiles * MB * 32 * 4;
+  s.recv = reinterpret_cast<float*>(q);   q += static_cast<size_t>(p.C) * MB * ((max_share(p) + 3) & ~3) * 4;
+  s.xs = reinterpret_cast<float*>(q);     q += static_cast<size_t>(MB) * nsp * 4;
+  s.ui = reinterpret_cast<WUnit*>(q);     q += static_cast<size_t>(p.max_units) * sizeof(WUnit);
+  q = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(q) + 15) & ~uintptr_t(15));
+  s.ring = reinterpret_cast<uint4*>(q);
+  return s;
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<unsigned>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Cursor over this warp's items of a chunk: chunk-local item k = ulc * nt + tl, and
+// the warp takes k = warp, warp + 16, ...; advancing by 16 needs no division.
+struct ItemCursor {
+  int ulc, tl;
+  __device__ __forceinline__ void init(int k, int nt) { ulc = 0; tl = k; while (tl >= nt) { tl -= nt; ++ulc; } }
+  __device__ __forceinline__ void next(int nt) { tl += kWW; while (tl >= nt) { tl -= nt; ++ulc; } }
+};
+
+template <int MB>
+__global__ void __launch_bounds__(kTW, 2) lut_gemv_warp_kernel(const __grid_constant__ PassParam p, const int CU) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int ci = blockIdx.x / p.C;
+  const int t0 = ci * p.tiles / p.ncl, t1 = (ci + 1) * p.tiles / p.ncl, nt = t1 - t0;
+  const int u0 = rank * p.units / p.C, u1 = (rank + 1) * p.units / p.C, nu = u1 - u0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nsp = (p.n_sal + 3) & ~3;
+  const int seg_first = find_seg(p, u0);
+  const WSmem S = wcarve(smem, p, MB, CU);
+  const int rows_c = nt * 32;
+  const int msh = (max_share(p) + 3) & ~3;
+  auto started = cluster.barrier_arrive();
+
+  const int nchunks = (nu + CU - 1) / CU;
+  uint4* my_ring = S.ring + warp * kRing * 32 + lane;
+
+  // ---- weights-only staging (before the dependency wait) ----
+  for (int ul = threadIdx.x; ul < nu; ul += kTW) {
+    const int u = u0 + ul;
+    const int sg = find_seg(p, u);
+    const SegParam& G = p.seg[sg];
+    WUnit I;
+    I.base = G.bits ? G.bits + static_cast<long long>(u - G.unit0) * 32 : nullptr;
+    I.tstride = 32 * G.nq;
+    I.ls = sg - seg_first;
+    S.ui[ul] = I;
+  }
+  const int nls = find_seg(p, u1 - 1) - seg_first + 1;
+  const int n_cs = nu * 16, n_rs = nls * nt * 4;
+  for (int ch = threadIdx.x; ch < n_cs + n_rs; ch += kTW) {
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    float* d;
+    if (ch < n_cs) {
+      const int ul = ch >> 4, j0 = (ch & 15) * 8;
+      const int u = u0 + ul;
+      const SegParam& G = p.seg[find_seg(p, u)];
+      const int cc = (u - G.unit0) * 128 + j0;
+      const int valid = G.xsrc == 2 ? 0 : max(0, min(8, G.ncols - cc));
+      if (G.cscale == nullptr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = j < valid ? 1.f : 0.f;
+      } else if (valid > 0) {
+        load8(G.cscale, cc, G.cdt, valid, G.cvec != 0, v);
       }
-      if (p.ydt == BISCO_BF16)
-        reinterpret_cast<__nv_bfloat16*>(p.Y)[m * p.ldy + o] = __float2bfloat16_rn(sum);
-      else
-        reinterpret_cast<float*>(p.Y)[m * p.ldy + o] = sum;
+      d = S.cs + ch * 8;
+    } else {
+      const int rc = ch - n_cs;
+      const int ls = rc / (nt * 4), r8 = (rc - ls * nt * 4) * 8;
+      const SegParam& G = p.seg[seg_first + ls];
+      const int o = t0 * 32 + r8;
+      const int valid = max(0, min(8, p.rows - o));
+      if (G.rscale == nullptr) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = j < valid ? 1.f : 0.f;
+      } else if (valid > 0) {
+        load8(G.rscale, o, G.rdt, valid, G.rvec != 0, v);
+      }
+      d = S.rsc + ls * p.max_tiles * 32 + r8;
     }
-    if (threadIdx.x == 0) p.cnt[b] = 0;
+    reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  float* my_part = S.part + static_cast<size_t>(warp) * p.max_tiles * MB * 32;
+  for (int idx = lane; idx < nt * MB * 32; idx += 32) my_part[idx] = 0.f;
+  __syncthreads();  // unit metadata visible
+
+  // stage this warp's first items of chunk 0
+  ItemCursor ic;
+  int n_issue = 0;  // items of the current chunk issued so far by this warp
+  auto issue = [&](int cu0, int cn) {  // stage the item under the issue cursor (one group)
+    if (ic.ulc < cn) {
+      const WUnit& I = S.ui[cu0 + ic.ulc];
+      if (I.base) cp_async16(my_ring + (n_issue % kRing) * 32, I.base + static_cast<long long>(t0 + ic.tl) * I.tstride + lane);
+      ic.next(nt);
+    }
+    ++n_issue;
+    cp_async_commit();
+  };
+  {
+    const int cn = min(CU, nu);
+    ic.init(warp, nt);
+    n_issue = 0;
+#pragma unroll
+    for (int j = 0; j < kRing - 1; ++j) issue(0, cn);
+  }
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  for (int idx = threadIdx.x; idx < MB * p.n_sal; idx += kTW) {
+    const int m = idx / p.n_sal, t = idx - m * p.n_sal;
+    float v = 0.f;
+    const int cc = __ldg(p.sal_idx + t);
+    if (cc < 0 || cc >= p.xcols) {
+      atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+    } else if (m < p.Mc) {
+      const long long i = static_cast<long long>(m) * p.ldx + cc;
+      const float xv = p.xdt == BISCO_BF16
+                           ? __uint_as_float(static_cast<unsigned>(__ldcg(reinterpret_cast<const unsigned short*>(p.X) + i)) << 16)
+                           : __ldcg(reinterpret_cast<const float*>(p.X) + i);
+      v = xv * __ldg(p.sal_scale + t);
+    }
+    S.xs[m * nsp + t] = v;
+  }
+
+  const unsigned char* tb = reinterpret_cast<const unsigned char*>(S.tables);
+  for (int c = 0; c < nchunks; ++c) {
+    const int cu0 = c * CU, cn = min(CU, nu - cu0);
+    if (c > 0) __syncthreads();  // the previous chunk's tables are no longer read
+    // scaled activations of the chunk: 8-column runs, one 16-byte load each
+    for (int ch = threadIdx.x; ch < cn * MB * 16; ch += kTW) {
+      const int ulc = ch / (MB * 16);
+      const int rem = ch - ulc * (MB * 16);
+      const int m = rem >> 4, j0 = (rem & 15) * 8;
+      const int u = u0 + cu0 + ulc;
+      const SegParam& G = p.seg[find_seg(p, u)];
+      const int cc = (u - G.unit0) * 128 + j0;
+      const int valid = max(0, min(8, G.ncols - cc));
+      float xv[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xv[j] = 0.f;
+      if (m < p.Mc && valid > 0 && G.xsrc != 2) {
+        if (G.xsrc == 0)
+          load8_l2(p.X, static_cast<long long>(m) * p.ldx + cc, p.xdt, valid, p.x_vec != 0, xv);
+        else
+          load8_l2(p.Z, static_cast<long long>(m) * p.ldz + cc, BISCO_F32, valid, p.z_vec != 0, xv);
+      }
+      const float* cv = S.cs + (cu0 + ulc) * 128 + j0;
+      float4* d4 = reinterpret_cast<float4*>(S.xt + (ulc * MB + m) * 128 + j0);
+      d4[0] = make_float4(xv[0] * cv[0], xv[1] * cv[1], xv[2] * cv[2], xv[3] * cv[3]);
+      d4[1] = make_float4(xv[4] * cv[4], xv[5] * cv[5], xv[6] * cv[6], xv[7] * cv[7]);
+    }
+    __syncthreads();
+    // tables: task (unit, batch row); lane f builds the 32 signed sums of field f
+    for (int q = warp; q < cn * MB; q += kWW) {
+      const int ulc = q / MB, m = q - ulc * MB;
+      if (lane < kFields) {
+        const float* x = S.xt + (ulc * MB + m) * 128 + 5 * lane;
+        const float x0 = x[0], x1 = x[1], x2 = x[2];
+        const float x3 = lane < 25 ? x[3] : 0.f, x4 = lane < 25 ? x[4] : 0.f;
+        const float d[5] = {2.f * x0, 2.f * x1, 2.f * x2, 2.f * x3, 2.f * x4};
+        float T[32];
+        T[0] = -((x0 + x1) + (x2 + x3) + x4);
+#pragma unroll
+        for (int e = 1; e < 32; ++e) T[e] = T[e & (e - 1)] + d[low_bit(e)];
+        float* dst = S.tables + static_cast<size_t>(ulc) * (p.col_stride_bytes / 4) + (m * kFields + lane) * kFieldStride;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          reinterpret_cast<float4*>(dst)[k] = make_float4(T[4 * k], T[4 * k + 1], T[4 * k + 2], T[4 * k + 3]);
+      }
+    }
+    __syncthreads();
+    // the activations are in: let the next kernel on the stream start its prefetch
+    if (c == 0) asm volatile("griddepcontrol.launch_dependents;");
+
+    // lookups over this warp's items of the chunk
+    const int n_my = (cn * nt > warp) ? (cn * nt - warp + kWW - 1) / kWW : 0;
+    ItemCursor pc;
+    pc.init(warp, nt);
+    for (int j = 0; j < n_my; ++j) {
+      issue(cu0, cn);
+      cp_async_wait<kRing - 1>();
+      const uint4 w = my_ring[(j % kRing) * 32];
+      const unsigned uoff = static_cast<unsigned>(pc.ulc) * static_cast<unsigned>(p.col_stride_bytes);
+      float a[MB > 1 ? MB : 2];
+#pragma unroll
+      for (int m = 0; m < (MB > 1 ? MB : 2); ++m) a[m] = 0.f;
+      if (MB == 1) {
+#pragma unroll
+        for (int F = 0; F < kFields; F += 2) {
+          const float v0 = *reinterpret_cast<const float*>(tb + (field_off(w, F) | uoff) + F * kFieldStride * 4);
+          const float v1 = *reinterpret_cast<const float*>(tb + (field_off(w, F + 1) | uoff) + (F + 1) * kFieldStride * 4);
+          fadd2(a[0], a[1], v0, v1);
+        }
+      } else {
+#pragma unroll
+        for (int F = 0; F < kFields; ++F) {
+          const unsigned off = field_off(w, F) | uoff;
+#pragma unroll
+          for (int m = 0; m < MB; m += 2) {
+            const float v0 = *reinterpret_cast<const float*>(tb + off + (m * kFields + F) * kFieldStride * 4);
+            const float v1 = *reinterpret_cast<const float*>(tb + off + ((m + 1) * kFields + F) * kFieldStride * 4);
+            fadd2(a[m], a[m + 1], v0, v1);
+          }
+        }
+      }
+      const float rs = S.rsc[S.ui[cu0 + pc.ulc].ls * p.max_tiles * 32 + pc.tl * 32 + lane];
+      float* pp = my_part + pc.tl * MB * 32 + lane;
+      if (MB == 1) {
+        sts_part(pp, fmaf(a[0] + a[1], rs, lds_part(pp)));
+      } else {
+#pragma unroll
+        for (int m = 0; m < MB; ++m) sts_part(pp + m * 32, fmaf(a[m], rs, lds_part(pp + m * 32)));
+      }
+      pc.next(nt);
+    }
+    cp_async_wait<0>();
+    if (c + 1 < nchunks) {  // first items of the next chunk
+      const int ncn = min(CU, nu - (c + 1) * CU);
+      ic.init(warp, nt);
+      n_issue = 0;
+#pragma unroll
+      for (int j = 0; j < kRing - 1; ++j) issue((c + 1) * CU, ncn);
+    }
+  }
+  if (nchunks == 0) asm volatile("griddepcontrol.launch_dependents;");
+  __syncthreads();  // all warps' partial sums are in shared memory
+
+  // ---- sum over warps (fixed order) and push to the CTA that owns each row ----
+  cluster.barrier_wait(std::move(started));
+  for (int idx = threadIdx.x; idx < nt * MB * 32; idx += kTW) {
+    const int tl = idx / (MB * 32);
+    const int rem = idx - tl * MB * 32;
+    const int m = rem >> 5, ln = rem & 31;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWW; ++w) v += S.part[(static_cast<size_t>(w) * p.max_tiles + tl) * MB * 32 + m * 32 + ln];
+    const int lr = tl * 32 + ln;
+    const int dst = share_owner(lr, rows_c, p.C);
+    float* rp = cluster.map_shared_rank(S.recv, dst);
+    rp[(rank * MB + m) * msh + (lr - share_begin(dst, rows_c, p.C))] = v;
+  }
+  cluster.sync();  // all partial sums have landed
+
+  // ---- reduce this CTA's share of rows in CTA-rank order, add salient columns, store ----
+  const int r0 = share_begin(rank, rows_c, p.C), r1 = share_begin(rank + 1, rows_c, p.C);
+  for (int lr = r0 + threadIdx.x; lr < r1; lr += kTW) {
+    const int o = t0 * 32 + lr;
+    if (o >= p.rows) continue;
+    const int sr = lr - r0;
+    float sum[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) sum[m] = 0.f;
+    for (int src = 0; src < p.C; ++src) {
+#pragma unroll
+      for (int m = 0; m < MB; ++m) sum[m] += S.recv[(src * MB + m) * msh + sr];
+    }
+    if (p.n_sal > 0) {
+      const int8_t* qrow = p.sal_q + static_cast<long long>(o) * p.sal_stride;
+      for (int tq = 0; tq < p.n_sal; tq += 16) {
+        const uint4 qq = __ldg(reinterpret_cast<const uint4*>(qrow + tq));
+        const unsigned qw[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int tt = tq + k;
+          if (tt < p.n_sal) {
+            const float qv = static_cast<float>(static_cast<int8_t>((qw[k >> 2] >> (8 * (k & 3))) & 0xFF));
+#pragma unroll
+            for (int m = 0; m < MB; ++m) sum[m] = fmaf(qv, S.xs[m * nsp + tt], sum[m]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      if (m < p.Mc) {
+        if (p.ydt == BISCO_BF16)
+          reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(sum[m]);
+        else
+          reinterpret_cast<float*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = sum[m];
+      }
+    }
   }
 }
 
 template <int MB>
 cudaError_t set_attrs() {
-  return cudaFuncSetAttribute(lut_gemv_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(query_smem_limit()));
+  const int lim = static_cast<int>(query_smem_limit());
+  cudaError_t e = cudaFuncSetAttribute(lut_gemv_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  if (e == cudaSuccess && MB <= 2)
+    e = cudaFuncSetAttribute(lut_gemv_warp_kernel<MB <= 2 ? MB : 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
+  return e;
 }
 
 template <int MB>
 cudaError_t launch_mb(const PassParam& p, const Plan& plan, cudaStream_t stream, bool pdl) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.P);
-  cfg.blockDim = dim3(kThreads);
+  cfg.gridDim = dim3(plan.ncl * plan.C);
+  cfg.blockDim = dim3(plan.kind == 0 ? kTW : kThreads);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, lut_gemv_kernel<MB>, p);
+  cfg.numAttrs = pdl ? 2 : 1;
+  if constexpr (MB <= 2) {
+    if (plan.kind == 0) return cudaLaunchKernelEx(&cfg, lut_gemv_warp_kernel<MB>, p, plan.cu);
+  }
+  return cudaLaunchKernelEx(&cfg, lut_gemv_kernel<MB>, p, plan.cu);
+}
+
+template <int MB>
+int max_active_clusters_mb(int C, size_t smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, lut_gemv_kernel<MB>, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+int max_active_clusters(int MB, int C, size_t smem) {
+  switch (MB) {
+    case 1: return max_active_clusters_mb<1>(C, smem);
+    case 2: return max_active_clusters_mb<2>(C, smem);
+    case 4: return max_active_clusters_mb<4>(C, smem);
+    case 8: return max_active_clusters_mb<8>(C, smem);
+    default: return 0;
+  }
+}
+
+size_t plan_smem(const Plan& pl, int CU, int n_sal) {
+  const int nsp = (n_sal + 3) & ~3;
+  const int msh = ((pl.max_tiles * 32 + pl.C - 1) / pl.C + 3) & ~3;
+  if (pl.kind == 0)
+    return wsmem_bytes(CU, pl.col_stride_bytes, pl.max_units, pl.max_lseg, pl.max_tiles, pl.MB, pl.C, n_sal);
+  return static_cast<size_t>(CU) * pl.col_stride_bytes + static_cast<size_t>(pl.max_units) * 128 * 4 +
+         static_cast<size_t>(pl.max_lseg) * pl.max_tiles * 32 * 4 + static_cast<size_t>(pl.max_tiles) * pl.MB * 32 * 4 +
+         static_cast<size_t>(pl.C) * pl.MB * msh * 4 + static_cast<size_t>(pl.MB) * nsp * 4 +
+         static_cast<size_t>(pl.max_units) * sizeof(UnitInfo);
 }
 
 }  // namespace
@@ -348,49 +935,44 @@ size_t query_smem_limit() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  return n > 0 ? static_cast<size_t>(n) - 1024 : 48 * 1024;
+  return n > 0 ? static_cast<size_t>(n) : 48 * 1024;
 }
 
-static size_t plan_smem(const Plan& pl, int n_sal) {
-  const int nsp = (n_sal + 3) & ~3;
-  return static_cast<size_t>(pl.max_cols) * pl.col_stride_bytes +
-         static_cast<size_t>(pl.max_cols) * pl.MB * 128 * 4 + static_cast<size_t>(pl.MB) * nsp * 4 +
-         static_cast<size_t>(2) * pl.MB * pl.G * 32 * 4;
-}
-
-static int max_cols_of(long long L, int P, int G) {
-  int mx = 0;
-  for (int c = 0; c < P; ++c) {
-    const long long b = static_cast<long long>(c) * L / P, e = static_cast<long long>(c + 1) * L / P;
-    if (e > b) mx = std::max(mx, static_cast<int>((e - 1) / G - b / G + 1));
-  }
-  return mx;
-}
-
-Plan make_plan(int rows, int units, int MB, int n_sal, int num_sms, size_t smem_limit) {
+Plan make_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, int num_sms,
+               size_t smem_limit) {
   Plan pl{};
   pl.MB = MB;
   const int tiles = (rows + 31) / 32;
-  int G = MB <= 2 ? 8 : (MB == 4 ? 16 : 32);
-  const int tiles4 = (tiles + kWarps - 1) / kWarps * kWarps;
-  G = std::max(kWarps, std::min(G, tiles4));
-  pl.G = G;
-  pl.nblocks = (tiles + G - 1) / G;
-  pl.L = static_cast<long long>(pl.nblocks) * units * G;
+  pl.C = std::max(1, std::min(kMaxCluster, units));
   pl.col_stride_bytes = (MB * kFields * kFieldStride * 4 + 127) / 128 * 128;
-  long long P = (pl.L + 7) / 8;
-  P = std::min<long long>(P, num_sms);
-  P = std::max<long long>(P, pl.nblocks);
-  P = std::min<long long>(P, pl.L);
-  pl.P = static_cast<int>(std::max<long long>(P, 1));
-  for (;;) {
-    pl.max_cols = max_cols_of(pl.L, pl.P, G);
-    pl.smem = plan_smem(pl, n_sal);
-    if (pl.smem <= smem_limit || pl.P >= pl.L) break;
-    pl.P = static_cast<int>(std::min<long long>(pl.L, static_cast<long long>(pl.P) * 2));
+  pl.max_units = (units + pl.C - 1) / pl.C;
+  auto seg_of = [&](int u) {
+    int s = 0;
+    for (int k = 1; k < nseg; ++k)
+      if (u >= seg_unit0[k]) s = k;
+    return s;
+  };
+  pl.max_lseg = 1;
+  for (int r = 0; r < pl.C; ++r) {
+    const int u0 = r * units / pl.C, u1 = (r + 1) * units / pl.C;
+    if (u1 > u0) pl.max_lseg = std::max(pl.max_lseg, seg_of(u1 - 1) - seg_of(u0) + 1);
   }
-  pl.part_floats = static_cast<size_t>(pl.P) * 2 * MB * G * 32;
-  pl.cnt_ints = static_cast<size_t>(pl.nblocks);
+  ensure_kernel_attrs();
+  // Clusters that fit with at most one CTA per SM (a CTA that shares its SM with
+  // another CTA of the same launch would take twice as long). The query uses a
+  // shared-memory size that forces one CTA per SM.
+  int fit = max_active_clusters(MB, pl.C, smem_limit / 2 + 1024);
+  if (fit <= 0) fit = std::max(1, num_sms / pl.C);
+  pl.ncl = std::max(1, std::min(tiles, fit));
+  pl.max_tiles = (tiles + pl.ncl - 1) / pl.ncl;
+  // units per table chunk: as many as fit; for the column-split kernel prefer a size
+  // that leaves room for a CTA of the next kernel on the same SM (PDL prefetch)
+  pl.kind = MB <= 2 ? 0 : 1;
+  pl.cu = pl.max_units;
+  if (pl.kind == 0)
+    while (pl.cu > 1 && plan_smem(pl, pl.cu, n_sal) > smem_limit / 2 - 2048) --pl.cu;
+  while (pl.cu > 1 && plan_smem(pl, pl.cu, n_sal) > smem_limit) --pl.cu;
+  pl.smem = plan_smem(pl, pl.cu, n_sal);
   return pl;
 }
 

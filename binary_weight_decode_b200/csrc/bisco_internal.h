@@ -10,19 +10,20 @@
 
 namespace bisco {
 
-constexpr int kWarps = 4;                 // warps per CTA
+constexpr int kWarps = 8;                 // warps per CTA
 constexpr int kThreads = kWarps * 32;
-constexpr int kFields = 26;               // 5-bit fields per 128-column quad: 25 of 5 bits + 1 of 3 bits
+constexpr int kFields = 26;               // fields per 128-column quad: 25 of 5 bits + 1 of 3 bits
 constexpr int kFieldStride = 36;          // floats from one field's 32-entry table to the next
 constexpr int kMaxSeg = 6;                // K <= 4 bases + the U^T segment (+ a spare)
 constexpr int kMaxBases = 4;
+constexpr int kMaxCluster = 8;            // CTAs per cluster (portable limit)
 constexpr int kMaxBatchChunk = 8;         // batch rows handled by one launch
 constexpr int kStatusBytes = 256;         // status word region at the start of the workspace
 
 // One segment of a pass: a packed sign matrix whose columns multiply one input vector.
 struct SegParam {
-  const uint4* bits;     // packed [tiles][nq][32][4] words, as uint4 per (row, quad)
-  const void* cscale;    // column scale [ncols] or nullptr
+  const uint4* bits;     // packed [tiles][nq][32][4] words, as one uint4 per (row, quad)
+  const void* cscale;    // column scale [ncols] or nullptr (= 1)
   const void* rscale;    // row scale [rows] or nullptr (= 1)
   int nq;                // quads per row = ceil(ncols / 128)
   int ncols;             // columns (input features) of this segment
@@ -30,45 +31,51 @@ struct SegParam {
   int xsrc;              // 0: X, 1: Z (fp32 workspace vector), 2: none (zeros)
   int cdt;               // dtype of cscale
   int rdt;               // dtype of rscale
+  int cvec, rvec;        // 1 if cscale / rscale are 16-byte aligned (vector loads allowed)
 };
 
-// One launch of the LUT GEMV kernel.
+// One launch of the cluster LUT GEMV kernel.
+//
+// Grid: ncl clusters of C CTAs. Cluster c owns row tiles [c*tiles/ncl, (c+1)*tiles/ncl);
+// CTA r of a cluster owns units (128-column quads over all segments)
+// [r*units/C, (r+1)*units/C) and builds lookup tables for them only. The C partial
+// sums of a row meet in distributed shared memory.
 struct PassParam {
   SegParam seg[kMaxSeg];
   int nseg;
   int rows;              // output rows of the pass
   int tiles;             // ceil(rows / 32)
   int units;             // total quads over segments
-  int G;                 // row tiles per block (multiple of kWarps)
-  int nblocks;           // ceil(tiles / G)
-  long long L;           // linear work items = nblocks * units * G
-  int P;                 // CTAs
+  int C;                 // CTAs per cluster
+  int ncl;               // clusters
+  int max_tiles;         // max row tiles of a cluster
+  int max_units;         // max units of a CTA
+  int max_lseg;          // max segments a CTA's unit range touches
   int Mc;                // valid batch rows in this launch (<= MB)
-  int max_cols;          // table slots per CTA (smem sizing)
-  int col_stride_bytes;  // bytes of tables per slot (multiple of 128)
+  int col_stride_bytes;  // bytes of tables per unit (multiple of 128)
   // activations
-  const void* X; int xdt; long long ldx;   // X[m][i] at X + m*ldx + i (elements)
+  const void* X; int xdt; int ldx;          // X[m][i] at X + m*ldx + i (elements)
   int xcols;             // columns of X (salient indices must be below it)
-  const float* Z; long long ldz;
+  const float* Z; int ldz;
+  int x_vec, z_vec;      // 1 if rows of X (resp. Z) allow 16-byte vector loads
   // output
-  void* Y; int ydt; long long ldy;
+  void* Y; int ydt; int ldy;
   // salient columns (added once per output row)
   int n_sal, sal_stride;
   const int* sal_idx; const int8_t* sal_q; const float* sal_scale;
-  // workspace
-  float* part;           // [P][2][MB][G*32]
-  int* cnt;              // [nblocks]
-  int* status;
+  int* status;           // device status word (workspace)
 };
 
 struct Plan {
-  int G, P, nblocks, max_cols, col_stride_bytes, MB;
-  long long L;
+  int C, ncl, max_tiles, max_units, max_lseg, col_stride_bytes, MB;
+  int cu;                // units per table chunk (kind 1) or table units per warp (kind 0)
+  int kind;              // 0: warps own units (batch rows <= 2); 1: warps own row tiles
   size_t smem;
-  size_t part_floats, cnt_ints;
 };
 
-Plan make_plan(int rows, int units, int MB, int n_sal, int num_sms, size_t smem_limit);
+// seg_unit0[k] = first unit of segment k (k < nseg); used to count segments per CTA.
+Plan make_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, int num_sms,
+               size_t smem_limit);
 cudaError_t launch_pass(const PassParam& p, const Plan& plan, cudaStream_t stream, bool pdl);
 // Sets per-kernel attributes once per device; call before any stream capture.
 cudaError_t ensure_kernel_attrs();
