@@ -3,7 +3,7 @@
 Argument marshalling only: every step of the computation runs in the CUDA
 library. PyTorch provides device memory and streams. Importing this package
 fails loudly if ``libbisco.so`` has not been built
-(``python -m binary_weight_decode_b200.build``).
+(``python binary_weight_decode_b200/build.py``).
 
 The functions carry the names of the C entry points in ``include/bisco.h``.
 """
@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbisco.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m binary_weight_decode_b200.build`")
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python binary_weight_decode_b200/build.py`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -26,7 +26,7 @@ BISCO_F32, BISCO_BF16 = 0, 1
 
 EXPORTED = [
     "bisco_packed_words", "bisco_pack", "bisco_unpack", "bisco_workspace_size", "bisco_workspace_init",
-    "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string",
+    "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string", "bisco_gemv_noalloc",
 ]
 
 
@@ -70,6 +70,9 @@ _lib.bisco_workspace_init.restype = ctypes.c_int
 _lib.bisco_gemv.argtypes = [ctypes.POINTER(bisco_layer), _P, ctypes.c_int32, ctypes.c_int32, _P, ctypes.c_int32,
                             _P, ctypes.c_size_t, _P]
 _lib.bisco_gemv.restype = ctypes.c_int
+_lib.bisco_gemv_noalloc.argtypes = [ctypes.POINTER(bisco_layer), _P, ctypes.c_int32, ctypes.c_int32, _P,
+                                    ctypes.c_int32, _P]
+_lib.bisco_gemv_noalloc.restype = ctypes.c_int
 _lib.bisco_sync_status.argtypes = [_P, _P]
 _lib.bisco_sync_status.restype = ctypes.c_int
 _lib.bisco_bench.argtypes = [ctypes.POINTER(bisco_bench_args), ctypes.POINTER(bisco_bench_result)]
@@ -216,6 +219,15 @@ def bisco_gemv(layer, X, Y, ws, stream=None):
                          ctypes.c_void_p(Y.data_ptr()), _dtype_code(Y), ctypes.c_void_p(ws.data_ptr()),
                          ws.numel() * ws.element_size(), _stream_ptr(stream))
     _check(st, "bisco_gemv")
+    return Y
+
+
+def bisco_gemv_noalloc(layer, X, Y, stream=None):
+    """bisco_gemv with the library's built-in scratch array instead of a workspace."""
+    M = X.shape[0] if X.dim() == 2 else 1
+    st = _lib.bisco_gemv_noalloc(ctypes.byref(_desc(layer)), ctypes.c_void_p(X.data_ptr()), _dtype_code(X), M,
+                                 ctypes.c_void_p(Y.data_ptr()), _dtype_code(Y), _stream_ptr(stream))
+    _check(st, "bisco_gemv_noalloc")
     return Y
 
 

@@ -1,6 +1,6 @@
 """Build libbisco.so in-tree with nvcc for sm_100a.
 
-    python -m binary_weight_decode_b200.build
+    python binary_weight_decode_b200/build.py
 """
 
 import os
@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbisco.so")
-SOURCES = ["bisco_gemv.cu", "bisco_api.cpp"]
+SOURCES = ["bisco_gemv.cu", "bisco_api.cpp", "bisco_noalloc.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -141,6 +141,34 @@ bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype
  */
 bisco_status bisco_sync_status(void* stream, const void* ws);
 
+/*
+ * Largest correction rank bisco_gemv_noalloc accepts.
+ */
+#define BISCO_NOALLOC_MAX_RANK 4096
+
+/*
+ * bisco_gemv without a caller-provided workspace. (There is no counterpart in the
+ * papers: this is a deployment convenience of this library.)
+ *
+ * For callers that cannot allocate device memory -- e.g. a plug-in inside a host
+ * application that owns all device allocations, or code running while a stream is
+ * captured into a CUDA graph, where a new allocation would break the capture. The
+ * scratch space (status word and the correction's intermediate z for one batch chunk)
+ * is a fixed array of 256 + 8 * 4096 * 4 bytes in the library's device image; every GPU
+ * that loads the library keeps it until the process exits. This call allocates nothing.
+ *
+ * Arguments and results are those of bisco_gemv, minus the workspace. Layers with
+ * rank > BISCO_NOALLOC_MAX_RANK are rejected with BISCO_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
+ * make that first call before any stream capture starts.
+ * All calls share the one array: calls that may overlap on the GPU (different streams,
+ * or different host threads) race with each other; order them on one stream.
+ * Device-side errors are recorded in the shared array and cannot be read back through
+ * this entry point (use bisco_gemv with a workspace when that check matters).
+ */
+bisco_status bisco_gemv_noalloc(const bisco_layer* layer, const void* X, int32_t x_dtype, int32_t M,
+                                void* Y, int32_t y_dtype, void* stream);
+
 /* Benchmark request: a stream of n_layers GEMVs (distinct weight copies) captured
  * in one CUDA graph and replayed. */
 typedef struct {
