@@ -68,8 +68,10 @@ struct PassParam {
 
 struct Plan {
   int C, ncl, max_tiles, max_units, max_lseg, col_stride_bytes, MB;
-  int cu;                // units per table chunk (kind 1) or table units per warp (kind 0)
-  int kind;              // 0: warps own units (batch rows <= 2); 1: warps own row tiles
+  int cu;                // units per table chunk
+  int kind;              // 0: 16-warp kernel, 2: streaming kernel (batch rows <= 2); 1: warps own row tiles (4, 8)
+  int ns;                // streaming kernel: shared-memory ring slots (one (chunk, tile) stage each)
+  int gu;                // streaming kernel: unit groups of the 16 consumer warps
   size_t smem;
 };
 
