@@ -2,10 +2,15 @@
 // two-pass launch sequence of bisco_gemv.
 //
 // A layer with a binary low-rank correction ("BiLoCo", "The core idea": the
-// correction is applied as alpha * u * (v . x)) runs as two launches of the same
-// lookup-table kernel: pass Z computes z = alpha (.) (V x) into the workspace,
-// pass Y computes sum_k r_k (.) (B_k (c_k (.) x)) + U^T z + salient term into Y.
-// Pass Y reads z only after griddepcontrol.wait, i.e. after pass Z completed.
+// correction is applied as alpha * u * (v . x)) runs as two launches: pass Z computes
+// z = alpha (.) (V x) into the workspace, pass Y computes
+// sum_k r_k (.) (B_k (c_k (.) x)) + U^T z + salient term into Y. Pass Y reads z only
+// after griddepcontrol.wait, i.e. after pass Z completed.
+//
+// The batch is cut into chunks: up to 128 rows per launch on the tensor-core path
+// when a chunk has at least 16 rows (and the scales are bf16, so that folding a column
+// scale into the expanded signs is exact), otherwise up to 8 rows per launch on the
+// lookup-table kernels.
 
 #include <cuda_runtime.h>
 
@@ -122,8 +127,14 @@ Layout cached_layout(const bisco_layer* L, int MB, int dev) {
 }
 
 // Workspace bytes: the status word and, with a correction, z for one batch chunk.
+// ws_need is the minimum bisco_gemv accepts (chunks of 8 rows); ws_pref also lets the
+// tensor-core path take chunks of up to 128 rows for this batch size.
 size_t ws_need(const bisco_layer* L, int32_t) {
   return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
+}
+size_t ws_pref(const bisco_layer* L, int32_t M) {
+  const int rows = std::max(kMaxBatchChunk, std::min<int>(M, kTcMaxBatch));
+  return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(rows) * L->rank * 4 : 0);
 }
 
 bool plans_fit(const Layout& lo, size_t lim) {
@@ -133,6 +144,170 @@ bool plans_fit(const Layout& lo, size_t lim) {
 void fill_plan(PassParam& P, const Plan& pl) {
   P.C = pl.C; P.ncl = pl.ncl; P.max_tiles = pl.max_tiles; P.max_units = pl.max_units;
   P.max_lseg = pl.max_lseg; P.col_stride_bytes = pl.col_stride_bytes;
+}
+
+
+// Segments of pass Z: V (rows = rank) over X, row scale alpha.
+void pass_z(const bisco_layer* L, PassParam& pz, const void* Xc, int32_t x_dtype, int Mc, float* zbuf, int* status) {
+  const size_t xb = dtype_bytes(x_dtype);
+  pz.nseg = 1;
+  SegParam& V = pz.seg[0];
+  V.bits = reinterpret_cast<const uint4*>(L->v_bits);
+  V.nq = quads(L->in);
+  V.ncols = L->in;
+  V.unit0 = 0;
+  V.xsrc = 0;
+  V.cscale = nullptr;
+  V.cdt = BISCO_F32;
+  V.rscale = L->alpha;
+  V.rdt = BISCO_F32;
+  V.cvec = 0;
+  V.rvec = aligned16(L->alpha);
+  pz.rows = L->rank;
+  pz.tiles = (L->rank + 31) / 32;
+  pz.units = V.nq;
+  pz.Mc = Mc;
+  pz.X = Xc; pz.xdt = x_dtype; pz.ldx = L->in; pz.xcols = L->in;
+  pz.Z = nullptr; pz.ldz = 0;
+  pz.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
+  pz.z_vec = 0;
+  pz.Y = zbuf; pz.ydt = BISCO_F32; pz.ldy = L->rank;
+  pz.n_sal = 0; pz.sal_stride = 0;
+  pz.status = status;
+}
+
+// Segments of pass Y: the K binary bases over c_k (.) X, then U^T over z; a layer with
+// neither gets one empty unit so that the salient term still has a home.
+void pass_y(const bisco_layer* L, PassParam& py, const void* Xc, int32_t x_dtype, int Mc, void* Yc, int32_t y_dtype,
+            float* zbuf, int* status) {
+  const size_t xb = dtype_bytes(x_dtype);
+  int nseg = 0, unit = 0;
+  for (int k = 0; k < L->num_bases; ++k) {
+    SegParam& B = py.seg[nseg++];
+    B.bits = reinterpret_cast<const uint4*>(L->bits + static_cast<size_t>(k) * bisco_packed_words(L->out, L->in));
+    B.nq = quads(L->in);
+    B.ncols = L->in;
+    B.unit0 = unit;
+    unit += B.nq;
+    B.xsrc = 0;
+    B.cscale = static_cast<const unsigned char*>(L->col_scale) + static_cast<size_t>(k) * L->in * dtype_bytes(L->scale_dtype);
+    B.cdt = L->scale_dtype;
+    B.rscale = static_cast<const unsigned char*>(L->row_scale) + static_cast<size_t>(k) * L->out * dtype_bytes(L->scale_dtype);
+    B.rdt = L->scale_dtype;
+    B.cvec = aligned16(B.cscale);
+    B.rvec = aligned16(B.rscale);
+  }
+  if (L->rank > 0) {
+    SegParam& U = py.seg[nseg++];
+    U.bits = reinterpret_cast<const uint4*>(L->ut_bits);
+    U.nq = quads(L->rank);
+    U.ncols = L->rank;
+    U.unit0 = unit;
+    unit += U.nq;
+    U.xsrc = 1;
+    U.cscale = nullptr;
+    U.cdt = BISCO_F32;
+    U.rscale = nullptr;
+    U.rdt = BISCO_F32;
+    U.cvec = U.rvec = 0;
+  }
+  if (nseg == 0) {  // salient-only (or empty) layer: one empty unit
+    SegParam& E = py.seg[nseg++];
+    E.bits = nullptr; E.nq = 1; E.ncols = 0; E.unit0 = 0; E.xsrc = 2;
+    E.cscale = nullptr; E.rscale = nullptr; E.cdt = E.rdt = BISCO_F32;
+    E.cvec = E.rvec = 0;
+    unit = 1;
+  }
+  py.nseg = nseg;
+  py.rows = L->out;
+  py.tiles = (L->out + 31) / 32;
+  py.units = unit;
+  py.Mc = Mc;
+  py.X = Xc; py.xdt = x_dtype; py.ldx = L->in; py.xcols = L->in;
+  py.Z = zbuf; py.ldz = L->rank;
+  py.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
+  py.z_vec = (L->rank % 4) == 0;
+  py.Y = Yc; py.ydt = y_dtype; py.ldy = L->out;
+  py.n_sal = L->n_sal; py.sal_stride = L->sal_stride;
+  py.sal_idx = L->sal_idx; py.sal_q = L->sal_q; py.sal_scale = L->sal_scale;
+  py.status = status;
+}
+
+// One batch chunk and how it runs.
+struct Chunk {
+  int m0, Mc;
+  bool tc;
+  Layout lo;       // lookup-table plans (tc == false)
+  TcPlan tz, ty;   // tensor-core plans (tc == true)
+};
+
+// Tensor-core plans for a chunk of Mc rows, cached like the lookup-table layouts.
+bool tc_plans(const bisco_layer* L, int Mc, int32_t x_dtype, int dev, TcPlan* tz, TcPlan* ty) {
+  struct Key {
+    int dev, out, in, K, rank, n_sal, Np, xdt;
+    bool operator==(const Key& o) const {
+      return dev == o.dev && out == o.out && in == o.in && K == o.K && rank == o.rank && n_sal == o.n_sal &&
+             Np == o.Np && xdt == o.xdt;
+    }
+  };
+  struct Entry { Key k; TcPlan z, y; };
+  static std::mutex mu;
+  static std::vector<Entry>* cache = new std::vector<Entry>();
+  const Key k{dev, L->out, L->in, L->num_bases, L->rank, L->n_sal, (Mc + 15) / 16 * 16, x_dtype};
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (const Entry& e : *cache)
+      if (e.k == k) { *tz = e.z; *ty = e.y; return ty->S > 0 && (L->rank == 0 || tz->S > 0); }
+  }
+  const int sms = cached_sms(dev);
+  const size_t lim = cached_smem_limit(dev);
+  const bool xbf = x_dtype == BISCO_BF16;
+  TcPlan z{}, y{};
+  if (L->rank > 0) {
+    const int kind = 0, ncols = L->in;
+    z = make_tc_plan(L->rank, 1, &kind, &ncols, 0, xbf, Mc, sms, lim);
+  }
+  int kinds[kMaxSeg], ncols[kMaxSeg], nseg = 0;
+  for (int b = 0; b < L->num_bases; ++b) { kinds[nseg] = 0; ncols[nseg++] = L->in; }
+  if (L->rank > 0) { kinds[nseg] = 1; ncols[nseg++] = L->rank; }
+  if (nseg == 0) { kinds[nseg] = 2; ncols[nseg++] = 0; }
+  y = make_tc_plan(L->out, nseg, kinds, ncols, L->n_sal, xbf, Mc, sms, lim);
+  std::lock_guard<std::mutex> g(mu);
+  if (cache->size() > 4096) cache->clear();
+  cache->push_back(Entry{k, z, y});
+  *tz = z;
+  *ty = y;
+  return y.S > 0 && (L->rank == 0 || z.S > 0);
+}
+
+// Batch chunks of a call: tensor-core chunks where possible, lookup-table chunks of at
+// most 8 rows otherwise.
+bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws_bytes, int dev, std::vector<Chunk>* out) {
+  const size_t lim = cached_smem_limit(dev);
+  // rows the workspace can hold z for (the tensor-core path needs one chunk's z)
+  int tc_rows = kTcMaxBatch;
+  if (L->rank > 0) {
+    const size_t fit = (ws_bytes - kStatusBytes) / (static_cast<size_t>(L->rank) * 4);
+    tc_rows = static_cast<int>(std::min<size_t>(kTcMaxBatch, fit / 16 * 16));
+  }
+  const bool tc_ok = (L->num_bases == 0 || L->scale_dtype == BISCO_BF16) && tc_rows >= kTcMinBatch;
+  for (int m0 = 0; m0 < M;) {
+    Chunk ch{};
+    ch.m0 = m0;
+    const int rem = M - m0;
+    if (tc_ok && rem >= kTcMinBatch) {
+      ch.Mc = std::min(rem, tc_rows);
+      ch.tc = tc_plans(L, ch.Mc, x_dtype, dev, &ch.tz, &ch.ty);
+    }
+    if (!ch.tc) {
+      ch.Mc = std::min(kMaxBatchChunk, rem);
+      ch.lo = cached_layout(L, batch_block(ch.Mc), dev);
+      if (!plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
+    }
+    out->push_back(ch);
+    m0 += ch.Mc;
+  }
+  return BISCO_OK;
 }
 
 }  // namespace
@@ -185,7 +360,7 @@ bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* b
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
   (void)dev;
-  *bytes = ws_need(layer, M);
+  *bytes = ws_pref(layer, M);
   return BISCO_OK;
 }
 
@@ -206,112 +381,33 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
   if (ws_bytes < ws_need(L, M)) return BISCO_ERR_WORKSPACE;
-  const size_t lim = cached_smem_limit(dev);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   unsigned char* wsb = static_cast<unsigned char*>(ws);
   const size_t xb = dtype_bytes(x_dtype), yb = dtype_bytes(y_dtype);
 
   // Every launch is planned before the first one is issued, so an unsupported
   // request fails without touching any output.
-  std::vector<Layout> los;
-  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
-    const int Mc = std::min(kMaxBatchChunk, M - m0);
-    los.push_back(cached_layout(L, batch_block(Mc), dev));
-    if (!plans_fit(los.back(), lim)) return BISCO_ERR_UNSUPPORTED;
-  }
+  std::vector<Chunk> chunks;
+  st = plan_chunks(L, M, x_dtype, ws_bytes, dev, &chunks);
+  if (st != BISCO_OK) return st;
 
-  int chunk = 0;
-  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk, ++chunk) {
-    const int Mc = std::min(kMaxBatchChunk, M - m0);
-    const Layout& lo = los[chunk];
-    int* status = reinterpret_cast<int*>(wsb);
-    float* zbuf = reinterpret_cast<float*>(wsb + lo.off_z);
-    const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(m0) * L->in * xb;
-    void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(m0) * L->out * yb;
-
-    if (lo.has_z) {
-      PassParam pz{};
-      pz.nseg = 1;
-      SegParam& V = pz.seg[0];
-      V.bits = reinterpret_cast<const uint4*>(L->v_bits);
-      V.nq = quads(L->in);
-      V.ncols = L->in;
-      V.unit0 = 0;
-      V.xsrc = 0;
-      V.cscale = nullptr;
-      V.cdt = BISCO_F32;
-      V.rscale = L->alpha;
-      V.rdt = BISCO_F32;
-      V.cvec = 0;
-      V.rvec = aligned16(L->alpha);
-      pz.rows = L->rank;
-      pz.tiles = (L->rank + 31) / 32;
-      pz.units = V.nq;
-      fill_plan(pz, lo.pz);
-      pz.Mc = Mc;
-      pz.X = Xc; pz.xdt = x_dtype; pz.ldx = L->in; pz.xcols = L->in;
-      pz.Z = nullptr; pz.ldz = 0;
-      pz.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
-      pz.z_vec = 0;
-      pz.Y = zbuf; pz.ydt = BISCO_F32; pz.ldy = L->rank;
-      pz.n_sal = 0; pz.sal_stride = 0;
-      pz.status = status;
-      if (launch_pass(pz, lo.pz, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
-    }
-
-    PassParam py{};
-    int nseg = 0, unit = 0;
-    for (int k = 0; k < L->num_bases; ++k) {
-      SegParam& B = py.seg[nseg++];
-      B.bits = reinterpret_cast<const uint4*>(L->bits + static_cast<size_t>(k) * bisco_packed_words(L->out, L->in));
-      B.nq = quads(L->in);
-      B.ncols = L->in;
-      B.unit0 = unit;
-      unit += B.nq;
-      B.xsrc = 0;
-      B.cscale = static_cast<const unsigned char*>(L->col_scale) + static_cast<size_t>(k) * L->in * dtype_bytes(L->scale_dtype);
-      B.cdt = L->scale_dtype;
-      B.rscale = static_cast<const unsigned char*>(L->row_scale) + static_cast<size_t>(k) * L->out * dtype_bytes(L->scale_dtype);
-      B.rdt = L->scale_dtype;
-      B.cvec = aligned16(B.cscale);
-      B.rvec = aligned16(B.rscale);
-    }
+  int* status = reinterpret_cast<int*>(wsb);
+  float* zbuf = reinterpret_cast<float*>(wsb + kStatusBytes);
+  for (const Chunk& ch : chunks) {
+    const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(ch.m0) * L->in * xb;
+    void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(ch.m0) * L->out * yb;
     if (L->rank > 0) {
-      SegParam& U = py.seg[nseg++];
-      U.bits = reinterpret_cast<const uint4*>(L->ut_bits);
-      U.nq = quads(L->rank);
-      U.ncols = L->rank;
-      U.unit0 = unit;
-      unit += U.nq;
-      U.xsrc = 1;
-      U.cscale = nullptr;
-      U.cdt = BISCO_F32;
-      U.rscale = nullptr;
-      U.rdt = BISCO_F32;
-      U.cvec = U.rvec = 0;
+      PassParam pz{};
+      pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);
+      if (!ch.tc) fill_plan(pz, ch.lo.pz);
+      const cudaError_t e = ch.tc ? launch_tc(pz, ch.tz, s) : launch_pass(pz, ch.lo.pz, s, true);
+      if (e != cudaSuccess) return BISCO_ERR_CUDA;
     }
-    if (nseg == 0) {  // salient-only (or empty) layer: one empty unit
-      SegParam& E = py.seg[nseg++];
-      E.bits = nullptr; E.nq = 1; E.ncols = 0; E.unit0 = 0; E.xsrc = 2;
-      E.cscale = nullptr; E.rscale = nullptr; E.cdt = E.rdt = BISCO_F32;
-      E.cvec = E.rvec = 0;
-      unit = 1;
-    }
-    py.nseg = nseg;
-    py.rows = L->out;
-    py.tiles = (L->out + 31) / 32;
-    py.units = unit;
-    fill_plan(py, lo.py);
-    py.Mc = Mc;
-    py.X = Xc; py.xdt = x_dtype; py.ldx = L->in; py.xcols = L->in;
-    py.Z = zbuf; py.ldz = L->rank;
-    py.x_vec = aligned16(Xc) && (static_cast<size_t>(L->in) * xb) % 16 == 0;
-    py.z_vec = (L->rank % 4) == 0;
-    py.Y = Yc; py.ydt = y_dtype; py.ldy = L->out;
-    py.n_sal = L->n_sal; py.sal_stride = L->sal_stride;
-    py.sal_idx = L->sal_idx; py.sal_q = L->sal_q; py.sal_scale = L->sal_scale;
-    py.status = status;
-    if (launch_pass(py, lo.py, s, true) != cudaSuccess) return BISCO_ERR_CUDA;
+    PassParam py{};
+    pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
+    if (!ch.tc) fill_plan(py, ch.lo.py);
+    const cudaError_t e = ch.tc ? launch_tc(py, ch.ty, s) : launch_pass(py, ch.lo.py, s, true);
+    if (e != cudaSuccess) return BISCO_ERR_CUDA;
   }
   return BISCO_OK;
 }
@@ -338,7 +434,14 @@ bisco_status bisco_bench(const bisco_bench_args* a, bisco_bench_result* r) {
   for (int i = 0; i < a->n_layers; ++i)
     if (a->ws_bytes < ws_need(&a->layers[i], a->M)) return BISCO_ERR_WORKSPACE;
 
-  if (ensure_kernel_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
+  if (ensure_kernel_attrs() != cudaSuccess || tc_ensure_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
+  int launches = 0;
+  {
+    std::vector<Chunk> chunks;
+    const bisco_status st = plan_chunks(&a->layers[0], a->M, a->x_dtype, a->ws_bytes, dev, &chunks);
+    if (st != BISCO_OK) return st;
+    launches = static_cast<int>(chunks.size()) * (a->layers[0].rank > 0 ? 2 : 1);
+  }
   cudaStream_t user = static_cast<cudaStream_t>(a->stream);
   cudaStream_t cs = nullptr;
   cudaGraph_t graph = nullptr;
@@ -382,8 +485,7 @@ bisco_status bisco_bench(const bisco_bench_args* a, bisco_bench_result* r) {
     if (result == BISCO_OK && cudaEventElapsedTime(&ms, e0, e1) == cudaSuccess) {
       r->us_per_replay = ms * 1000.0 / a->reps;
       r->us_per_gemv = r->us_per_replay / a->n_layers;
-      const int chunks = (a->M + kMaxBatchChunk - 1) / kMaxBatchChunk;
-      r->kernels_per_gemv = chunks * (a->layers[0].rank > 0 ? 2 : 1);
+      r->kernels_per_gemv = launches;
     } else {
       fail(BISCO_ERR_CUDA);
     }

@@ -85,4 +85,21 @@ cudaError_t ensure_kernel_attrs();
 int query_num_sms();
 size_t query_smem_limit();
 
+// Tensor-core path (16..128 batch rows per launch): one launch per pass.
+constexpr int kTcMinBatch = 32;           // smallest batch chunk sent to the tensor cores
+constexpr int kTcMaxBatch = 64;           // batch rows per launch (three pipeline stages fit)
+struct TcPlan {
+  int Np;                // batch rows padded to a multiple of 16 (MMA N per part)
+  int tmem_cols;         // tensor-memory columns allocated per CTA
+  int stages;            // shared-memory stages
+  int tiles;             // 128-row output tiles (clusters)
+  int S;                 // CTAs per cluster (K split); 0 = plan not possible
+  size_t smem;
+};
+// seg_kind[s] is SegParam::xsrc of segment s; seg_ncols[s] its columns.
+TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncols, int n_sal, bool x_bf16, int Mc,
+                    int num_sms, size_t smem_limit);
+cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream);
+cudaError_t tc_ensure_attrs();
+
 }  // namespace bisco

@@ -1,0 +1,650 @@
+// Tensor-core path for larger batches (16 to 64 batch rows per launch).
+//
+// With many batch rows the product is a dense contraction: for each segment,
+//   D_seg[o][m] = sum_i A_seg[o][i] * B_seg[i][m].
+// The signs are expanded in shared memory into bf16 tiles and multiplied on the
+// 5th-generation tensor cores (tcgen05.mma, kind::f16, fp32 accumulators in tensor
+// memory):
+//   * a binary base k: A = +-c_k[i] (the column scale folded into the sign; exact in
+//     bf16 because the scales are bf16), B = X (exact for bf16 activations; fp32
+//     activations are split into bf16 high and low parts). Each base has its own
+//     accumulator, and its row scale r_k is applied in the epilogue ("FluxBin",
+//     Sec. 3.1, decoupled row-column binary bases);
+//   * the correction's U^T: A = +-1, B = z split into high and low parts
+//     ("BiLoCo", "The core idea": the second factor u applied to z = alpha (.) (V x));
+//   * the salient columns: A = q (int8 values, exact in bf16), B = s_t * x[idx_t]
+//     split the same way ("BiSCo-LLM", Sensitivity Protection). U^T and the salient
+//     columns share one accumulator (no row scale);
+//   * the correction's first phase z = alpha (.) (V x): A = +-1, B = X, alpha applied
+//     in the epilogue as V's row scale.
+// Every product is exact in fp32 and the sums are fp32, as on the CUDA-core path; a
+// split value keeps 16 significant bits of its fp32 value.
+//
+// Work decomposition: cluster c owns 128 output rows; CTA r of the cluster takes 1/S of
+// the (segment, 128-column K tile) steps. A step's tiles live in a shared-memory stage,
+// K-major with the 128-byte swizzle: each tile is two blocks of 64 columns; a row of a
+// block is 128 bytes, its 16-byte chunks permuted by XOR with (row mod 8), and groups
+// of 8 rows are 1024 bytes apart. The loop is software-pipelined: while step i is
+// expanded, cp.async brings in the raw sign words and column scales of step i + 2 (a
+// four-slot ring) and the bf16 activation tile of step i + 1 (straight into its stage,
+// once the MMAs that last read that stage are done). Eight warps expand step i's signs
+// from shared memory; one thread issues the step's eight K=16 MMAs and commits them to
+// the stage's mbarrier. The S partial results meet in distributed shared memory and are
+// added in CTA-rank order.
+// A CTA takes more than half of an SM's shared memory, so no two CTAs (each holding up
+// to 512 tensor-memory columns) ever share an SM.
+
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "bisco_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace bisco {
+
+namespace {
+
+constexpr int kTcWarps = 8;
+constexpr int kTcThreads = kTcWarps * 32;
+constexpr int kTcRows = 128;       // output rows per cluster (MMA M)
+constexpr int kTcK = 128;          // input columns per step (eight K=16 MMAs)
+constexpr int kTcMaxStages = 3;
+constexpr int kTcRawSlots = 4;     // raw sign-word / column-scale ring (prefetch distance 2)
+constexpr int kTcRawBytes = kTcRows * 16 + kTcK * 2;  // 128 rows x 16 bytes + 128 bf16 scales
+constexpr int kTcMaxBlocks = kMaxSeg + 1;
+constexpr unsigned long long kTcWaitNs = 200000000ull;  // bound on every wait (200 ms)
+
+__device__ __forceinline__ unsigned saddr(const void* p) { return static_cast<unsigned>(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ unsigned long long tc_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool tc_try(uint64_t* b, unsigned parity) {
+  unsigned done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(saddr(b)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Waits (bounded in time) until the phase with the given parity has completed.
+__device__ __forceinline__ bool tc_wait(uint64_t* b, unsigned parity) {
+  if (tc_try(b, parity)) return true;
+  const unsigned long long end = tc_ns() + kTcWaitNs;
+  while (!tc_try(b, parity))
+    if (tc_ns() > end) return false;
+  return true;
+}
+
+// Shared-memory matrix descriptor, K-major with the 128-byte swizzle: start address
+// (16-byte units), leading byte offset 1 (unused by this layout), stride byte offset
+// 1024 (8 rows of 128 bytes), descriptor version 1 (bits 46-47), layout 2 = 128-byte
+// swizzle (bits 61-63). A K step of 16 elements inside a 64-column block starts 32
+// bytes further; the hardware applies the swizzle to the address bits.
+__device__ __forceinline__ uint64_t smem_desc_sw128(const void* start) {
+  const uint64_t a = (saddr(start) >> 4) & 0x3FFFu;
+  return a | (1ull << 16) | (static_cast<uint64_t>(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), bf16 A and B
+// (bits 7-9 and 10-12 = 1), both K-major, N >> 3 at bit 17, M >> 4 at bit 24 (M = 128).
+__device__ __forceinline__ uint32_t mma_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(kTcRows >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* b) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(saddr(b)) : "memory");
+}
+
+// Byte offset of the 16-byte chunk (row, k8) (columns 8 k8 .. 8 k8 + 7) in a tile of
+// `rows` rows and 128 columns (two 64-column blocks, 128-byte swizzle).
+__device__ __forceinline__ unsigned tile_off(int row, int k8, int rows) {
+  return (k8 >> 3) * static_cast<unsigned>(rows) * 128u + row * 128u + (((k8 & 7) ^ (row & 7)) << 4);
+}
+
+// 16-byte cp.async with zero fill past src_bytes (0..16).
+__device__ __forceinline__ void cp16(void* dst, const void* src, unsigned src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+__device__ __forceinline__ unsigned pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const unsigned*>(&h);
+}
+
+__device__ __forceinline__ float x_at(const PassParam& p, int m, long long col) {
+  const long long i = static_cast<long long>(m) * p.ldx + col;
+  return p.xdt == BISCO_BF16 ? __uint_as_float(static_cast<unsigned>(__ldcg(reinterpret_cast<const unsigned short*>(p.X) + i)) << 16)
+                             : __ldcg(reinterpret_cast<const float*>(p.X) + i);
+}
+
+// Segment kinds of the tensor-core pass (the salient columns form one extra segment).
+enum { kSegX = 0, kSegZ = 1, kSegSal = 3 };
+
+struct TcSeg {
+  const uint4* bits;
+  const void* cscale;
+  int nq, ncols, kind, cvec;
+};
+
+__device__ __forceinline__ TcSeg tc_seg(const PassParam& p, int s) {
+  TcSeg g;
+  if (s < p.nseg) {
+    const SegParam& G = p.seg[s];
+    g.bits = G.bits; g.cscale = G.cscale; g.nq = G.nq; g.ncols = G.ncols; g.kind = G.xsrc; g.cvec = G.cvec;
+  } else {
+    g.bits = nullptr; g.cscale = nullptr; g.nq = 0; g.ncols = p.n_sal; g.kind = kSegSal; g.cvec = 0;
+  }
+  return g;
+}
+
+// 16 bytes of a B tile: columns c..c+7 of batch row m (part 0: the value or its high
+// bf16 part; part 1: the low part).
+__device__ __forceinline__ uint4 b_chunk(const PassParam& p, const TcSeg& g, int m, int c, int part, int split) {
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = 0.f;
+  if (m < p.Mc) {
+    const int valid = max(0, min(8, g.ncols - c));
+    if (g.kind == kSegSal) {
+      for (int j = 0; j < valid; ++j) {
+        const int cc = __ldg(p.sal_idx + c + j);
+        if (cc >= 0 && cc < p.xcols) v[j] = x_at(p, m, cc) * __ldg(p.sal_scale + c + j);
+        else if (part == 0) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+      }
+    } else if (g.kind == kSegX) {
+      if (p.xdt == BISCO_BF16 && split == 1 && p.x_vec && valid == 8)
+        return __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(p.X) + static_cast<long long>(m) * p.ldx + c));
+      for (int j = 0; j < valid; ++j) v[j] = x_at(p, m, c + j);
+    } else if (g.kind == kSegZ) {
+      for (int j = 0; j < valid; ++j) v[j] = __ldcg(p.Z + static_cast<long long>(m) * p.ldz + c + j);
+    }
+  }
+  if (split == 2) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float hi = __bfloat162float(__float2bfloat16_rn(v[j]));
+      v[j] = part == 0 ? hi : v[j] - hi;
+    }
+  }
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+}
+
+// 16 bytes of an A tile: columns c..c+7 of output row o.
+__device__ __forceinline__ uint4 a_chunk(const PassParam& p, const TcSeg& g, int o, int c) {
+  if (o >= p.rows || c >= g.ncols || (g.kind != kSegSal && g.bits == nullptr)) return make_uint4(0u, 0u, 0u, 0u);
+  const int valid = min(8, g.ncols - c);
+  if (g.kind == kSegSal) {  // q[o][t] as bf16
+    const int8_t* q = p.sal_q + static_cast<long long>(o) * p.sal_stride + c;
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = j < valid ? static_cast<float>(q[j]) : 0.f;
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+  }
+  // sign byte of columns c..c+7 from the packed layout (c is a multiple of 8)
+  const unsigned* words = reinterpret_cast<const unsigned*>(g.bits + (static_cast<long long>(o >> 5) * g.nq + (c >> 7)) * 32 + (o & 31));
+  const unsigned byte = (__ldg(words + ((c >> 5) & 3)) >> (c & 31)) & 0xFFu;
+  // column scales as bf16 bits (1.0 without scales), zero past the segment's columns
+  unsigned cs[4];
+  if (g.cscale == nullptr) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) cs[e] = (2 * e < valid ? 0x3F80u : 0u) | ((2 * e + 1 < valid ? 0x3F80u : 0u) << 16);
+  } else if (g.cvec && valid == 8) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(g.cscale) + c));
+    cs[0] = v.x; cs[1] = v.y; cs[2] = v.z; cs[3] = v.w;
+  } else {
+    const unsigned short* cp = reinterpret_cast<const unsigned short*>(g.cscale) + c;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      cs[e] = (2 * e < valid ? static_cast<unsigned>(__ldg(cp + 2 * e)) : 0u) |
+              ((2 * e + 1 < valid ? static_cast<unsigned>(__ldg(cp + 2 * e + 1)) : 0u) << 16);
+  }
+  // a clear bit is the sign -1: set the bf16 sign bit
+  unsigned w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const unsigned nb = ~(byte >> (2 * e));
+    w[e] = cs[e] ^ (((nb & 1u) << 15) | ((nb & 2u) << 30));
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Expands columns 64h .. 64h+63 of row r of a step from the raw ring slot: 64 sign bits
+// and the step's 128 column scales (bf16 bits; 1.0 when the segment has none, 0 past its
+// columns). A clear bit is the sign -1: the bf16 sign bit is set.
+__device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* raw, int r, int h, int ncols_left,
+                                         bool has_cscale) {
+  const uint4 bw = *reinterpret_cast<const uint4*>(raw + r * 16);
+  const unsigned lo = h ? bw.z : bw.x, hi = h ? bw.w : bw.y;
+  const unsigned short* cs = reinterpret_cast<const unsigned short*>(raw + kTcRows * 16);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int k8 = 8 * h + j;
+    const unsigned byte = ((j < 4 ? lo : hi) >> (8 * (j & 3))) & 0xFFu;
+    unsigned c[4];
+    if (has_cscale) {
+      const uint4 cv = *reinterpret_cast<const uint4*>(cs + 8 * k8);
+      c[0] = cv.x; c[1] = cv.y; c[2] = cv.z; c[3] = cv.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        c[e] = (8 * k8 + 2 * e < ncols_left ? 0x3F80u : 0u) | ((8 * k8 + 2 * e + 1 < ncols_left ? 0x3F80u : 0u) << 16);
+    }
+    unsigned w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const unsigned nb = ~(byte >> (2 * e));
+      w[e] = c[e] ^ (((nb & 1u) << 15) | ((nb & 2u) << 30));
+    }
+    *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Accumulator blocks in tensor memory: one per X segment (row scale applied in the
+// epilogue), one shared by U^T and the salient columns.
+struct TcAcc {
+  int nblk;
+  int col[kTcMaxBlocks];    // first column
+  int split[kTcMaxBlocks];  // 1 or 2 parts of Np columns
+  int rseg[kTcMaxBlocks];   // segment whose row scale applies (-1: none)
+  int blk_of_seg[kTcMaxBlocks];
+  int ncols;
+};
+
+__host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, bool has_sal, bool x_bf16, int Np) {
+  TcAcc a{};
+  int shared = -1, col = 0;
+  for (int s = 0; s < nseg + (has_sal ? 1 : 0); ++s) {
+    const int kind = s < nseg ? seg_kind[s] : kSegSal;
+    if (kind == kSegX) {
+      const int b = a.nblk++;
+      a.col[b] = col;
+      a.split[b] = x_bf16 ? 1 : 2;
+      a.rseg[b] = s;
+      col += a.split[b] * Np;
+      a.blk_of_seg[s] = b;
+    } else {
+      if (shared < 0) {
+        shared = a.nblk++;
+        a.col[shared] = col;
+        a.split[shared] = 2;
+        a.rseg[shared] = -1;
+        col += 2 * Np;
+      }
+      a.blk_of_seg[s] = shared;
+    }
+  }
+  a.ncols = col;
+  return a;
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ PassParam p, const int S, const int Np, const int nstages, const int tmem_cols) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int o0 = (blockIdx.x / S) * kTcRows;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has_sal = p.n_sal > 0;
+  const int nseg_all = p.nseg + (has_sal ? 1 : 0);
+  int kinds[kMaxSeg];
+  for (int s = 0; s < kMaxSeg; ++s) kinds[s] = s < p.nseg ? p.seg[s].xsrc : kSegZ;
+  const TcAcc acc = tc_acc(p.nseg, kinds, has_sal, p.xdt == BISCO_BF16, Np);
+  const unsigned a_bytes = kTcRows * kTcK * 2, b_bytes = static_cast<unsigned>(2 * Np) * kTcK * 2;
+  const unsigned stage_bytes = a_bytes + b_bytes;
+
+  uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem);   // [kTcMaxStages]
+  uint64_t* all_done = mma_done + kTcMaxStages;             // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(all_done + 1);
+  unsigned char* raw_ring = smem + 1024;                    // [kTcRawSlots][kTcRawBytes]
+  unsigned char* stages = raw_ring + kTcRawSlots * kTcRawBytes;
+  float* recv = reinterpret_cast<float*>(stages);           // used after the main loop
+
+  // (segment, K tile) steps; this CTA's range
+  int steps_of[kTcMaxBlocks];
+  int nsteps = 0;
+  for (int s = 0; s < nseg_all; ++s) {
+    steps_of[s] = (tc_seg(p, s).ncols + kTcK - 1) / kTcK;
+    nsteps += steps_of[s];
+  }
+  const int st0 = rank * nsteps / S, st1 = (rank + 1) * nsteps / S;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s <= kTcMaxStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mma_done + s)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)), "r"(tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+  // Peers write into this CTA's shared memory at the end; the split barrier tells them
+  // that every CTA of the cluster is running.
+  auto started = cluster.barrier_arrive();
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  bool ok = true;
+  unsigned touched = 0;  // accumulator blocks written by this CTA (same in every thread)
+  const int n = st1 - st0;
+  // (segment, K tile) of the CTA-local step j
+  auto step_pos = [&](int j, int& sg, int& kt) {
+    int rem = st0 + j;
+    sg = 0;
+    while (sg < nseg_all - 1 && rem >= steps_of[sg]) { rem -= steps_of[sg]; ++sg; }
+    kt = rem;
+  };
+  const int tile_rows = ((p.rows + 31) / 32) * 32;  // rows present in the packed layout
+  // raw sign words (128 rows x 16 bytes) and column scales of step j -> ring slot j % 4
+  auto issue_raw = [&](int j) {
+    int sg, kt;
+    step_pos(j, sg, kt);
+    const TcSeg g = tc_seg(p, sg);
+    if (g.kind == kSegSal || g.bits == nullptr) return;
+    unsigned char* dst = raw_ring + (j % kTcRawSlots) * kTcRawBytes;
+    if (threadIdx.x < kTcRows) {
+      const int o = o0 + threadIdx.x;
+      const bool in = o < tile_rows;
+      const uint4* src = g.bits + (static_cast<long long>(in ? o >> 5 : 0) * g.nq + kt) * 32 + (in ? (o & 31) : 0);
+      cp16(dst + threadIdx.x * 16, src, in ? 16u : 0u);
+    } else if (g.cscale != nullptr && threadIdx.x < kTcRows + kTcK / 8) {
+      const int cc = kt * kTcK + (threadIdx.x - kTcRows) * 8;
+      const int valid = max(0, min(8, g.ncols - cc));
+      unsigned char* cd = dst + kTcRows * 16 + (threadIdx.x - kTcRows) * 16;
+      const unsigned short* cs = reinterpret_cast<const unsigned short*>(g.cscale);
+      if (g.cvec) {  // 16-byte aligned scales: asynchronous copy with zero fill
+        cp16(cd, cs + (valid > 0 ? cc : 0), static_cast<unsigned>(valid * 2));
+      } else {       // unaligned (e.g. the second base of a layer with in % 8 != 0): plain loads
+        unsigned short v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = e < valid ? __ldg(cs + cc + e) : 0;
+        *reinterpret_cast<uint4*>(cd) = make_uint4(v[0] | (static_cast<unsigned>(v[1]) << 16), v[2] | (static_cast<unsigned>(v[3]) << 16),
+                                                   v[4] | (static_cast<unsigned>(v[5]) << 16), v[6] | (static_cast<unsigned>(v[7]) << 16));
+      }
+    }
+  };
+  // bf16 activation tile of step j straight into its stage (bases over bf16 X only)
+  auto b_direct = [&](int sg) {
+    const TcSeg g = tc_seg(p, sg);
+    return g.kind == kSegX && p.xdt == BISCO_BF16 && p.x_vec;
+  };
+  auto issue_b = [&](int j) {
+    int sg, kt;
+    step_pos(j, sg, kt);
+    if (!b_direct(sg)) return;
+    const TcSeg g = tc_seg(p, sg);
+    unsigned char* B = stages + static_cast<size_t>(j % nstages) * stage_bytes + a_bytes;
+    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcThreads) {
+      const int m = ch % Np, k8 = ch / Np;
+      const int c = kt * kTcK + 8 * k8;
+      const int valid = (m < p.Mc) ? max(0, min(8, g.ncols - c)) : 0;
+      const unsigned short* src = reinterpret_cast<const unsigned short*>(p.X) + (valid > 0 ? static_cast<long long>(m) * p.ldx + c : 0);
+      cp16(B + tile_off(m, k8, Np), src, static_cast<unsigned>(valid * 2));
+    }
+  };
+  // prologue: raw data of steps 0 and 1, activations of step 0
+  if (n > 0) issue_raw(0);
+  if (n > 1) issue_raw(1);
+  if (n > 0) issue_b(0);
+  cp_commit();
+  for (int i = 0; i < n; ++i) {
+    // look ahead: activations of step i + 1 (into its stage, once free), raw data of i + 2
+    if (i + 1 < n) {
+      if (i + 1 >= nstages &&
+          !tc_wait(mma_done + (i + 1) % nstages, static_cast<unsigned>((i + 1) / nstages - 1) & 1u))
+        ok = false;
+      issue_b(i + 1);
+    }
+    if (i + 2 < n) issue_raw(i + 2);
+    cp_commit();
+    cp_wait1();       // all groups but the one just committed: step i's data has landed
+    __syncthreads();  // ... for every thread
+    int seg, kt;
+    step_pos(i, seg, kt);
+    const TcSeg g = tc_seg(p, seg);
+    const int blk = acc.blk_of_seg[seg];
+    const int split = acc.split[blk];
+    const int sl = i % nstages;
+    unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
+    unsigned char* B = A + a_bytes;
+    const int c0 = kt * kTcK;
+    if (g.kind == kSegSal || g.bits == nullptr) {
+      for (int ch = threadIdx.x; ch < kTcRows * 16; ch += kTcThreads) {
+        const int r = ch & (kTcRows - 1), k8 = ch >> 7;
+        *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = a_chunk(p, g, o0 + r, c0 + 8 * k8);
+      }
+    } else {
+      a_expand(A, raw_ring + (i % kTcRawSlots) * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7,
+               g.ncols - c0, g.cscale != nullptr);
+    }
+    const int brows = split * Np;
+    if (!b_direct(seg)) {
+      for (int ch = threadIdx.x; ch < brows * 16; ch += kTcThreads) {
+        const int nn = ch % brows, k8 = ch / brows;
+        const int part = nn / Np, m = nn - part * Np;
+        *reinterpret_cast<uint4*>(B + tile_off(nn, k8, brows)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
+      }
+    }
+    // make the generic-proxy and cp.async stores visible to the tensor core
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t idesc = mma_idesc(brows);
+      const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk]);
+      const bool first = !((touched >> blk) & 1u);
+#pragma unroll
+      for (int kk = 0; kk < kTcK / 16; ++kk) {
+        const unsigned koff = (kk & 3) * 32u;  // K step inside a 64-column block
+        mma_bf16(d, smem_desc_sw128(A + (kk >> 2) * (kTcRows * 128) + koff),
+                 smem_desc_sw128(B + (kk >> 2) * (brows * 128) + koff), idesc, (first && kk == 0) ? 0u : 1u);
+      }
+      mma_commit(mma_done + sl);
+    }
+    touched |= 1u << blk;
+  }
+  if (threadIdx.x == 0) mma_commit(all_done);
+  if (!tc_wait(all_done, 0u)) ok = false;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+
+  // every CTA of the cluster is done with its stages before partial sums are pushed
+  cluster.barrier_wait(std::move(started));
+  if (S > 1) cluster.sync();
+  const int rows_per = (kTcRows + S - 1) / S;
+  if (warp < 4) {
+    // warp w reads tensor-memory lanes 32w..32w+31 = rows of this CTA's tile
+    const int r = warp * 32 + lane;
+    const int o = o0 + r;
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float rsv[kTcMaxBlocks];
+    for (int b = 0; b < acc.nblk; ++b) {
+      rsv[b] = 1.f;
+      const int s = acc.rseg[b];
+      if (s >= 0 && o < p.rows && p.seg[s].rscale != nullptr)
+        rsv[b] = p.seg[s].rdt == BISCO_BF16
+                     ? __uint_as_float(static_cast<unsigned>(__ldg(reinterpret_cast<const unsigned short*>(p.seg[s].rscale) + o)) << 16)
+                     : __ldg(reinterpret_cast<const float*>(p.seg[s].rscale) + o);
+    }
+    const int dst = r / rows_per;
+    float* rp = S > 1 ? cluster.map_shared_rank(recv, dst) + (static_cast<size_t>(rank) * rows_per + (r - dst * rows_per)) * Np
+                      : nullptr;
+    for (int m0 = 0; m0 < Np; m0 += 16) {
+      float y[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) y[j] = 0.f;
+      for (int b = 0; b < acc.nblk; ++b) {
+        if (!((touched >> b) & 1u)) continue;
+        for (int part = 0; part < acc.split[b]; ++part) {
+          uint32_t v[16];
+          const uint32_t ta = lane_addr + static_cast<uint32_t>(acc.col[b] + part * Np + m0);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+                "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+              : "r"(ta));
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+          for (int j = 0; j < 16; ++j) y[j] = fmaf(__uint_as_float(v[j]), rsv[b], y[j]);
+        }
+      }
+      if (S > 1) {
+        // push to the row's owner CTA: recv[rank][row - first row of owner][m], 16-byte stores
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(rp + m0 + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+      } else if (o < p.rows) {
+        // no K split: this CTA holds the whole sum of its rows
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + j;
+          if (m < p.Mc) {
+            if (p.ydt == BISCO_BF16)
+              reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(y[j]);
+            else
+              reinterpret_cast<float*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = y[j];
+          }
+        }
+      }
+    }
+  }
+  if (S > 1) {
+    cluster.sync();  // all partial sums have landed
+    // ---- owner: add the S partials in rank order and store ----
+    const int rr0 = rank * rows_per, rr1 = min(kTcRows, rr0 + rows_per);
+    const int nr = rr1 - rr0;
+    if (nr > 0) {
+      for (int idx = threadIdx.x; idx < nr * Np; idx += kTcThreads) {
+        const int m = idx / nr, lr = idx - m * nr;
+        const int o = o0 + rr0 + lr;
+        if (o >= p.rows || m >= p.Mc) continue;
+        float sum = 0.f;
+        for (int src = 0; src < S; ++src) sum += recv[(static_cast<size_t>(src) * rows_per + lr) * Np + m];
+        if (p.ydt == BISCO_BF16)
+          reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(sum);
+        else
+          reinterpret_cast<float*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = sum;
+      }
+    }
+  }
+  if (!ok && threadIdx.x == 0) atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
+}
+
+int tc_max_clusters(int S, size_t smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_kernel, &cfg) != cudaSuccess) return 0;
+  return n;
+}
+
+}  // namespace
+
+cudaError_t tc_ensure_attrs() {
+  static std::once_flag once[64];
+  static cudaError_t err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::call_once(once[dev & 63], [&] {
+    err[dev & 63] = cudaFuncSetAttribute(tc_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(query_smem_limit()));
+  });
+  return err[dev & 63];
+}
+
+TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncols, int n_sal, bool x_bf16, int Mc,
+                    int num_sms, size_t smem_limit) {
+  TcPlan t{};
+  t.Np = (Mc + 15) / 16 * 16;
+  const TcAcc acc = tc_acc(nseg, seg_kind, n_sal > 0, x_bf16, t.Np);
+  if (acc.ncols > 512) return t;  // does not fit in tensor memory
+  t.tmem_cols = 32;
+  while (t.tmem_cols < acc.ncols) t.tmem_cols *= 2;
+  int nsteps = 0;
+  for (int s = 0; s < nseg; ++s) nsteps += (seg_ncols[s] + kTcK - 1) / kTcK;
+  if (n_sal > 0) nsteps += (n_sal + kTcK - 1) / kTcK;
+  if (nsteps == 0) return t;
+  const size_t stage = static_cast<size_t>(kTcRows) * kTcK * 2 + static_cast<size_t>(2 * t.Np) * kTcK * 2;
+  const size_t fixed = 1024 + static_cast<size_t>(kTcRawSlots) * kTcRawBytes;
+  t.stages = static_cast<int>(std::min<size_t>(kTcMaxStages, (smem_limit - fixed) / stage));
+  if (t.stages < 2) return t;
+  // more than half of the SM's shared memory: one CTA per SM (tensor memory is not shared)
+  t.smem = std::max(fixed + t.stages * stage, smem_limit / 2 + 4096);
+  t.smem = std::min(t.smem, smem_limit);
+  if (fixed + t.stages * stage > t.smem) return t;
+  tc_ensure_attrs();
+  t.tiles = (rows + kTcRows - 1) / kTcRows;
+  // split K over a cluster so that the grid covers the SMs
+  int S = std::max(1, std::min({kMaxCluster, nsteps, num_sms / std::max(1, t.tiles)}));
+  while (S > 1 && (S & (S - 1))) --S;  // power of two
+  for (; S >= 1; S /= 2) {
+    const size_t recv = static_cast<size_t>(S) * ((kTcRows + S - 1) / S) * t.Np * 4;
+    if (recv > static_cast<size_t>(t.stages) * stage) continue;
+    if (tc_max_clusters(S, t.smem) >= 1) break;
+  }
+  if (S < 1) return t;
+  t.S = S;
+  return t;
+}
+
+cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream) {
+  const cudaError_t e = tc_ensure_attrs();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(t.tiles * t.S);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = t.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = t.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, t.S, t.Np, t.stages, t.tmem_cols);
+}
+
+}  // namespace bisco
