@@ -884,7 +884,7 @@ struct SSmem {
   uint64_t* empty;      // [TS] stage released by the gu warps of its tile group
   unsigned char* ring;  // [NS][CU * 512] sign words
   float* tables;        // [CU][MB][26][36]
-  float* xt;            // [CU][MB][128] scaled activations of the chunk
+  float* xt;            // [max_units][MB][128] scaled activations of all the CTA's units
   float* cs;            // [max_units][128] column scales
   float* rsc;           // [max_lseg][max_tiles * 32] row scales
   float* part;          // [GU][max_tiles][MB][32] partial sums per unit group
@@ -903,7 +903,7 @@ __host__ __device__ __forceinline__ size_t ssmem_bytes(int CU, int NS, int GU, i
   const int msh = ((max_tiles * 32 + C - 1) / C + 3) & ~3;
   const int TS = max_stages(max_tiles, max_units, CU);
   return static_cast<size_t>((16 * TS + 127) / 128 * 128) + static_cast<size_t>(NS) * CU * 512 +
-         static_cast<size_t>(CU) * col_stride + static_cast<size_t>(CU) * MB * 128 * 4 +
+         static_cast<size_t>(CU) * col_stride + static_cast<size_t>(max_units) * MB * 128 * 4 +
          static_cast<size_t>(max_units) * 128 * 4 + static_cast<size_t>(max_lseg) * max_tiles * 32 * 4 +
          static_cast<size_t>(GU) * max_tiles * MB * 32 * 4 + static_cast<size_t>(C) * MB * msh * 4 +
          static_cast<size_t>(MB) * nsp * 4;
@@ -918,7 +918,7 @@ __device__ __forceinline__ SSmem scarve(unsigned char* smem, const PassParam& p,
   q += (16 * TS + 127) / 128 * 128;
   s.ring = q;                             q += static_cast<size_t>(NS) * CU * 512;
   s.tables = reinterpret_cast<float*>(q); q += static_cast<size_t>(CU) * p.col_stride_bytes;
-  s.xt = reinterpret_cast<float*>(q);     q += static_cast<size_t>(CU) * MB * 128 * 4;
+  s.xt = reinterpret_cast<float*>(q);     q += static_cast<size_t>(p.max_units) * MB * 128 * 4;
   s.cs = reinterpret_cast<float*>(q);     q += static_cast<size_t>(p.max_units) * 128 * 4;
   s.rsc = reinterpret_cast<float*>(q);    q += static_cast<size_t>(p.max_lseg) * p.max_tiles * 32 * 4;
   s.part = reinterpret_cast<float*>(q);   q += static_cast<size_t>(GU) * p.max_tiles * MB * 32 * 4;
@@ -1172,15 +1172,15 @@ __global__ void __launch_bounds__(kST, 2)
     float* my_part = S.part + static_cast<size_t>(gb) * p.max_tiles * MB * 32 + lane;
     const unsigned cstride = static_cast<unsigned>(p.col_stride_bytes);
     constexpr int kBatch = MB == 1 ? 4 : 2;
-    for (int c = 0; c < nchunks; ++c) {
-      const int cu0 = c * CU, cn = min(CU, nu - cu0);
-      __syncthreads();  // scales staged (c = 0); previous chunk's tables no longer read (c > 0)
-      // scaled activations of the chunk: 8-column runs, one 16-byte load each
-      for (int ch = threadIdx.x; ch < cn * MB * 16; ch += kST) {
+    __syncthreads();  // column scales staged
+    // scaled activations of all the CTA's units at once (one round trip to L2):
+    // 8-column runs, one 16-byte load each
+    for (int ch = threadIdx.x; ch < nu * MB * 16; ch += kST) {
+      {
         const int ulc = ch / (MB * 16);
         const int rem = ch - ulc * (MB * 16);
         const int m = rem >> 4, j0 = (rem & 15) * 8;
-        const int u = u0 + cu0 + ulc;
+        const int u = u0 + ulc;
         const SegParam& G = p.seg[find_seg(p, u)];
         const int cc = (u - G.unit0) * 128 + j0;
         const int valid = max(0, min(8, G.ncols - cc));
@@ -1193,17 +1193,20 @@ __global__ void __launch_bounds__(kST, 2)
           else
             load8_l2(p.Z, static_cast<long long>(m) * p.ldz + cc, BISCO_F32, valid, p.z_vec != 0, xv);
         }
-        const float* cv = S.cs + (cu0 + ulc) * 128 + j0;
+        const float* cv = S.cs + ulc * 128 + j0;
         float4* d4 = reinterpret_cast<float4*>(S.xt + (ulc * MB + m) * 128 + j0);
         d4[0] = make_float4(xv[0] * cv[0], xv[1] * cv[1], xv[2] * cv[2], xv[3] * cv[3]);
         d4[1] = make_float4(xv[4] * cv[4], xv[5] * cv[5], xv[6] * cv[6], xv[7] * cv[7]);
       }
-      __syncthreads();
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int cu0 = c * CU, cn = min(CU, nu - cu0);
+      __syncthreads();  // activations staged (c = 0); previous chunk's tables no longer read (c > 0)
       // tables: task (unit, batch row); lane f builds the 32 signed sums of field f
       for (int tq = warp; tq < cn * MB; tq += kSW) {
         const int ulc = tq / MB, m = tq - ulc * MB;
         if (lane < kFields) {
-          const float* x = S.xt + (ulc * MB + m) * 128 + 5 * lane;
+          const float* x = S.xt + ((cu0 + ulc) * MB + m) * 128 + 5 * lane;
           const float x0 = x[0], x1 = x[1], x2 = x[2];
           const float x3 = lane < 25 ? x[3] : 0.f, x4 = lane < 25 ? x[4] : 0.f;
           const float d[5] = {2.f * x0, 2.f * x1, 2.f * x2, 2.f * x3, 2.f * x4};
@@ -1468,7 +1471,7 @@ Plan make_stream_plan(int rows, int units, const int* seg_unit0, int nseg, int M
     pl.col_stride_bytes = (MB * kFields * kFieldStride * 4 + 127) / 128 * 128;
     pl.max_units = (units + C - 1) / C;
     pl.max_lseg = max_segments_per_cta(units, C, seg_unit0, nseg);
-    int fit = max_active_clusters(MB, 2, C, smem_limit / 2 + 1024);
+    int fit = max_active_clusters(MB, 2, C, std::max<size_t>(budget, smem_limit / 2 + 1024));
     if (fit <= 0) continue;
     pl.ncl = std::max(1, std::min(tiles, fit));
     pl.max_tiles = (tiles + pl.ncl - 1) / pl.ncl;
@@ -1514,6 +1517,7 @@ size_t query_smem_limit() {
 Plan make_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, int num_sms,
                size_t smem_limit) {
   ensure_kernel_attrs();
+  const int tiles = (rows + 31) / 32;
   if (MB <= 2) {
     // Prefer plans that leave room on each SM for a CTA of the next kernel.
     Plan s = make_stream_plan(rows, units, seg_unit0, nseg, MB, n_sal, smem_limit, smem_limit / 2 - 1024);
@@ -1525,7 +1529,6 @@ Plan make_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int 
   Plan pl{};
   pl.MB = MB;
   pl.kind = MB <= 2 ? 0 : 1;
-  const int tiles = (rows + 31) / 32;
   pl.C = std::max(1, std::min(kMaxCluster, units));
   pl.col_stride_bytes = (MB * kFields * kFieldStride * 4 + 127) / 128 * 128;
   pl.max_units = (units + pl.C - 1) / pl.C;
