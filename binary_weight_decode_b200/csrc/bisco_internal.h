@@ -87,7 +87,7 @@ size_t query_smem_limit();
 
 // Tensor-core path (16..128 batch rows per launch): one launch per pass.
 constexpr int kTcMinBatch = 32;           // smallest batch chunk sent to the tensor cores
-constexpr int kTcMaxBatch = 64;           // batch rows per launch (three pipeline stages fit)
+constexpr int kTcMaxBatch = 128;          // batch rows per launch
 struct TcPlan {
   int Np;                // batch rows padded to a multiple of 16 (MMA N per part)
   int tmem_cols;         // tensor-memory columns allocated per CTA

@@ -1,4 +1,4 @@
-// Tensor-core path for larger batches (16 to 64 batch rows per launch).
+// Tensor-core path for larger batches (32 to 128 batch rows per launch).
 //
 // With many batch rows the product is a dense contraction: for each segment,
 //   D_seg[o][m] = sum_i A_seg[o][i] * B_seg[i][m].
@@ -24,13 +24,16 @@
 // the (segment, 128-column K tile) steps. A step's tiles live in a shared-memory stage,
 // K-major with the 128-byte swizzle: each tile is two blocks of 64 columns; a row of a
 // block is 128 bytes, its 16-byte chunks permuted by XOR with (row mod 8), and groups
-// of 8 rows are 1024 bytes apart. The loop is software-pipelined: while step i is
-// expanded, cp.async brings in the raw sign words and column scales of step i + 2 (a
-// four-slot ring) and the bf16 activation tile of step i + 1 (straight into its stage,
-// once the MMAs that last read that stage are done). Eight warps expand step i's signs
-// from shared memory; one thread issues the step's eight K=16 MMAs and commits them to
-// the stage's mbarrier. The S partial results meet in distributed shared memory and are
-// added in CTA-rank order.
+// of 8 rows are 1024 bytes apart. cp.async brings in the raw sign words and column
+// scales two steps ahead (a four-slot ring) and the bf16 activation tile of a step into
+// its stage. The warps are specialised: eight producer warps wait until a stage is free,
+// copy the activation tile into it (completion counted on the stage's "full" mbarrier),
+// expand the step's signs from the raw ring and mark the stage full; a ninth warp waits
+// for each full stage, issues the step's eight K=16 MMAs and commits them to the stage's
+// "free" mbarrier, so expansion of later stages overlaps the MMAs of earlier ones. Every
+// waiter walks every stage in order, so one pair of barriers per stage slot suffices.
+// The S partial results meet in distributed shared memory and are added in CTA-rank
+// order.
 // A CTA takes more than half of an SM's shared memory, so no two CTAs (each holding up
 // to 512 tensor-memory columns) ever share an SM.
 
@@ -49,8 +52,8 @@ namespace bisco {
 
 namespace {
 
-constexpr int kTcWarps = 8;
-constexpr int kTcThreads = kTcWarps * 32;
+constexpr int kTcProducers = 256;              // 8 producer warps
+constexpr int kTcThreads = kTcProducers + 32;  // + 1 MMA warp
 constexpr int kTcRows = 128;       // output rows per cluster (MMA M)
 constexpr int kTcK = 128;          // input columns per step (eight K=16 MMAs)
 constexpr int kTcMaxStages = 3;
@@ -78,6 +81,15 @@ __device__ __forceinline__ bool tc_try(uint64_t* b, unsigned parity) {
       : "memory");
   return done != 0;
 }
+
+__device__ __forceinline__ void bar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
+}
+// Arrives on b once all cp.async operations issued so far by this thread have completed.
+__device__ __forceinline__ void bar_arrive_cp(uint64_t* b) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
+}
+__device__ __forceinline__ void producers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kTcProducers) : "memory"); }
 
 // Waits (bounded in time) until the phase with the given parity has completed.
 __device__ __forceinline__ bool tc_wait(uint64_t* b, unsigned parity) {
@@ -129,6 +141,7 @@ __device__ __forceinline__ void cp16(void* dst, const void* src, unsigned src_by
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -316,7 +329,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const unsigned a_bytes = kTcRows * kTcK * 2, b_bytes = static_cast<unsigned>(2 * Np) * kTcK * 2;
   const unsigned stage_bytes = a_bytes + b_bytes;
 
-  uint64_t* mma_done = reinterpret_cast<uint64_t*>(smem);   // [kTcMaxStages]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // [kTcMaxStages] stage filled
+  uint64_t* mma_done = full + kTcMaxStages;                 // [kTcMaxStages] stage's MMAs done
   uint64_t* all_done = mma_done + kTcMaxStages;             // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(all_done + 1);
   unsigned char* raw_ring = smem + 1024;                    // [kTcRawSlots][kTcRawBytes]
@@ -333,6 +347,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int st0 = rank * nsteps / S, st1 = (rank + 1) * nsteps / S;
 
   if (threadIdx.x == 0) {
+    // full: one cp.async-completion arrival and one plain arrival per producer thread
+    for (int s = 0; s < kTcMaxStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(full + s)), "r"(2 * kTcProducers) : "memory");
     for (int s = 0; s <= kTcMaxStages; ++s)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mma_done + s)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -402,7 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!b_direct(sg)) return;
     const TcSeg g = tc_seg(p, sg);
     unsigned char* B = stages + static_cast<size_t>(j % nstages) * stage_bytes + a_bytes;
-    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcThreads) {
+    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
       const int m = ch % Np, k8 = ch / Np;
       const int c = kt * kTcK + 8 * k8;
       const int valid = (m < p.Mc) ? max(0, min(8, g.ncols - c)) : 0;
@@ -410,57 +427,72 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       cp16(B + tile_off(m, k8, Np), src, static_cast<unsigned>(valid * 2));
     }
   };
-  // prologue: raw data of steps 0 and 1, activations of step 0
-  if (n > 0) issue_raw(0);
-  if (n > 1) issue_raw(1);
-  if (n > 0) issue_b(0);
-  cp_commit();
+  // accumulator blocks this CTA writes (every thread walks the steps)
   for (int i = 0; i < n; ++i) {
-    // look ahead: activations of step i + 1 (into its stage, once free), raw data of i + 2
-    if (i + 1 < n) {
-      if (i + 1 >= nstages &&
-          !tc_wait(mma_done + (i + 1) % nstages, static_cast<unsigned>((i + 1) / nstages - 1) & 1u))
-        ok = false;
-      issue_b(i + 1);
-    }
-    if (i + 2 < n) issue_raw(i + 2);
+    int sg, kt;
+    step_pos(i, sg, kt);
+    touched |= 1u << acc.blk_of_seg[sg];
+  }
+  if (warp < kTcProducers / 32) {
+    // ---------------- producers ----------------
+    if (n > 0) issue_raw(0);
+    if (n > 1) issue_raw(1);
     cp_commit();
-    cp_wait1();       // all groups but the one just committed: step i's data has landed
-    __syncthreads();  // ... for every thread
-    int seg, kt;
-    step_pos(i, seg, kt);
-    const TcSeg g = tc_seg(p, seg);
-    const int blk = acc.blk_of_seg[seg];
-    const int split = acc.split[blk];
-    const int sl = i % nstages;
-    unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
-    unsigned char* B = A + a_bytes;
-    const int c0 = kt * kTcK;
-    if (g.kind == kSegSal || g.bits == nullptr) {
-      for (int ch = threadIdx.x; ch < kTcRows * 16; ch += kTcThreads) {
-        const int r = ch & (kTcRows - 1), k8 = ch >> 7;
-        *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = a_chunk(p, g, o0 + r, c0 + 8 * k8);
+    for (int i = 0; i < n; ++i) {
+      const int sl = i % nstages;
+      // the stage is free once the MMAs that last read it are done
+      if (i >= nstages && !tc_wait(mma_done + sl, static_cast<unsigned>(i / nstages - 1) & 1u)) ok = false;
+      issue_b(i);
+      bar_arrive_cp(full + sl);
+      if (i + 2 < n) issue_raw(i + 2);
+      cp_commit();
+      if (i == 0) cp_wait1(); else cp_wait2();  // this thread's copies of step i's raw data
+      producers_sync();                         // ... and every producer's
+      int seg, kt;
+      step_pos(i, seg, kt);
+      const TcSeg g = tc_seg(p, seg);
+      const int split = acc.split[acc.blk_of_seg[seg]];
+      unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
+      unsigned char* B = A + a_bytes;
+      const int c0 = kt * kTcK;
+      if (g.kind == kSegSal || g.bits == nullptr) {
+        for (int ch = threadIdx.x; ch < kTcRows * 16; ch += kTcProducers) {
+          const int r = ch & (kTcRows - 1), k8 = ch >> 7;
+          *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = a_chunk(p, g, o0 + r, c0 + 8 * k8);
+        }
+      } else {
+        a_expand(A, raw_ring + (i % kTcRawSlots) * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7,
+                 g.ncols - c0, g.cscale != nullptr);
       }
-    } else {
-      a_expand(A, raw_ring + (i % kTcRawSlots) * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7,
-               g.ncols - c0, g.cscale != nullptr);
-    }
-    const int brows = split * Np;
-    if (!b_direct(seg)) {
-      for (int ch = threadIdx.x; ch < brows * 16; ch += kTcThreads) {
-        const int nn = ch % brows, k8 = ch / brows;
-        const int part = nn / Np, m = nn - part * Np;
-        *reinterpret_cast<uint4*>(B + tile_off(nn, k8, brows)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
+      const int brows = split * Np;
+      if (!b_direct(seg)) {
+        for (int ch = threadIdx.x; ch < brows * 16; ch += kTcProducers) {
+          const int nn = ch % brows, k8 = ch / brows;
+          const int part = nn / Np, m = nn - part * Np;
+          *reinterpret_cast<uint4*>(B + tile_off(nn, k8, brows)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
+        }
       }
+      // make the generic-proxy stores visible to the tensor core, then mark the stage full
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      bar_arrive(full + sl);
     }
-    // make the generic-proxy and cp.async stores visible to the tensor core
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncthreads();
-    if (threadIdx.x == 0) {
+  } else if (lane == 0) {
+    // ---------------- MMA issue (one thread) ----------------
+    unsigned written = 0;
+    for (int i = 0; i < n; ++i) {
+      const int sl = i % nstages;
+      if (!tc_wait(full + sl, static_cast<unsigned>(i / nstages) & 1u)) ok = false;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async-written activations
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      int seg, kt;
+      step_pos(i, seg, kt);
+      const int blk = acc.blk_of_seg[seg];
+      const int brows = acc.split[blk] * Np;
+      unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
+      unsigned char* B = A + a_bytes;
       const uint32_t idesc = mma_idesc(brows);
       const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk]);
-      const bool first = !((touched >> blk) & 1u);
+      const bool first = !((written >> blk) & 1u);
 #pragma unroll
       for (int kk = 0; kk < kTcK / 16; ++kk) {
         const unsigned koff = (kk & 3) * 32u;  // K step inside a 64-column block
@@ -468,10 +500,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                  smem_desc_sw128(B + (kk >> 2) * (brows * 128) + koff), idesc, (first && kk == 0) ? 0u : 1u);
       }
       mma_commit(mma_done + sl);
+      written |= 1u << blk;
     }
-    touched |= 1u << blk;
+    mma_commit(all_done);
   }
-  if (threadIdx.x == 0) mma_commit(all_done);
+  __syncwarp();
   if (!tc_wait(all_done, 0u)) ok = false;
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 
@@ -553,7 +586,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   }
-  if (!ok && threadIdx.x == 0) atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
+  if (!ok) atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0)
