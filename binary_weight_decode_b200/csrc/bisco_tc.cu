@@ -253,6 +253,10 @@ __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* 
   const uint4 bw = *reinterpret_cast<const uint4*>(raw + r * 16);
   const unsigned lo = h ? bw.z : bw.x, hi = h ? bw.w : bw.y;
   const unsigned short* cs = reinterpret_cast<const unsigned short*>(raw + kTcRows * 16);
+  // columns 64h.. are the h-th 64-column block: row r of it at h*128*128 + r*128, chunk j
+  // of the row at ((j ^ (r mod 8)) * 16)
+  unsigned char* rowp = A + h * (kTcRows * 128) + r * 128;
+  const int rx = r & 7;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int k8 = 8 * h + j;
@@ -272,7 +276,7 @@ __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* 
       const unsigned nb = ~(byte >> (2 * e));
       w[e] = c[e] ^ (((nb & 1u) << 15) | ((nb & 2u) << 30));
     }
-    *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint4*>(rowp + ((j ^ rx) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -419,12 +423,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!b_direct(sg)) return;
     const TcSeg g = tc_seg(p, sg);
     unsigned char* B = stages + static_cast<size_t>(j % nstages) * stage_bytes + a_bytes;
-    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
-      const int m = ch % Np, k8 = ch / Np;
-      const int c = kt * kTcK + 8 * k8;
+    // chunk ch = k8 * Np + m; this thread takes ch = tid, tid + 256, ...: m and k8 advance
+    // by fixed steps (no division per chunk)
+    int m = threadIdx.x % Np, k8 = threadIdx.x / Np;
+    const int dm = kTcProducers % Np, dk = kTcProducers / Np;
+    const int c_base = kt * kTcK;
+    const unsigned short* xrow = reinterpret_cast<const unsigned short*>(p.X);
+    for (; k8 < 16; ) {
+      const int c = c_base + 8 * k8;
       const int valid = (m < p.Mc) ? max(0, min(8, g.ncols - c)) : 0;
-      const unsigned short* src = reinterpret_cast<const unsigned short*>(p.X) + (valid > 0 ? static_cast<long long>(m) * p.ldx + c : 0);
+      const unsigned short* src = xrow + (valid > 0 ? static_cast<long long>(m) * p.ldx + c : 0);
       cp16(B + tile_off(m, k8, Np), src, static_cast<unsigned>(valid * 2));
+      m += dm;
+      k8 += dk;
+      if (m >= Np) { m -= Np; ++k8; }
     }
   };
   // accumulator blocks this CTA writes (every thread walks the steps)
