@@ -78,6 +78,29 @@ def traffic_for(workload, M):
     return None
 
 
+def max_over_ranks(value, dist, device):
+    """The largest of `value` over all ranks (the job is as slow as its slowest rank);
+    `value` itself when there is no process group."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def launches_per_gemv(M, rank, scale_bf16, tc_min=32, tc_max=128, lut_max=8):
+    """Kernel launches of one bisco_gemv call: the library's batch-chunk schedule
+    (tensor-core chunks of up to 128 rows from 32 rows up when the scales are bf16,
+    lookup-table chunks of up to 8 rows otherwise), one launch per pass per chunk."""
+    chunks, rem = 0, M
+    while rem > 0:
+        take = min(rem, tc_max) if (scale_bf16 and rem >= tc_min) else min(rem, lut_max)
+        rem -= take
+        chunks += 1
+    return chunks * (2 if rank else 1)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -253,7 +276,7 @@ def main():
     with torch.cuda.graph(graph, stream=stream):
         for i in range(S):
             bw.bisco_gemv(dls[i], Xd, Yd[i], ws, stream=stream)
-    kernels_per_gemv = (2 if L.rank else 1) * math.ceil(M / 8)
+    kernels_per_gemv = launches_per_gemv(M, L.rank, L.K == 0 or L.scale_dtype == "bf16")
 
     def barrier():
         if dist is not None:
@@ -278,10 +301,7 @@ def main():
     barrier()
     ms = e0.elapsed_time(e1)
     clocks = sampler.stop()
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     gemvs = args.steps * S
     us_per_gemv = ms * 1000.0 / gemvs
     value = world * gemvs * nbytes / (ms / 1000.0) / 1e9
@@ -304,10 +324,7 @@ def main():
     e3.record(stream)
     barrier()
     ms_e2e = e2.elapsed_time(e3)
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dist, "cuda")
     e2e_value = world * e2e_steps * S * nbytes / (ms_e2e / 1000.0) / 1e9
 
     peak, peak_kind = hbm_peak()

@@ -1,0 +1,72 @@
+"""Host-side logic of bench.py's multi-GPU (replica) mode, on CPU.
+
+bench.py --gpus N runs N independent replicas (the single-layer product has no data-path
+collective) and reports the slowest rank's time: two gloo ranks on CPU check that every
+rank gets the maximum. The batch-chunk schedule behind the launch count is checked
+against its definition.
+"""
+
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+import importlib.util  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        b = _bench()
+        mine = 1.5 + rank * 2.25  # per-rank timings differ
+        out[rank] = b.max_over_ranks(mine, dist, "cpu")
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_two_gloo_ranks():
+    world, port = 2, _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        ctx = mp.get_context("spawn")
+        procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(120)
+            assert p.exitcode == 0
+        assert out[0] == out[1] == pytest.approx(1.5 + 2.25)
+
+
+def test_max_without_process_group_is_identity():
+    assert _bench().max_over_ranks(3.25, None, "cpu") == 3.25
+
+
+@pytest.mark.parametrize("M,rank,bf16,expected", [
+    (1, 0, True, 1), (1, 256, True, 2), (8, 0, True, 1), (9, 0, True, 2), (16, 0, True, 2),
+    (32, 0, True, 1), (33, 0, True, 1), (128, 256, True, 2), (130, 0, True, 2), (160, 0, True, 2),
+    (190, 0, True, 2), (64, 0, False, 8), (31, 0, True, 4),
+])
+def test_launch_schedule(M, rank, bf16, expected):
+    assert _bench().launches_per_gemv(M, rank, bf16) == expected
