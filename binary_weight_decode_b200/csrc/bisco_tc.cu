@@ -26,9 +26,9 @@
 // block is 128 bytes, its 16-byte chunks permuted by XOR with (row mod 8), and groups
 // of 8 rows are 1024 bytes apart. cp.async brings in the raw sign words and column
 // scales two steps ahead (a four-slot ring) and the bf16 activation tile of a step into
-// its stage. The warps are specialised: eight producer warps wait until a stage is free,
+// its stage. The warps are specialised: 16 producer warps wait until a stage is free,
 // copy the activation tile into it (completion counted on the stage's "full" mbarrier),
-// expand the step's signs from the raw ring and mark the stage full; a ninth warp waits
+// expand the step's signs from the raw ring and mark the stage full; one more warp waits
 // for each full stage, issues the step's eight K=16 MMAs and commits them to the stage's
 // "free" mbarrier, so expansion of later stages overlaps the MMAs of earlier ones. Every
 // waiter walks every stage in order, so one pair of barriers per stage slot suffices.
@@ -52,7 +52,7 @@ namespace bisco {
 
 namespace {
 
-constexpr int kTcProducers = 256;              // 8 producer warps
+constexpr int kTcProducers = 512;              // 16 producer warps
 constexpr int kTcThreads = kTcProducers + 32;  // + 1 MMA warp
 constexpr int kTcRows = 128;       // output rows per cluster (MMA M)
 constexpr int kTcK = 128;          // input columns per step (eight K=16 MMAs)
@@ -183,17 +183,30 @@ __device__ __forceinline__ uint4 b_chunk(const PassParam& p, const TcSeg& g, int
   if (m < p.Mc) {
     const int valid = max(0, min(8, g.ncols - c));
     if (g.kind == kSegSal) {
-      for (int j = 0; j < valid; ++j) {
-        const int cc = __ldg(p.sal_idx + c + j);
-        if (cc >= 0 && cc < p.xcols) v[j] = x_at(p, m, cc) * __ldg(p.sal_scale + c + j);
+      int cc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) cc[j] = j < valid ? __ldg(p.sal_idx + c + j) : -1;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= valid) continue;
+        if (cc[j] >= 0 && cc[j] < p.xcols) v[j] = x_at(p, m, cc[j]) * __ldg(p.sal_scale + c + j);
         else if (part == 0) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
       }
     } else if (g.kind == kSegX) {
       if (p.xdt == BISCO_BF16 && split == 1 && p.x_vec && valid == 8)
         return __ldcg(reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned short*>(p.X) + static_cast<long long>(m) * p.ldx + c));
-      for (int j = 0; j < valid; ++j) v[j] = x_at(p, m, c + j);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = j < valid ? x_at(p, m, c + j) : 0.f;
     } else if (g.kind == kSegZ) {
-      for (int j = 0; j < valid; ++j) v[j] = __ldcg(p.Z + static_cast<long long>(m) * p.ldz + c + j);
+      const float* zr = p.Z + static_cast<long long>(m) * p.ldz + c;
+      if (p.z_vec && valid == 8) {  // two 16-byte loads
+        const float4 a = __ldcg(reinterpret_cast<const float4*>(zr));
+        const float4 b = __ldcg(reinterpret_cast<const float4*>(zr) + 1);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = j < valid ? __ldcg(zr + j) : 0.f;
+      }
     }
   }
   if (split == 2) {
@@ -245,22 +258,22 @@ __device__ __forceinline__ uint4 a_chunk(const PassParam& p, const TcSeg& g, int
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Expands columns 64h .. 64h+63 of row r of a step from the raw ring slot: 64 sign bits
+// Expands columns 32q .. 32q+31 of row r of a step from the raw ring slot: 32 sign bits
 // and the step's 128 column scales (bf16 bits; 1.0 when the segment has none, 0 past its
 // columns). A clear bit is the sign -1: the bf16 sign bit is set.
-__device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* raw, int r, int h, int ncols_left,
+__device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* raw, int r, int q, int ncols_left,
                                          bool has_cscale) {
-  const uint4 bw = *reinterpret_cast<const uint4*>(raw + r * 16);
-  const unsigned lo = h ? bw.z : bw.x, hi = h ? bw.w : bw.y;
+  const unsigned word = reinterpret_cast<const unsigned*>(raw + r * 16)[q];
   const unsigned short* cs = reinterpret_cast<const unsigned short*>(raw + kTcRows * 16);
-  // columns 64h.. are the h-th 64-column block: row r of it at h*128*128 + r*128, chunk j
-  // of the row at ((j ^ (r mod 8)) * 16)
-  unsigned char* rowp = A + h * (kTcRows * 128) + r * 128;
+  // columns 32q.. lie in the (q/2)-th 64-column block: row r of it at (q/2)*128*128 + r*128,
+  // chunk j of the row at ((j ^ (r mod 8)) * 16), j = 4(q mod 2) .. 4(q mod 2)+3
+  unsigned char* rowp = A + (q >> 1) * (kTcRows * 128) + r * 128;
   const int rx = r & 7;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int k8 = 8 * h + j;
-    const unsigned byte = ((j < 4 ? lo : hi) >> (8 * (j & 3))) & 0xFFu;
+  for (int jj = 0; jj < 4; ++jj) {
+    const int j = 4 * (q & 1) + jj;
+    const int k8 = 4 * q + jj;
+    const unsigned byte = (word >> (8 * jj)) & 0xFFu;
     unsigned c[4];
     if (has_cscale) {
       const uint4 cv = *reinterpret_cast<const uint4*>(cs + 8 * k8);
@@ -474,10 +487,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else {
         a_expand(A, raw_ring + (i % kTcRawSlots) * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7,
-                 g.ncols - c0, g.cscale != nullptr);
+                 g.ncols - c0, g.cscale != nullptr);  // 512 producers: 128 rows x 4 column quarters
       }
       const int brows = split * Np;
       if (!b_direct(seg)) {
+        // fp32-valued inputs (z, salient, fp32 X): loads of several chunks in flight at once
+#pragma unroll 4
         for (int ch = threadIdx.x; ch < brows * 16; ch += kTcProducers) {
           const int nn = ch % brows, k8 = ch / brows;
           const int part = nn / Np, m = nn - part * Np;
