@@ -436,20 +436,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!b_direct(sg)) return;
     const TcSeg g = tc_seg(p, sg);
     unsigned char* B = stages + static_cast<size_t>(j % nstages) * stage_bytes + a_bytes;
-    // chunk ch = k8 * Np + m; this thread takes ch = tid, tid + 256, ...: m and k8 advance
-    // by fixed steps (no division per chunk)
-    int m = threadIdx.x % Np, k8 = threadIdx.x / Np;
-    const int dm = kTcProducers % Np, dk = kTcProducers / Np;
+    // chunk ch = m * 16 + k8: consecutive lanes read consecutive 16-byte pieces of one
+    // activation row (two 256-byte rows per warp), so a warp's copies coalesce
     const int c_base = kt * kTcK;
     const unsigned short* xrow = reinterpret_cast<const unsigned short*>(p.X);
-    for (; k8 < 16; ) {
+    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
+      const int m = ch >> 4, k8 = ch & 15;
       const int c = c_base + 8 * k8;
       const int valid = (m < p.Mc) ? max(0, min(8, g.ncols - c)) : 0;
       const unsigned short* src = xrow + (valid > 0 ? static_cast<long long>(m) * p.ldx + c : 0);
       cp16(B + tile_off(m, k8, Np), src, static_cast<unsigned>(valid * 2));
-      m += dm;
-      k8 += dk;
-      if (m >= Np) { m -= Np; ++k8; }
     }
   };
   // accumulator blocks this CTA writes (every thread walks the steps)
@@ -494,7 +490,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // fp32-valued inputs (z, salient, fp32 X): loads of several chunks in flight at once
 #pragma unroll 4
         for (int ch = threadIdx.x; ch < brows * 16; ch += kTcProducers) {
-          const int nn = ch % brows, k8 = ch / brows;
+          const int nn = ch >> 4, k8 = ch & 15;  // lanes along a row: coalesced reads
           const int part = nn / Np, m = nn - part * Np;
           *reinterpret_cast<uint4*>(B + tile_off(nn, k8, brows)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
         }
