@@ -558,17 +558,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < 16; ++j) y[j] = 0.f;
       for (int b = 0; b < acc.nblk; ++b) {
         if (!((touched >> b) & 1u)) continue;
-        for (int part = 0; part < acc.split[b]; ++part) {
-          uint32_t v[16];
-          const uint32_t ta = lane_addr + static_cast<uint32_t>(acc.col[b] + part * Np + m0);
+        // both parts of the block in flight before one wait
+        uint32_t v0[16], v1[16];
+        const uint32_t ta = lane_addr + static_cast<uint32_t>(acc.col[b] + m0);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v0[0]), "=r"(v0[1]), "=r"(v0[2]), "=r"(v0[3]), "=r"(v0[4]), "=r"(v0[5]), "=r"(v0[6]), "=r"(v0[7]),
+              "=r"(v0[8]), "=r"(v0[9]), "=r"(v0[10]), "=r"(v0[11]), "=r"(v0[12]), "=r"(v0[13]), "=r"(v0[14]), "=r"(v0[15])
+            : "r"(ta));
+        const bool two = acc.split[b] == 2;
+        if (two)
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
-                "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-              : "r"(ta));
-          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+              : "=r"(v1[0]), "=r"(v1[1]), "=r"(v1[2]), "=r"(v1[3]), "=r"(v1[4]), "=r"(v1[5]), "=r"(v1[6]), "=r"(v1[7]),
+                "=r"(v1[8]), "=r"(v1[9]), "=r"(v1[10]), "=r"(v1[11]), "=r"(v1[12]), "=r"(v1[13]), "=r"(v1[14]), "=r"(v1[15])
+              : "r"(ta + static_cast<uint32_t>(Np)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-          for (int j = 0; j < 16; ++j) y[j] = fmaf(__uint_as_float(v[j]), rsv[b], y[j]);
+        for (int j = 0; j < 16; ++j) {
+          float t = __uint_as_float(v0[j]);
+          if (two) t += __uint_as_float(v1[j]);
+          y[j] = fmaf(t, rsv[b], y[j]);
         }
       }
       if (S > 1) {
@@ -596,12 +606,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int rr0 = rank * rows_per, rr1 = min(kTcRows, rr0 + rows_per);
     const int nr = rr1 - rr0;
     if (nr > 0) {
+      // (a) lanes along batch columns: 16-byte reads of recv[src][lr][m..m+3], sum in rank
+      //     order, into a transposed tile [m][lr] (row stride nr + 1: no bank conflicts)
+      float* tr = recv + static_cast<size_t>(S) * rows_per * Np;
+      const int tstride = nr + 1;
+      for (int idx = threadIdx.x; idx < nr * (Np / 4); idx += kTcThreads) {
+        const int lr = idx / (Np / 4), m4 = (idx - lr * (Np / 4)) * 4;
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < S; ++src) {
+          const float4 v = *reinterpret_cast<const float4*>(recv + (static_cast<size_t>(src) * rows_per + lr) * Np + m4);
+          sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+        }
+        tr[(m4 + 0) * tstride + lr] = sum.x;
+        tr[(m4 + 1) * tstride + lr] = sum.y;
+        tr[(m4 + 2) * tstride + lr] = sum.z;
+        tr[(m4 + 3) * tstride + lr] = sum.w;
+      }
+      __syncthreads();
+      // (b) lanes along output rows: coalesced stores of Y[m][o]
       for (int idx = threadIdx.x; idx < nr * Np; idx += kTcThreads) {
         const int m = idx / nr, lr = idx - m * nr;
         const int o = o0 + rr0 + lr;
         if (o >= p.rows || m >= p.Mc) continue;
-        float sum = 0.f;
-        for (int src = 0; src < S; ++src) sum += recv[(static_cast<size_t>(src) * rows_per + lr) * Np + m];
+        const float sum = tr[m * tstride + lr];
         if (p.ydt == BISCO_BF16)
           reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(sum);
         else
@@ -674,7 +701,8 @@ TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncol
   int S = std::max(1, std::min({kMaxCluster, nsteps, num_sms / std::max(1, t.tiles)}));
   while (S > 1 && (S & (S - 1))) --S;  // power of two
   for (; S >= 1; S /= 2) {
-    const size_t recv = static_cast<size_t>(S) * ((kTcRows + S - 1) / S) * t.Np * 4;
+    const size_t rows_per = (kTcRows + S - 1) / S;
+    const size_t recv = (static_cast<size_t>(S) * rows_per * t.Np + static_cast<size_t>(t.Np) * (rows_per + 1)) * 4;
     if (recv > static_cast<size_t>(t.stages) * stage) continue;
     if (tc_max_clusters(S, t.smem) >= 1) break;
   }
