@@ -535,11 +535,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cluster.barrier_wait(std::move(started));
   if (S > 1) cluster.sync();
   const int rows_per = (kTcRows + S - 1) / S;
-  if (warp < 4) {
-    // warp w reads tensor-memory lanes 32w..32w+31 = rows of this CTA's tile
-    const int r = warp * 32 + lane;
+  if (warp < kTcProducers / 32) {
+    // warp w reads tensor-memory lanes 32 (w mod 4) .. + 31 (= rows of this CTA's tile) and
+    // columns 16 (w / 4), + 64, ...: the 16 producer warps share the read-out
+    const int lg = warp & 3;
+    const int r = lg * 32 + lane;
     const int o = o0 + r;
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(lg * 32) << 16);
     float rsv[kTcMaxBlocks];
     for (int b = 0; b < acc.nblk; ++b) {
       rsv[b] = 1.f;
@@ -552,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int dst = r / rows_per;
     float* rp = S > 1 ? cluster.map_shared_rank(recv, dst) + (static_cast<size_t>(rank) * rows_per + (r - dst * rows_per)) * Np
                       : nullptr;
-    for (int m0 = 0; m0 < Np; m0 += 16) {
+    for (int m0 = 16 * (warp >> 2); m0 < Np; m0 += 16 * (kTcProducers / 128)) {
       float y[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) y[j] = 0.f;
