@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(kTW, 2) lut_gemv_warp_kernel(const __grid_cons
   __syncthreads();  // unit metadata visible
 
   // stage this warp's first items of chunk 0
-  ItemCursor ic;
+  ItemCursor ic{0, 0};
   int n_issue = 0;  // items of the current chunk issued so far by this warp
   auto issue = [&](int cu0, int cn) {  // stage the item under the issue cursor (one group)
     if (ic.ulc < cn) {

@@ -1,10 +1,10 @@
-"""GPU parity of the tensor-core path (batch chunks of 32..64 rows) against the oracle.
+"""GPU parity of the tensor-core path (batch chunks of 32..128 rows) against the oracle.
 
 bisco_gemv sends a batch chunk of at least 32 rows to the tensor cores when the layer's
 scales are bf16: the signs are expanded to bf16 tiles (column scale folded in, exact),
 fp32-valued inputs (the correction's z, salient inputs, fp32 activations) are split into
 high and low bf16 parts, and the products accumulate in fp32. The bars are those of
-tests/test_gemv_gpu.py. Batch sizes straddle the chunk boundaries (32, 64) so that
+tests/test_gemv_gpu.py. Batch sizes straddle the chunk boundaries (32, 128) so that
 mixed schedules (tensor-core chunks followed by lookup-table chunks) are covered too.
 """
 
@@ -30,8 +30,8 @@ CASES = [
     (300, 700, 2, 24, 0.02, 33, "bf16", "f32"),     # correction + salient
     (640, 1000, 1, 96, 0.01, 64, "bf16", "bf16"),
     (512, 1024, 2, 0, 0.0, 128, "bf16", "f32"),
-    (384, 640, 3, 40, 0.0, 130, "bf16", "f32"),     # 64 + 64 on the tensor cores + 2 on the LUT path
-    (160, 384, 2, 8, 0.03, 150, "bf16", "f32"),     # 64 + 64 + 22
+    (384, 640, 3, 40, 0.0, 130, "bf16", "f32"),     # 128 on the tensor cores + 2 on the LUT path
+    (160, 384, 2, 8, 0.03, 150, "bf16", "f32"),     # 128 + 22 (lookup-table chunks of 8, 8, 6)
     (257, 129, 4, 0, 0.0, 40, "bf16", "f32"),       # four bases
     (192, 512, 2, 17, 0.0, 48, "f32", "f32"),       # fp32 activations: split on the bases
     (128, 256, 0, 64, 0.05, 32, "bf16", "f32"),     # correction + salient, no base

@@ -57,7 +57,8 @@ def _rel_l2(a, b):
 def test_two_calls_in_a_row_match_the_workspace_entry_point():
     # call 1: a layer whose correction needs the scratch z; call 2: another layer and
     # batch size (two batch chunks), so state left in the shared array by call 1 must not leak
-    cases = [(640, 1000, 2, 96, 0.01, 3), (300, 520, 1, 40, 0.0, 11)]
+    # (a third call at batch 64 runs on the tensor cores, z of 64 rows in the scratch array)
+    cases = [(640, 1000, 2, 96, 0.01, 3), (300, 520, 1, 40, 0.0, 11), (256, 512, 2, 64, 0.02, 64)]
     for i, (out, in_, K, rank, sal, M) in enumerate(cases):
         X = make_activations(0, (500 + i,), M, in_, "bf16")
         L = make_layer(0, (500 + i,), out, in_, K, "bf16", rank=rank, sal_frac=sal,
