@@ -21,27 +21,33 @@
 // split value keeps 16 significant bits of its fp32 value.
 //
 // Work decomposition: cluster c owns 128 output rows; CTA r of the cluster takes 1/S of
-// the (segment, 128-column K tile) steps. A step's tiles live in a shared-memory stage,
-// K-major with the 128-byte swizzle: each tile is two blocks of 64 columns; a row of a
-// block is 128 bytes, its 16-byte chunks permuted by XOR with (row mod 8), and groups
-// of 8 rows are 1024 bytes apart. cp.async brings in the raw sign words and column
-// scales two steps ahead (a four-slot ring) and the bf16 activation tile of a step into
-// its stage. The warps are specialised: 16 producer warps wait until a stage is free,
-// copy the activation tile into it (completion counted on the stage's "full" mbarrier),
-// expand the step's signs from the raw ring and mark the stage full; one more warp waits
-// for each full stage, issues the step's eight K=16 MMAs and commits them to the stage's
-// "free" mbarrier, so expansion of later stages overlaps the MMAs of earlier ones. Every
-// waiter walks every stage in order, so one pair of barriers per stage slot suffices.
+// the (segment, 128-column K tile, part) steps, where a split segment (high and low bf16
+// parts) has two steps per K tile, one per part, into two column blocks of its
+// accumulator. A step's tiles live in a shared-memory stage, K-major with the 128-byte
+// swizzle: each tile is two blocks of 64 columns; a row of a block is 128 bytes, its
+// 16-byte chunks permuted by XOR with (row mod 8), and groups of 8 rows are 1024 bytes
+// apart. cp.async brings in the raw sign words and column scales two steps ahead (a
+// four-slot ring). A bf16 activation tile comes in through the tensor memory accelerator
+// (two 64-column boxes per step, written in the 128-byte swizzle by the copy engine and
+// counted in bytes on the stage's "full" mbarrier); fp32-valued B tiles are written by
+// the producers. The warps are specialised: 16 producer warps wait until a stage is
+// free, start its activation copy, expand the step's signs from the raw ring and mark
+// the stage full; one more warp waits for each full stage, issues the step's eight K=16
+// MMAs and commits them to the stage's "free" mbarrier, so expansion of later stages
+// overlaps the MMAs of earlier ones. Every waiter walks every stage in order, so one
+// pair of barriers per stage slot suffices.
 // The S partial results meet in distributed shared memory and are added in CTA-rank
 // order.
 // A CTA takes more than half of an SM's shared memory, so no two CTAs (each holding up
 // to 512 tensor-memory columns) ever share an SM.
 
 #include <cooperative_groups.h>
+#include <cuda.h>  // CUtensorMap and the tensor-map encoder's argument types (no driver library is linked)
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "bisco_internal.h"
@@ -52,14 +58,15 @@ namespace bisco {
 
 namespace {
 
-constexpr int kTcProducers = 512;              // 16 producer warps
-constexpr int kTcThreads = kTcProducers + 32;  // + 1 MMA warp
+constexpr int kTcProducers = 512;              // 16 producer (sign expansion) warps
+constexpr int kTcThreads = kTcProducers + 96;  // + 1 MMA warp + 2 loader warps (signs, activations)
 constexpr int kTcRows = 128;       // output rows per cluster (MMA M)
 constexpr int kTcK = 128;          // input columns per step (eight K=16 MMAs)
-constexpr int kTcMaxStages = 3;
-constexpr int kTcRawSlots = 4;     // raw sign-word / column-scale ring (prefetch distance 2)
+constexpr int kTcMaxStages = 4;
+constexpr int kTcRawSlots = 4;     // raw sign-word / column-scale ring
 constexpr int kTcRawBytes = kTcRows * 16 + kTcK * 2;  // 128 rows x 16 bytes + 128 bf16 scales
 constexpr int kTcMaxBlocks = kMaxSeg + 1;
+constexpr int kTcHeader = 2048;    // barriers and the segment table, ahead of the raw ring
 constexpr unsigned long long kTcWaitNs = 200000000ull;  // bound on every wait (200 ms)
 
 __device__ __forceinline__ unsigned saddr(const void* p) { return static_cast<unsigned>(__cvta_generic_to_shared(p)); }
@@ -85,11 +92,24 @@ __device__ __forceinline__ bool tc_try(uint64_t* b, unsigned parity) {
 __device__ __forceinline__ void bar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
 }
-// Arrives on b once all cp.async operations issued so far by this thread have completed.
+// Arrives on b and adds `bytes` to the transaction count of its current phase.
+__device__ __forceinline__ void bar_expect_tx(uint64_t* b, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes) : "memory");
+}
+// Arrives on b once all cp.async operations issued so far by this thread have completed
+// (the arrival is one of the phase's expected arrivals).
 __device__ __forceinline__ void bar_arrive_cp(uint64_t* b) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
 }
-__device__ __forceinline__ void producers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kTcProducers) : "memory"); }
+// One box of a 2-D tensor map into this CTA's shared memory; completion counted in
+// bytes on bar. Coordinates are (column, row) in elements; out-of-range elements read 0.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          saddr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(saddr(bar))
+      : "memory");
+}
 
 // Waits (bounded in time) until the phase with the given parity has completed.
 __device__ __forceinline__ bool tc_wait(uint64_t* b, unsigned parity) {
@@ -139,9 +159,6 @@ __device__ __forceinline__ unsigned tile_off(int row, int k8, int rows) {
 __device__ __forceinline__ void cp16(void* dst, const void* src, unsigned src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait2() { asm volatile("cp.async.wait_group 2;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -173,6 +190,35 @@ __device__ __forceinline__ TcSeg tc_seg(const PassParam& p, int s) {
   }
   return g;
 }
+
+// A launch's segments as the main loop reads them every step (a table in shared memory,
+// filled once per CTA: kernel parameters indexed by a run-time segment number are slow).
+struct TcSegInfo {
+  TcSeg g;
+  int parts;   // steps per K tile (2: high and low bf16 parts of fp32-valued B)
+  int ktiles;  // 128-column K tiles
+  int blk;     // accumulator block
+};
+
+// (segment, K tile, part) of a step; next() moves to the following step.
+struct TcCursor {
+  int seg, kt, part;
+  __device__ __forceinline__ void init(const TcSegInfo* si, int nseg_all, int step) {
+    seg = 0;
+    while (seg < nseg_all - 1 && step >= si[seg].ktiles * si[seg].parts) {
+      step -= si[seg].ktiles * si[seg].parts;
+      ++seg;
+    }
+    kt = step / si[seg].parts;
+    part = step - kt * si[seg].parts;
+  }
+  __device__ __forceinline__ void next(const TcSegInfo* si) {
+    if (++part == si[seg].parts) {
+      part = 0;
+      if (++kt == si[seg].ktiles) { kt = 0; ++seg; }
+    }
+  }
+};
 
 // 16 bytes of a B tile: columns c..c+7 of batch row m (part 0: the value or its high
 // bf16 part; part 1: the low part).
@@ -263,7 +309,7 @@ __device__ __forceinline__ uint4 a_chunk(const PassParam& p, const TcSeg& g, int
 // columns). A clear bit is the sign -1: the bf16 sign bit is set.
 __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* raw, int r, int q, int ncols_left,
                                          bool has_cscale) {
-  const unsigned word = reinterpret_cast<const unsigned*>(raw + r * 16)[q];
+  const unsigned nword = ~reinterpret_cast<const unsigned*>(raw + r * 16)[q];  // set bit: sign -1
   const unsigned short* cs = reinterpret_cast<const unsigned short*>(raw + kTcRows * 16);
   // columns 32q.. lie in the (q/2)-th 64-column block: row r of it at (q/2)*128*128 + r*128,
   // chunk j of the row at ((j ^ (r mod 8)) * 16), j = 4(q mod 2) .. 4(q mod 2)+3
@@ -273,7 +319,7 @@ __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* 
   for (int jj = 0; jj < 4; ++jj) {
     const int j = 4 * (q & 1) + jj;
     const int k8 = 4 * q + jj;
-    const unsigned byte = (word >> (8 * jj)) & 0xFFu;
+    const unsigned nbyte = nword >> (8 * jj);
     unsigned c[4];
     if (has_cscale) {
       const uint4 cv = *reinterpret_cast<const uint4*>(cs + 8 * k8);
@@ -283,12 +329,11 @@ __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* 
       for (int e = 0; e < 4; ++e)
         c[e] = (8 * k8 + 2 * e < ncols_left ? 0x3F80u : 0u) | ((8 * k8 + 2 * e + 1 < ncols_left ? 0x3F80u : 0u) << 16);
     }
+    // bits 2e and 2e+1 of the inverted byte become the sign bits (15, 31) of word e:
+    // b * 0x40008000 for b < 4 puts bit 0 of b at 15 and 30, bit 1 at 16 and 31 (no carries)
     unsigned w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const unsigned nb = ~(byte >> (2 * e));
-      w[e] = c[e] ^ (((nb & 1u) << 15) | ((nb & 2u) << 30));
-    }
+    for (int e = 0; e < 4; ++e) w[e] = c[e] ^ ((((nbyte >> (2 * e)) & 3u) * 0x40008000u) & 0x80008000u);
     *reinterpret_cast<uint4*>(rowp + ((j ^ rx) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
@@ -332,7 +377,8 @@ __host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, 
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ PassParam p, const int S, const int Np, const int nstages, const int tmem_cols) {
+    tc_gemm_kernel(const __grid_constant__ PassParam p, const __grid_constant__ CUtensorMap tmap_x, const int use_tma, const int S,
+                   const int Np, const int nstages, const int tmem_cols) {
   extern __shared__ __align__(1024) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -343,32 +389,45 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int kinds[kMaxSeg];
   for (int s = 0; s < kMaxSeg; ++s) kinds[s] = s < p.nseg ? p.seg[s].xsrc : kSegZ;
   const TcAcc acc = tc_acc(p.nseg, kinds, has_sal, p.xdt == BISCO_BF16, Np);
-  const unsigned a_bytes = kTcRows * kTcK * 2, b_bytes = static_cast<unsigned>(2 * Np) * kTcK * 2;
+  const unsigned a_bytes = kTcRows * kTcK * 2, b_bytes = static_cast<unsigned>(Np) * kTcK * 2;
   const unsigned stage_bytes = a_bytes + b_bytes;
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // [kTcMaxStages] stage filled
   uint64_t* mma_done = full + kTcMaxStages;                 // [kTcMaxStages] stage's MMAs done
   uint64_t* all_done = mma_done + kTcMaxStages;             // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(all_done + 1);
-  unsigned char* raw_ring = smem + 1024;                    // [kTcRawSlots][kTcRawBytes]
+  uint64_t* raw_full = all_done + 1;                        // [kTcRawSlots] raw slot landed
+  uint64_t* raw_free = raw_full + kTcRawSlots;              // [kTcRawSlots] raw slot read by every producer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_free + kTcRawSlots);
+  TcSegInfo* si = reinterpret_cast<TcSegInfo*>(smem + 256);  // [nseg_all]
+  unsigned char* raw_ring = smem + kTcHeader;               // [kTcRawSlots][kTcRawBytes]
   unsigned char* stages = raw_ring + kTcRawSlots * kTcRawBytes;
   float* recv = reinterpret_cast<float*>(stages);           // used after the main loop
 
-  // (segment, K tile) steps; this CTA's range
-  int steps_of[kTcMaxBlocks];
+  // (segment, K tile, part) steps; this CTA's range
   int nsteps = 0;
-  for (int s = 0; s < nseg_all; ++s) {
-    steps_of[s] = (tc_seg(p, s).ncols + kTcK - 1) / kTcK;
-    nsteps += steps_of[s];
-  }
+  for (int s = 0; s < nseg_all; ++s) nsteps += (tc_seg(p, s).ncols + kTcK - 1) / kTcK * acc.split[acc.blk_of_seg[s]];
   const int st0 = rank * nsteps / S, st1 = (rank + 1) * nsteps / S;
 
+  if (threadIdx.x < nseg_all) {
+    TcSegInfo& e = si[threadIdx.x];
+    e.g = tc_seg(p, threadIdx.x);
+    e.blk = acc.blk_of_seg[threadIdx.x];
+    e.parts = acc.split[e.blk];
+    e.ktiles = (e.g.ncols + kTcK - 1) / kTcK;
+  }
   if (threadIdx.x == 0) {
-    // full: one cp.async-completion arrival and one plain arrival per producer thread
+    // full: one arrival per producer thread once its part of the stage is written, plus
+    // one by the loader when it starts the stage's activation copy (with its byte count)
     for (int s = 0; s < kTcMaxStages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(full + s)), "r"(2 * kTcProducers) : "memory");
-    for (int s = 0; s <= kTcMaxStages; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(full + s)), "r"(kTcProducers + 1) : "memory");
+    for (int s = 0; s <= kTcMaxStages; ++s)  // mma_done[] and all_done
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mma_done + s)) : "memory");
+    // raw_full: two arrivals per loader lane (its copies landed; its plain stores done);
+    // raw_free: every producer thread
+    for (int s = 0; s < kTcRawSlots; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_full + s)), "r"(64) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_free + s)), "r"(kTcProducers) : "memory");
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -384,95 +443,94 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // that every CTA of the cluster is running.
   auto started = cluster.barrier_arrive();
 
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-
   bool ok = true;
-  unsigned touched = 0;  // accumulator blocks written by this CTA (same in every thread)
+  unsigned touched = 0;  // bit 2 b + part: accumulator columns written by this CTA (same in every thread)
   const int n = st1 - st0;
-  // (segment, K tile) of the CTA-local step j
-  auto step_pos = [&](int j, int& sg, int& kt) {
-    int rem = st0 + j;
-    sg = 0;
-    while (sg < nseg_all - 1 && rem >= steps_of[sg]) { rem -= steps_of[sg]; ++sg; }
-    kt = rem;
-  };
-  const int tile_rows = ((p.rows + 31) / 32) * 32;  // rows present in the packed layout
-  // raw sign words (128 rows x 16 bytes) and column scales of step j -> ring slot j % 4
-  auto issue_raw = [&](int j) {
-    int sg, kt;
-    step_pos(j, sg, kt);
-    const TcSeg g = tc_seg(p, sg);
-    if (g.kind == kSegSal || g.bits == nullptr) return;
-    unsigned char* dst = raw_ring + (j % kTcRawSlots) * kTcRawBytes;
-    if (threadIdx.x < kTcRows) {
-      const int o = o0 + threadIdx.x;
-      const bool in = o < tile_rows;
-      const uint4* src = g.bits + (static_cast<long long>(in ? o >> 5 : 0) * g.nq + kt) * 32 + (in ? (o & 31) : 0);
-      cp16(dst + threadIdx.x * 16, src, in ? 16u : 0u);
-    } else if (g.cscale != nullptr && threadIdx.x < kTcRows + kTcK / 8) {
-      const int cc = kt * kTcK + (threadIdx.x - kTcRows) * 8;
-      const int valid = max(0, min(8, g.ncols - cc));
-      unsigned char* cd = dst + kTcRows * 16 + (threadIdx.x - kTcRows) * 16;
-      const unsigned short* cs = reinterpret_cast<const unsigned short*>(g.cscale);
-      if (g.cvec) {  // 16-byte aligned scales: asynchronous copy with zero fill
-        cp16(cd, cs + (valid > 0 ? cc : 0), static_cast<unsigned>(valid * 2));
-      } else {       // unaligned (e.g. the second base of a layer with in % 8 != 0): plain loads
-        unsigned short v[8];
+  const int tiles_here = min(4, (p.rows + 31) / 32 - o0 / 32);  // 32-row tiles of this block in the packed layout
+  // accumulator blocks this CTA writes (every thread walks the steps)
+  TcCursor cur;
+  cur.init(si, nseg_all, st0);
+  for (int i = 0; i < n; ++i, cur.next(si)) touched |= 1u << (2 * si[cur.seg].blk + cur.part);
+  cur.init(si, nseg_all, st0);
+
+  if (warp == kTcProducers / 32 + 1) {
+    // ---------------- sign loader warp ----------------
+    // Raw sign words (32 rows x 16 bytes of each of the four row tiles of the packed
+    // layout; lane l copies row l of every tile, so a warp's copies are 512 contiguous
+    // bytes) and the step's 128 column scales go to raw slot i % 4 with cp.async (bulk
+    // copies issued back to back by one thread are served one after another), up to four
+    // steps ahead of the producers. Sign words never depend on the previous kernel, so the
+    // first slots are filled before the dependency wait.
+    for (int i = 0; i < n; ++i) {
+      const int rs = i % kTcRawSlots;
+      if (i >= kTcRawSlots && !tc_wait(raw_free + rs, static_cast<unsigned>(i / kTcRawSlots - 1) & 1u)) ok = false;
+      const TcSeg& g = si[cur.seg].g;
+      unsigned char* dst = raw_ring + rs * kTcRawBytes;
+      const bool bits = g.kind != kSegSal && g.bits != nullptr;
+      if (bits) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = e < valid ? __ldg(cs + cc + e) : 0;
-        *reinterpret_cast<uint4*>(cd) = make_uint4(v[0] | (static_cast<unsigned>(v[1]) << 16), v[2] | (static_cast<unsigned>(v[3]) << 16),
-                                                   v[4] | (static_cast<unsigned>(v[5]) << 16), v[6] | (static_cast<unsigned>(v[7]) << 16));
+        for (int t = 0; t < 4; ++t) {  // row 32 t + lane; rows past the layout's tiles read 0
+          const bool in = t < tiles_here;
+          const uint4* src = g.bits + (static_cast<long long>(in ? o0 / 32 + t : 0) * g.nq + cur.kt) * 32 + lane;
+          cp16(dst + (t * 32 + lane) * 16, src, in ? 16u : 0u);
+        }
+      }
+      if (lane < kTcK / 8) {
+        // column scales (bf16) for columns 8 lane .. + 7 of the K tile, zero past the segment
+        if (bits && g.cscale != nullptr) {
+          const int cc = cur.kt * kTcK + lane * 8;
+          const int valid = max(0, min(8, g.ncols - cc));
+          unsigned char* cd = dst + kTcRows * 16 + lane * 16;
+          const unsigned short* cs = reinterpret_cast<const unsigned short*>(g.cscale);
+          if (g.cvec) {  // 16-byte aligned scales: asynchronous copy with zero fill
+            cp16(cd, cs + (valid > 0 ? cc : 0), static_cast<unsigned>(valid * 2));
+          } else {       // unaligned (e.g. the second base of a layer with in % 8 != 0): plain loads
+            unsigned short v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = e < valid ? __ldg(cs + cc + e) : 0;
+            *reinterpret_cast<uint4*>(cd) =
+                make_uint4(v[0] | (static_cast<unsigned>(v[1]) << 16), v[2] | (static_cast<unsigned>(v[3]) << 16),
+                           v[4] | (static_cast<unsigned>(v[5]) << 16), v[6] | (static_cast<unsigned>(v[7]) << 16));
+          }
+        }
+      }
+      bar_arrive_cp(raw_full + rs);  // once this lane's copies have landed
+      bar_arrive(raw_full + rs);     // this lane's plain stores (release)
+      cur.next(si);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  } else if (warp == kTcProducers / 32 + 2) {
+    // ---------------- activation loader warp ----------------
+    // The activation tile of step j goes into its stage as soon as the MMAs that last
+    // read the stage are done (tensor-map copies, or one arrival when the producers write
+    // the B tile themselves).
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // activations may come from the previous kernel
+    for (int j = 0; j < n; ++j, cur.next(si)) {
+      const int sl = j % nstages;
+      if (j >= nstages && !tc_wait(mma_done + sl, static_cast<unsigned>(j / nstages - 1) & 1u)) ok = false;
+      unsigned char* B = stages + static_cast<size_t>(sl) * stage_bytes + a_bytes;
+      if (use_tma && si[cur.seg].g.kind == kSegX) {
+        // both 64-column blocks (rows past the batch read 0), one box from each of lanes 0, 1
+        if (lane == 0) bar_expect_tx(full + sl, b_bytes);
+        __syncwarp();
+        if (lane < 2) tma_load_2d(B + lane * Np * 128, &tmap_x, cur.kt * kTcK + lane * 64, 0, full + sl);
+      } else if (lane == 0) {
+        bar_arrive(full + sl);
       }
     }
-  };
-  // bf16 activation tile of step j straight into its stage (bases over bf16 X only)
-  auto b_direct = [&](int sg) {
-    const TcSeg g = tc_seg(p, sg);
-    return g.kind == kSegX && p.xdt == BISCO_BF16 && p.x_vec;
-  };
-  auto issue_b = [&](int j) {
-    int sg, kt;
-    step_pos(j, sg, kt);
-    if (!b_direct(sg)) return;
-    const TcSeg g = tc_seg(p, sg);
-    unsigned char* B = stages + static_cast<size_t>(j % nstages) * stage_bytes + a_bytes;
-    // chunk ch = m * 16 + k8: consecutive lanes read consecutive 16-byte pieces of one
-    // activation row (two 256-byte rows per warp), so a warp's copies coalesce
-    const int c_base = kt * kTcK;
-    const unsigned short* xrow = reinterpret_cast<const unsigned short*>(p.X);
-    for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
-      const int m = ch >> 4, k8 = ch & 15;
-      const int c = c_base + 8 * k8;
-      const int valid = (m < p.Mc) ? max(0, min(8, g.ncols - c)) : 0;
-      const unsigned short* src = xrow + (valid > 0 ? static_cast<long long>(m) * p.ldx + c : 0);
-      cp16(B + tile_off(m, k8, Np), src, static_cast<unsigned>(valid * 2));
-    }
-  };
-  // accumulator blocks this CTA writes (every thread walks the steps)
-  for (int i = 0; i < n; ++i) {
-    int sg, kt;
-    step_pos(i, sg, kt);
-    touched |= 1u << acc.blk_of_seg[sg];
+  } else {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
   }
   if (warp < kTcProducers / 32) {
     // ---------------- producers ----------------
-    if (n > 0) issue_raw(0);
-    if (n > 1) issue_raw(1);
-    cp_commit();
-    for (int i = 0; i < n; ++i) {
-      const int sl = i % nstages;
+    for (int i = 0; i < n; ++i, cur.next(si)) {
+      const int sl = i % nstages, rs = i % kTcRawSlots;
       // the stage is free once the MMAs that last read it are done
       if (i >= nstages && !tc_wait(mma_done + sl, static_cast<unsigned>(i / nstages - 1) & 1u)) ok = false;
-      issue_b(i);
-      bar_arrive_cp(full + sl);
-      if (i + 2 < n) issue_raw(i + 2);
-      cp_commit();
-      if (i == 0) cp_wait1(); else cp_wait2();  // this thread's copies of step i's raw data
-      producers_sync();                         // ... and every producer's
-      int seg, kt;
-      step_pos(i, seg, kt);
-      const TcSeg g = tc_seg(p, seg);
-      const int split = acc.split[acc.blk_of_seg[seg]];
+      if (!tc_wait(raw_full + rs, static_cast<unsigned>(i / kTcRawSlots) & 1u)) ok = false;
+      const int seg = cur.seg, kt = cur.kt, part = cur.part;
+      const TcSeg& g = si[seg].g;
+      const int split = si[seg].parts;
       unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
       unsigned char* B = A + a_bytes;
       const int c0 = kt * kTcK;
@@ -482,50 +540,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = a_chunk(p, g, o0 + r, c0 + 8 * k8);
         }
       } else {
-        a_expand(A, raw_ring + (i % kTcRawSlots) * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7,
-                 g.ncols - c0, g.cscale != nullptr);  // 512 producers: 128 rows x 4 column quarters
+        a_expand(A, raw_ring + rs * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7, g.ncols - c0,
+                 g.cscale != nullptr);  // 512 producers: 128 rows x 4 column quarters
       }
-      const int brows = split * Np;
-      if (!b_direct(seg)) {
-        // fp32-valued inputs (z, salient, fp32 X): loads of several chunks in flight at once
+      if (!(use_tma && g.kind == kSegX)) {
+        // fp32-valued inputs (z, salient, fp32 X) and unaligned bf16 X: several chunks in flight
 #pragma unroll 4
-        for (int ch = threadIdx.x; ch < brows * 16; ch += kTcProducers) {
-          const int nn = ch >> 4, k8 = ch & 15;  // lanes along a row: coalesced reads
-          const int part = nn / Np, m = nn - part * Np;
-          *reinterpret_cast<uint4*>(B + tile_off(nn, k8, brows)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
+        for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
+          const int m = ch >> 4, k8 = ch & 15;  // lanes along a row: coalesced reads
+          *reinterpret_cast<uint4*>(B + tile_off(m, k8, Np)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
         }
       }
       // make the generic-proxy stores visible to the tensor core, then mark the stage full
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       bar_arrive(full + sl);
+      bar_arrive(raw_free + rs);
     }
-  } else if (lane == 0) {
+  } else if (warp == kTcProducers / 32 && lane == 0) {
     // ---------------- MMA issue (one thread) ----------------
-    unsigned written = 0;
-    for (int i = 0; i < n; ++i) {
+    unsigned written = 0;  // bit 2 b + part: accumulator columns already written
+    const uint32_t idesc = mma_idesc(Np);
+    for (int i = 0; i < n; ++i, cur.next(si)) {
       const int sl = i % nstages;
       if (!tc_wait(full + sl, static_cast<unsigned>(i / nstages) & 1u)) ok = false;
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // cp.async-written activations
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      int seg, kt;
-      step_pos(i, seg, kt);
-      const int blk = acc.blk_of_seg[seg];
-      const int brows = acc.split[blk] * Np;
+      const int blk = si[cur.seg].blk, part = cur.part;
       unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
       unsigned char* B = A + a_bytes;
-      const uint32_t idesc = mma_idesc(brows);
-      const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk]);
-      const bool first = !((written >> blk) & 1u);
+      const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk] + part * Np);
+      const unsigned bit = 1u << (2 * blk + part);
+      const bool first = !(written & bit);
 #pragma unroll
       for (int kk = 0; kk < kTcK / 16; ++kk) {
         const unsigned koff = (kk & 3) * 32u;  // K step inside a 64-column block
         mma_bf16(d, smem_desc_sw128(A + (kk >> 2) * (kTcRows * 128) + koff),
-                 smem_desc_sw128(B + (kk >> 2) * (brows * 128) + koff), idesc, (first && kk == 0) ? 0u : 1u);
+                 smem_desc_sw128(B + (kk >> 2) * (Np * 128) + koff), idesc, (first && kk == 0) ? 0u : 1u);
       }
       mma_commit(mma_done + sl);
-      written |= 1u << blk;
+      written |= bit;
     }
     mma_commit(all_done);
+  }
+  // row scales of this thread's epilogue row, loaded while the last MMAs run
+  float rsv[kTcMaxBlocks];
+  {
+    const int o = o0 + (warp & 3) * 32 + lane;
+    for (int b = 0; b < acc.nblk; ++b) {
+      rsv[b] = 1.f;
+      const int s = acc.rseg[b];
+      if (s >= 0 && o < p.rows && p.seg[s].rscale != nullptr)
+        rsv[b] = p.seg[s].rdt == BISCO_BF16
+                     ? __uint_as_float(static_cast<unsigned>(__ldg(reinterpret_cast<const unsigned short*>(p.seg[s].rscale) + o)) << 16)
+                     : __ldg(reinterpret_cast<const float*>(p.seg[s].rscale) + o);
+    }
   }
   __syncwarp();
   if (!tc_wait(all_done, 0u)) ok = false;
@@ -535,6 +602,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   cluster.barrier_wait(std::move(started));
   if (S > 1) cluster.sync();
   const int rows_per = (kTcRows + S - 1) / S;
+  // recv[src][row][m] with a row stride of Np + 4 floats: a warp's 32 rows then start in
+  // 32 different banks (a stride of Np floats put every lane's 16-byte pushes into the same
+  // four banks)
+  const int rstride = Np + 4;
   if (warp < kTcProducers / 32) {
     // warp w reads tensor-memory lanes 32 (w mod 4) .. + 31 (= rows of this CTA's tile) and
     // columns 16 (w / 4), + 64, ...: the 16 producer warps share the read-out
@@ -542,34 +613,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = lg * 32 + lane;
     const int o = o0 + r;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(lg * 32) << 16);
-    float rsv[kTcMaxBlocks];
-    for (int b = 0; b < acc.nblk; ++b) {
-      rsv[b] = 1.f;
-      const int s = acc.rseg[b];
-      if (s >= 0 && o < p.rows && p.seg[s].rscale != nullptr)
-        rsv[b] = p.seg[s].rdt == BISCO_BF16
-                     ? __uint_as_float(static_cast<unsigned>(__ldg(reinterpret_cast<const unsigned short*>(p.seg[s].rscale) + o)) << 16)
-                     : __ldg(reinterpret_cast<const float*>(p.seg[s].rscale) + o);
-    }
     const int dst = r / rows_per;
-    float* rp = S > 1 ? cluster.map_shared_rank(recv, dst) + (static_cast<size_t>(rank) * rows_per + (r - dst * rows_per)) * Np
+    float* rp = S > 1 ? cluster.map_shared_rank(recv, dst) + (static_cast<size_t>(rank) * rows_per + (r - dst * rows_per)) * rstride
                       : nullptr;
     for (int m0 = 16 * (warp >> 2); m0 < Np; m0 += 16 * (kTcProducers / 128)) {
       float y[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) y[j] = 0.f;
       for (int b = 0; b < acc.nblk; ++b) {
-        if (!((touched >> b) & 1u)) continue;
-        // both parts of the block in flight before one wait
+        // a CTA whose steps cover one part of a split block only reads that part
+        const bool t0 = (touched >> (2 * b)) & 1u, t1 = (touched >> (2 * b + 1)) & 1u;
+        if (!t0 && !t1) continue;
+        // the block's parts in flight before one wait
         uint32_t v0[16], v1[16];
         const uint32_t ta = lane_addr + static_cast<uint32_t>(acc.col[b] + m0);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-            : "=r"(v0[0]), "=r"(v0[1]), "=r"(v0[2]), "=r"(v0[3]), "=r"(v0[4]), "=r"(v0[5]), "=r"(v0[6]), "=r"(v0[7]),
-              "=r"(v0[8]), "=r"(v0[9]), "=r"(v0[10]), "=r"(v0[11]), "=r"(v0[12]), "=r"(v0[13]), "=r"(v0[14]), "=r"(v0[15])
-            : "r"(ta));
-        const bool two = acc.split[b] == 2;
-        if (two)
+        if (t0)
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+              : "=r"(v0[0]), "=r"(v0[1]), "=r"(v0[2]), "=r"(v0[3]), "=r"(v0[4]), "=r"(v0[5]), "=r"(v0[6]), "=r"(v0[7]),
+                "=r"(v0[8]), "=r"(v0[9]), "=r"(v0[10]), "=r"(v0[11]), "=r"(v0[12]), "=r"(v0[13]), "=r"(v0[14]), "=r"(v0[15])
+              : "r"(ta));
+        if (t1)
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
               : "=r"(v1[0]), "=r"(v1[1]), "=r"(v1[2]), "=r"(v1[3]), "=r"(v1[4]), "=r"(v1[5]), "=r"(v1[6]), "=r"(v1[7]),
@@ -578,8 +642,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          float t = __uint_as_float(v0[j]);
-          if (two) t += __uint_as_float(v1[j]);
+          const float t = (t0 ? __uint_as_float(v0[j]) : 0.f) + (t1 ? __uint_as_float(v1[j]) : 0.f);
           y[j] = fmaf(t, rsv[b], y[j]);
         }
       }
@@ -610,13 +673,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (nr > 0) {
       // (a) lanes along batch columns: 16-byte reads of recv[src][lr][m..m+3], sum in rank
       //     order, into a transposed tile [m][lr] (row stride nr + 1: no bank conflicts)
-      float* tr = recv + static_cast<size_t>(S) * rows_per * Np;
+      float* tr = recv + static_cast<size_t>(S) * rows_per * rstride;
       const int tstride = nr + 1;
       for (int idx = threadIdx.x; idx < nr * (Np / 4); idx += kTcThreads) {
         const int lr = idx / (Np / 4), m4 = (idx - lr * (Np / 4)) * 4;
         float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int src = 0; src < S; ++src) {
-          const float4 v = *reinterpret_cast<const float4*>(recv + (static_cast<size_t>(src) * rows_per + lr) * Np + m4);
+          const float4 v = *reinterpret_cast<const float4*>(recv + (static_cast<size_t>(src) * rows_per + lr) * rstride + m4);
           sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
         }
         tr[(m4 + 0) * tstride + lr] = sum.x;
@@ -662,6 +725,45 @@ int tc_max_clusters(int S, size_t smem) {
   return n;
 }
 
+// The driver's tensor-map encoder, looked up once through the runtime (no link-time
+// dependency on the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map of the launch's activation rows X[0 .. Mc)[0 .. xcols) (bf16, row stride ldx
+// elements): boxes of 64 columns (128 bytes) x Np rows in the 128-byte swizzle, the layout
+// the MMA descriptors expect; rows Mc .. Np-1 and columns past xcols read as zero.
+// False when the launch has no binary base over X, X is not bf16, or its rows are not
+// 16-byte aligned (the producers then write the B tiles).
+bool x_tensor_map(const PassParam& p, int Np, CUtensorMap* map) {
+  if (p.xdt != BISCO_BF16 || !p.x_vec || p.Mc <= 0 || p.xcols <= 0 || Np > 256) return false;
+  bool has_x = false;
+  for (int s = 0; s < p.nseg; ++s) has_x = has_x || (p.seg[s].xsrc == kSegX && p.seg[s].bits != nullptr);
+  if (!has_x) return false;
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.xcols), static_cast<cuuint64_t>(p.Mc)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.ldx) * 2};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(Np)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p.X), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t tc_ensure_attrs() {
@@ -686,11 +788,11 @@ TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncol
   t.tmem_cols = 32;
   while (t.tmem_cols < acc.ncols) t.tmem_cols *= 2;
   int nsteps = 0;
-  for (int s = 0; s < nseg; ++s) nsteps += (seg_ncols[s] + kTcK - 1) / kTcK;
-  if (n_sal > 0) nsteps += (n_sal + kTcK - 1) / kTcK;
+  for (int s = 0; s < nseg; ++s) nsteps += (seg_ncols[s] + kTcK - 1) / kTcK * acc.split[acc.blk_of_seg[s]];
+  if (n_sal > 0) nsteps += (n_sal + kTcK - 1) / kTcK * 2;
   if (nsteps == 0) return t;
-  const size_t stage = static_cast<size_t>(kTcRows) * kTcK * 2 + static_cast<size_t>(2 * t.Np) * kTcK * 2;
-  const size_t fixed = 1024 + static_cast<size_t>(kTcRawSlots) * kTcRawBytes;
+  const size_t stage = static_cast<size_t>(kTcRows) * kTcK * 2 + static_cast<size_t>(t.Np) * kTcK * 2;
+  const size_t fixed = kTcHeader + static_cast<size_t>(kTcRawSlots) * kTcRawBytes;
   t.stages = static_cast<int>(std::min<size_t>(kTcMaxStages, (smem_limit - fixed) / stage));
   if (t.stages < 2) return t;
   // more than half of the SM's shared memory: one CTA per SM (tensor memory is not shared)
@@ -704,7 +806,7 @@ TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncol
   while (S > 1 && (S & (S - 1))) --S;  // power of two
   for (; S >= 1; S /= 2) {
     const size_t rows_per = (kTcRows + S - 1) / S;
-    const size_t recv = (static_cast<size_t>(S) * rows_per * t.Np + static_cast<size_t>(t.Np) * (rows_per + 1)) * 4;
+    const size_t recv = (static_cast<size_t>(S) * rows_per * (t.Np + 4) + static_cast<size_t>(t.Np) * (rows_per + 1)) * 4;
     if (recv > static_cast<size_t>(t.stages) * stage) continue;
     if (tc_max_clusters(S, t.smem) >= 1) break;
   }
@@ -730,7 +832,10 @@ cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream) 
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, t.S, t.Np, t.stages, t.tmem_cols);
+  CUtensorMap map;
+  std::memset(&map, 0, sizeof(map));
+  const int use_tma = x_tensor_map(p, t.Np, &map) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, map, use_tma, t.S, t.Np, t.stages, t.tmem_cols);
 }
 
 }  // namespace bisco
