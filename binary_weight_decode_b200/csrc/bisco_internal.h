@@ -90,8 +90,10 @@ constexpr int kTcMinBatch = 32;           // smallest batch chunk sent to the te
 constexpr int kTcMaxBatch = 128;          // batch rows per launch
 struct TcPlan {
   int Np;                // batch rows padded to a multiple of 16 (MMA N per part)
-  int tmem_cols;         // tensor-memory columns allocated per CTA
-  int stages;            // shared-memory stages
+  int a_base;            // first tensor-memory column of the expanded sign tiles (after the accumulators)
+  int astages;           // sign-tile stages in tensor memory (64 columns each)
+  int stages;            // activation-tile stages in shared memory
+  int raw_slots;         // sign-word ring slots in shared memory (one step each)
   int tiles;             // 128-row output tiles (clusters)
   int S;                 // CTAs per cluster (K split); 0 = plan not possible
   size_t smem;

@@ -62,11 +62,14 @@ constexpr int kTcProducers = 512;              // 16 producer (sign expansion) w
 constexpr int kTcThreads = kTcProducers + 96;  // + 1 MMA warp + 2 loader warps (signs, activations)
 constexpr int kTcRows = 128;       // output rows per cluster (MMA M)
 constexpr int kTcK = 128;          // input columns per step (eight K=16 MMAs)
-constexpr int kTcMaxStages = 4;
-constexpr int kTcRawSlots = 4;     // raw sign-word / column-scale ring
+constexpr int kTcMaxAStages = 4;   // expanded sign tiles in tensor memory (64 columns each)
+constexpr int kTcMaxBStages = 6;   // activation tiles in shared memory
+constexpr int kTcTmemCols = 512;   // the whole tensor memory (one CTA per SM)
+constexpr int kTcMaxRaw = 64;      // raw sign-word / column-scale ring slots (as many as shared memory holds)
 constexpr int kTcRawBytes = kTcRows * 16 + kTcK * 2;  // 128 rows x 16 bytes + 128 bf16 scales
 constexpr int kTcMaxBlocks = kMaxSeg + 1;
 constexpr int kTcHeader = 2048;    // barriers and the segment table, ahead of the raw ring
+constexpr int kTcSegTable = 1280;  // offset of the segment table in the header
 constexpr unsigned long long kTcWaitNs = 200000000ull;  // bound on every wait (200 ms)
 
 __device__ __forceinline__ unsigned saddr(const void* p) { return static_cast<unsigned>(__cvta_generic_to_shared(p)); }
@@ -136,13 +139,18 @@ __device__ __forceinline__ uint32_t mma_idesc(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(kTcRows >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
+// D (tensor memory) (+)= A (tensor memory: lane = row, two bf16 per column along K)
+// x B (shared memory, descriptor). No memory clobber: the issuing thread touches none of
+// the operands; the mbarrier waits before and the commit after order the data, and
+// volatile statements keep their order. (With the operand addresses computed ahead, the
+// MMAs of a step issue back to back at the tensor core's rate: measured 64 cycles per
+// 128 x 128 x 16 MMA, against 82 with a memory clobber and 143 with A in shared memory.)
+__device__ __forceinline__ void mma_ts_bf16(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.u32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* b) {
@@ -304,20 +312,16 @@ __device__ __forceinline__ uint4 a_chunk(const PassParam& p, const TcSeg& g, int
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Expands columns 32q .. 32q+31 of row r of a step from the raw ring slot: 32 sign bits
-// and the step's 128 column scales (bf16 bits; 1.0 when the segment has none, 0 past its
+// Expands columns 32q .. 32q+31 of row r of a step from the raw ring slot into 16
+// words of bf16 pairs (column 32q + 2t in the low half of word t): 32 sign bits and the
+// step's 128 column scales (bf16 bits; 1.0 when the segment has none, 0 past its
 // columns). A clear bit is the sign -1: the bf16 sign bit is set.
-__device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* raw, int r, int q, int ncols_left,
-                                         bool has_cscale) {
+__device__ __forceinline__ void a_words(uint32_t (&w)[16], const unsigned char* raw, int r, int q, int ncols_left,
+                                        bool has_cscale) {
   const unsigned nword = ~reinterpret_cast<const unsigned*>(raw + r * 16)[q];  // set bit: sign -1
   const unsigned short* cs = reinterpret_cast<const unsigned short*>(raw + kTcRows * 16);
-  // columns 32q.. lie in the (q/2)-th 64-column block: row r of it at (q/2)*128*128 + r*128,
-  // chunk j of the row at ((j ^ (r mod 8)) * 16), j = 4(q mod 2) .. 4(q mod 2)+3
-  unsigned char* rowp = A + (q >> 1) * (kTcRows * 128) + r * 128;
-  const int rx = r & 7;
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
-    const int j = 4 * (q & 1) + jj;
     const int k8 = 4 * q + jj;
     const unsigned nbyte = nword >> (8 * jj);
     unsigned c[4];
@@ -331,19 +335,27 @@ __device__ __forceinline__ void a_expand(unsigned char* A, const unsigned char* 
     }
     // bits 2e and 2e+1 of the inverted byte become the sign bits (15, 31) of word e:
     // b * 0x40008000 for b < 4 puts bit 0 of b at 15 and 30, bit 1 at 16 and 31 (no carries)
-    unsigned w[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) w[e] = c[e] ^ ((((nbyte >> (2 * e)) & 3u) * 0x40008000u) & 0x80008000u);
-    *reinterpret_cast<uint4*>(rowp + ((j ^ rx) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    for (int e = 0; e < 4; ++e) w[4 * jj + e] = c[e] ^ ((((nbyte >> (2 * e)) & 3u) * 0x40008000u) & 0x80008000u);
   }
+}
+
+// Stores 16 consecutive 32-bit tensor-memory columns of this thread's lane (the warp's
+// 32 lanes at once).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]), "r"(w[10]),
+      "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
+      : "memory");
 }
 
 // Accumulator blocks in tensor memory: one per X segment (row scale applied in the
 // epilogue), one shared by U^T and the salient columns.
 struct TcAcc {
   int nblk;
-  int col[kTcMaxBlocks];    // first column
-  int split[kTcMaxBlocks];  // 1 or 2 parts of Np columns
+  int col[kTcMaxBlocks];    // first of the block's Np columns
+  int split[kTcMaxBlocks];  // 1 or 2 parts (steps per K tile, accumulated into the same columns)
   int rseg[kTcMaxBlocks];   // segment whose row scale applies (-1: none)
   int blk_of_seg[kTcMaxBlocks];
   int ncols;
@@ -359,7 +371,7 @@ __host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, 
       a.col[b] = col;
       a.split[b] = x_bf16 ? 1 : 2;
       a.rseg[b] = s;
-      col += a.split[b] * Np;
+      col += Np;
       a.blk_of_seg[s] = b;
     } else {
       if (shared < 0) {
@@ -367,7 +379,7 @@ __host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, 
         a.col[shared] = col;
         a.split[shared] = 2;
         a.rseg[shared] = -1;
-        col += 2 * Np;
+        col += Np;
       }
       a.blk_of_seg[s] = shared;
     }
@@ -378,7 +390,7 @@ __host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, 
 
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ PassParam p, const __grid_constant__ CUtensorMap tmap_x, const int use_tma, const int S,
-                   const int Np, const int nstages, const int tmem_cols) {
+                   const int Np, const int nA, const int nB, const int R, const int a_base) {
   extern __shared__ __align__(1024) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -389,19 +401,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int kinds[kMaxSeg];
   for (int s = 0; s < kMaxSeg; ++s) kinds[s] = s < p.nseg ? p.seg[s].xsrc : kSegZ;
   const TcAcc acc = tc_acc(p.nseg, kinds, has_sal, p.xdt == BISCO_BF16, Np);
-  const unsigned a_bytes = kTcRows * kTcK * 2, b_bytes = static_cast<unsigned>(Np) * kTcK * 2;
-  const unsigned stage_bytes = a_bytes + b_bytes;
+  const unsigned b_bytes = static_cast<unsigned>(Np) * kTcK * 2;  // one activation stage
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);       // [kTcMaxStages] stage filled
-  uint64_t* mma_done = full + kTcMaxStages;                 // [kTcMaxStages] stage's MMAs done
-  uint64_t* all_done = mma_done + kTcMaxStages;             // [1]
-  uint64_t* raw_full = all_done + 1;                        // [kTcRawSlots] raw slot landed
-  uint64_t* raw_free = raw_full + kTcRawSlots;              // [kTcRawSlots] raw slot read by every producer
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_free + kTcRawSlots);
-  TcSegInfo* si = reinterpret_cast<TcSegInfo*>(smem + 256);  // [nseg_all]
-  unsigned char* raw_ring = smem + kTcHeader;               // [kTcRawSlots][kTcRawBytes]
-  unsigned char* stages = raw_ring + kTcRawSlots * kTcRawBytes;
-  float* recv = reinterpret_cast<float*>(stages);           // used after the main loop
+  uint64_t* a_full = reinterpret_cast<uint64_t*>(smem);     // [kTcMaxAStages] sign tile expanded
+  uint64_t* a_free = a_full + kTcMaxAStages;                // [kTcMaxAStages] its MMAs done
+  uint64_t* b_full = a_free + kTcMaxAStages;                // [kTcMaxBStages] activation tile landed
+  uint64_t* b_free = b_full + kTcMaxBStages;                // [kTcMaxBStages] its MMAs done
+  uint64_t* all_done = b_free + kTcMaxBStages;              // [1]
+  uint64_t* raw_full = all_done + 1;                        // [R] raw slot landed
+  uint64_t* raw_free = raw_full + kTcMaxRaw;                // [R] raw slot read by every producer
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_free + kTcMaxRaw);
+  TcSegInfo* si = reinterpret_cast<TcSegInfo*>(smem + kTcSegTable);  // [nseg_all]
+  unsigned char* raw_ring = smem + kTcHeader;               // [R][kTcRawBytes]
+  // [nB] activation tiles, 1024-byte aligned (128-byte swizzle atoms)
+  unsigned char* stages = raw_ring + (static_cast<size_t>(R) * kTcRawBytes + 1023) / 1024 * 1024;
+  float* recv = reinterpret_cast<float*>(raw_ring);         // used after the main loop (ring and stages)
 
   // (segment, K tile, part) steps; this CTA's range
   int nsteps = 0;
@@ -416,22 +430,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     e.ktiles = (e.g.ncols + kTcK - 1) / kTcK;
   }
   if (threadIdx.x == 0) {
-    // full: one arrival per producer thread once its part of the stage is written, plus
-    // one by the loader when it starts the stage's activation copy (with its byte count)
-    for (int s = 0; s < kTcMaxStages; ++s)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(full + s)), "r"(kTcProducers + 1) : "memory");
-    for (int s = 0; s <= kTcMaxStages; ++s)  // mma_done[] and all_done
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(mma_done + s)) : "memory");
+    // a_full: every producer thread (its lane's columns stored); b_full: the activation
+    // loader (with the tensor copy's byte count); a_free, b_free, all_done: MMA commits
+    for (int s = 0; s < kTcMaxAStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(a_full + s)), "r"(kTcProducers) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(a_free + s)) : "memory");
+    }
+    for (int s = 0; s < kTcMaxBStages; ++s) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(b_full + s)) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(b_free + s)) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(all_done)) : "memory");
     // raw_full: two arrivals per loader lane (its copies landed; its plain stores done);
     // raw_free: every producer thread
-    for (int s = 0; s < kTcRawSlots; ++s) {
+    for (int s = 0; s < R; ++s) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_full + s)), "r"(64) : "memory");
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_free + s)), "r"(kTcProducers) : "memory");
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)), "r"(tmem_cols)
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(saddr(tmem_slot)), "n"(kTcTmemCols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -444,26 +463,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto started = cluster.barrier_arrive();
 
   bool ok = true;
-  unsigned touched = 0;  // bit 2 b + part: accumulator columns written by this CTA (same in every thread)
+  unsigned touched = 0;  // bit b: accumulator block written by this CTA (same in every thread)
   const int n = st1 - st0;
   const int tiles_here = min(4, (p.rows + 31) / 32 - o0 / 32);  // 32-row tiles of this block in the packed layout
   // accumulator blocks this CTA writes (every thread walks the steps)
   TcCursor cur;
   cur.init(si, nseg_all, st0);
-  for (int i = 0; i < n; ++i, cur.next(si)) touched |= 1u << (2 * si[cur.seg].blk + cur.part);
+  for (int i = 0; i < n; ++i, cur.next(si)) touched |= 1u << si[cur.seg].blk;
   cur.init(si, nseg_all, st0);
 
   if (warp == kTcProducers / 32 + 1) {
     // ---------------- sign loader warp ----------------
     // Raw sign words (32 rows x 16 bytes of each of the four row tiles of the packed
     // layout; lane l copies row l of every tile, so a warp's copies are 512 contiguous
-    // bytes) and the step's 128 column scales go to raw slot i % 4 with cp.async (bulk
-    // copies issued back to back by one thread are served one after another), up to four
-    // steps ahead of the producers. Sign words never depend on the previous kernel, so the
-    // first slots are filled before the dependency wait.
+    // bytes) and the step's 128 column scales go to raw slot i % R with cp.async (bulk
+    // copies issued back to back by one thread are served one after another), up to R
+    // steps ahead of the producers. The ring takes the shared memory the activation tiles
+    // leave (tens of slots): with a few slots in flight per SM the sign stream ran at
+    // 0.6 TB/s (bytes in flight / latency). Sign words never depend on the previous
+    // kernel, so the first R slots are requested before the dependency wait.
     for (int i = 0; i < n; ++i) {
-      const int rs = i % kTcRawSlots;
-      if (i >= kTcRawSlots && !tc_wait(raw_free + rs, static_cast<unsigned>(i / kTcRawSlots - 1) & 1u)) ok = false;
+      const int rs = i % R;
+      if (i >= R && !tc_wait(raw_free + rs, static_cast<unsigned>(i / R - 1) & 1u)) ok = false;
       const TcSeg& g = si[cur.seg].g;
       unsigned char* dst = raw_ring + rs * kTcRawBytes;
       const bool bits = g.kind != kSegSal && g.bits != nullptr;
@@ -506,16 +527,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // the B tile themselves).
     asm volatile("griddepcontrol.wait;" ::: "memory");  // activations may come from the previous kernel
     for (int j = 0; j < n; ++j, cur.next(si)) {
-      const int sl = j % nstages;
-      if (j >= nstages && !tc_wait(mma_done + sl, static_cast<unsigned>(j / nstages - 1) & 1u)) ok = false;
-      unsigned char* B = stages + static_cast<size_t>(sl) * stage_bytes + a_bytes;
+      const int sb = j % nB;
+      if (j >= nB && !tc_wait(b_free + sb, static_cast<unsigned>(j / nB - 1) & 1u)) ok = false;
+      unsigned char* B = stages + static_cast<size_t>(sb) * b_bytes;
       if (use_tma && si[cur.seg].g.kind == kSegX) {
         // both 64-column blocks (rows past the batch read 0), one box from each of lanes 0, 1
-        if (lane == 0) bar_expect_tx(full + sl, b_bytes);
+        if (lane == 0) bar_expect_tx(b_full + sb, b_bytes);
         __syncwarp();
-        if (lane < 2) tma_load_2d(B + lane * Np * 128, &tmap_x, cur.kt * kTcK + lane * 64, 0, full + sl);
+        if (lane < 2) tma_load_2d(B + lane * Np * 128, &tmap_x, cur.kt * kTcK + lane * 64, 0, b_full + sb);
       } else if (lane == 0) {
-        bar_arrive(full + sl);
+        bar_arrive(b_full + sb);
       }
     }
   } else {
@@ -523,61 +544,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   if (warp < kTcProducers / 32) {
     // ---------------- producers ----------------
+    // Thread (row r, quarter q) expands columns 32q .. 32q+31 of row r of every step into
+    // 16 tensor-memory columns of lane r (the A operand of the step's MMAs).
+    const int r = threadIdx.x & (kTcRows - 1), q = threadIdx.x >> 7;
+    const uint32_t a_lane = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + static_cast<uint32_t>(a_base + 16 * q);
     for (int i = 0; i < n; ++i, cur.next(si)) {
-      const int sl = i % nstages, rs = i % kTcRawSlots;
-      // the stage is free once the MMAs that last read it are done
-      if (i >= nstages && !tc_wait(mma_done + sl, static_cast<unsigned>(i / nstages - 1) & 1u)) ok = false;
-      if (!tc_wait(raw_full + rs, static_cast<unsigned>(i / kTcRawSlots) & 1u)) ok = false;
+      const int sa = i % nA, sb = i % nB, rs = i % R;
+      // the sign stage is free once the MMAs that last read it are done
+      if (i >= nA && !tc_wait(a_free + sa, static_cast<unsigned>(i / nA - 1) & 1u)) ok = false;
+      if (!tc_wait(raw_full + rs, static_cast<unsigned>(i / R) & 1u)) ok = false;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int seg = cur.seg, kt = cur.kt, part = cur.part;
       const TcSeg& g = si[seg].g;
-      const int split = si[seg].parts;
-      unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
-      unsigned char* B = A + a_bytes;
       const int c0 = kt * kTcK;
+      uint32_t w[16];
       if (g.kind == kSegSal || g.bits == nullptr) {
-        for (int ch = threadIdx.x; ch < kTcRows * 16; ch += kTcProducers) {
-          const int r = ch & (kTcRows - 1), k8 = ch >> 7;
-          *reinterpret_cast<uint4*>(A + tile_off(r, k8, kTcRows)) = a_chunk(p, g, o0 + r, c0 + 8 * k8);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const uint4 v = a_chunk(p, g, o0 + r, c0 + 32 * q + 8 * jj);
+          w[4 * jj] = v.x; w[4 * jj + 1] = v.y; w[4 * jj + 2] = v.z; w[4 * jj + 3] = v.w;
         }
       } else {
-        a_expand(A, raw_ring + rs * kTcRawBytes, threadIdx.x & (kTcRows - 1), threadIdx.x >> 7, g.ncols - c0,
-                 g.cscale != nullptr);  // 512 producers: 128 rows x 4 column quarters
+        a_words(w, raw_ring + rs * kTcRawBytes, r, q, g.ncols - c0, g.cscale != nullptr);
       }
+      tmem_st16(a_lane + static_cast<uint32_t>(64 * sa), w);
       if (!(use_tma && g.kind == kSegX)) {
-        // fp32-valued inputs (z, salient, fp32 X) and unaligned bf16 X: several chunks in flight
+        // fp32-valued inputs (z, salient, fp32 X) and unaligned bf16 X: the producers write
+        // the B tile once its stage is free; several chunks in flight
+        if (i >= nB && !tc_wait(b_free + sb, static_cast<unsigned>(i / nB - 1) & 1u)) ok = false;
+        unsigned char* B = stages + static_cast<size_t>(sb) * b_bytes;
+        const int split = si[seg].parts;
 #pragma unroll 4
         for (int ch = threadIdx.x; ch < Np * 16; ch += kTcProducers) {
           const int m = ch >> 4, k8 = ch & 15;  // lanes along a row: coalesced reads
           *reinterpret_cast<uint4*>(B + tile_off(m, k8, Np)) = b_chunk(p, g, m, c0 + 8 * k8, part, split);
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic stores -> tensor core
       }
-      // make the generic-proxy stores visible to the tensor core, then mark the stage full
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      bar_arrive(full + sl);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      bar_arrive(a_full + sa);
       bar_arrive(raw_free + rs);
     }
   } else if (warp == kTcProducers / 32 && lane == 0) {
     // ---------------- MMA issue (one thread) ----------------
-    unsigned written = 0;  // bit 2 b + part: accumulator columns already written
+    unsigned written = 0;  // bit b: accumulator block already written
     const uint32_t idesc = mma_idesc(Np);
     for (int i = 0; i < n; ++i, cur.next(si)) {
-      const int sl = i % nstages;
-      if (!tc_wait(full + sl, static_cast<unsigned>(i / nstages) & 1u)) ok = false;
+      const int sa = i % nA, sb = i % nB;
+      if (!tc_wait(a_full + sa, static_cast<unsigned>(i / nA) & 1u)) ok = false;
+      if (!tc_wait(b_full + sb, static_cast<unsigned>(i / nB) & 1u)) ok = false;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const int blk = si[cur.seg].blk, part = cur.part;
-      unsigned char* A = stages + static_cast<size_t>(sl) * stage_bytes;
-      unsigned char* B = A + a_bytes;
-      const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk] + part * Np);
-      const unsigned bit = 1u << (2 * blk + part);
-      const bool first = !(written & bit);
+      const int blk = si[cur.seg].blk;
+      const uint64_t b0 = smem_desc_sw128(stages + static_cast<size_t>(sb) * b_bytes);
+      const uint32_t d = tmem + static_cast<uint32_t>(acc.col[blk]);
+      const uint32_t a = tmem + static_cast<uint32_t>(a_base + 64 * sa);
+      const uint32_t acc0 = ((written >> blk) & 1u) ? 1u : 0u;
+      // K = 16 per MMA: 8 columns of A; 32 bytes (descriptor +2) along a B row, the
+      // second 64-column block Np x 128 bytes further
 #pragma unroll
-      for (int kk = 0; kk < kTcK / 16; ++kk) {
-        const unsigned koff = (kk & 3) * 32u;  // K step inside a 64-column block
-        mma_bf16(d, smem_desc_sw128(A + (kk >> 2) * (kTcRows * 128) + koff),
-                 smem_desc_sw128(B + (kk >> 2) * (Np * 128) + koff), idesc, (first && kk == 0) ? 0u : 1u);
-      }
-      mma_commit(mma_done + sl);
-      written |= bit;
+      for (int kk = 0; kk < kTcK / 16; ++kk)
+        mma_ts_bf16(d, a + 8u * kk, b0 + static_cast<uint64_t>((kk >> 2) * (Np * 8) + (kk & 3) * 2), idesc, kk == 0 ? acc0 : 1u);
+      mma_commit(a_free + sa);
+      mma_commit(b_free + sb);
+      written |= 1u << blk;
     }
     mma_commit(all_done);
   }
@@ -621,29 +651,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int j = 0; j < 16; ++j) y[j] = 0.f;
       for (int b = 0; b < acc.nblk; ++b) {
-        // a CTA whose steps cover one part of a split block only reads that part
-        const bool t0 = (touched >> (2 * b)) & 1u, t1 = (touched >> (2 * b + 1)) & 1u;
-        if (!t0 && !t1) continue;
-        // the block's parts in flight before one wait
-        uint32_t v0[16], v1[16];
+        if (!((touched >> b) & 1u)) continue;
+        uint32_t v0[16];
         const uint32_t ta = lane_addr + static_cast<uint32_t>(acc.col[b] + m0);
-        if (t0)
-          asm volatile(
+        asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
               : "=r"(v0[0]), "=r"(v0[1]), "=r"(v0[2]), "=r"(v0[3]), "=r"(v0[4]), "=r"(v0[5]), "=r"(v0[6]), "=r"(v0[7]),
                 "=r"(v0[8]), "=r"(v0[9]), "=r"(v0[10]), "=r"(v0[11]), "=r"(v0[12]), "=r"(v0[13]), "=r"(v0[14]), "=r"(v0[15])
               : "r"(ta));
-        if (t1)
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-              : "=r"(v1[0]), "=r"(v1[1]), "=r"(v1[2]), "=r"(v1[3]), "=r"(v1[4]), "=r"(v1[5]), "=r"(v1[6]), "=r"(v1[7]),
-                "=r"(v1[8]), "=r"(v1[9]), "=r"(v1[10]), "=r"(v1[11]), "=r"(v1[12]), "=r"(v1[13]), "=r"(v1[14]), "=r"(v1[15])
-              : "r"(ta + static_cast<uint32_t>(Np)));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float t = (t0 ? __uint_as_float(v0[j]) : 0.f) + (t1 ? __uint_as_float(v1[j]) : 0.f);
-          y[j] = fmaf(t, rsv[b], y[j]);
+          y[j] = fmaf(__uint_as_float(v0[j]), rsv[b], y[j]);
         }
       }
       if (S > 1) {
@@ -705,7 +724,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kTcTmemCols) : "memory");
 }
 
 int tc_max_clusters(int S, size_t smem) {
@@ -784,21 +803,25 @@ TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncol
   TcPlan t{};
   t.Np = (Mc + 15) / 16 * 16;
   const TcAcc acc = tc_acc(nseg, seg_kind, n_sal > 0, x_bf16, t.Np);
-  if (acc.ncols > 512) return t;  // does not fit in tensor memory
-  t.tmem_cols = 32;
-  while (t.tmem_cols < acc.ncols) t.tmem_cols *= 2;
+  // tensor memory: the accumulators, then 64-column stages of expanded sign tiles
+  t.a_base = (acc.ncols + 63) / 64 * 64;
+  t.astages = std::min(kTcMaxAStages, (kTcTmemCols - t.a_base) / 64);
+  if (t.astages < 2) return t;
   int nsteps = 0;
   for (int s = 0; s < nseg; ++s) nsteps += (seg_ncols[s] + kTcK - 1) / kTcK * acc.split[acc.blk_of_seg[s]];
   if (n_sal > 0) nsteps += (n_sal + kTcK - 1) / kTcK * 2;
   if (nsteps == 0) return t;
-  const size_t stage = static_cast<size_t>(kTcRows) * kTcK * 2 + static_cast<size_t>(t.Np) * kTcK * 2;
-  const size_t fixed = kTcHeader + static_cast<size_t>(kTcRawSlots) * kTcRawBytes;
-  t.stages = static_cast<int>(std::min<size_t>(kTcMaxStages, (smem_limit - fixed) / stage));
-  if (t.stages < 2) return t;
+  const size_t stage = static_cast<size_t>(t.Np) * kTcK * 2;  // one activation tile
+  // activation tiles: up to six stages, leaving at least 16 sign-word slots; the rest of
+  // shared memory is sign-word ring
+  t.stages = static_cast<int>(std::min<size_t>(kTcMaxBStages, (smem_limit - kTcHeader - 16 * kTcRawBytes) / stage));
+  if (smem_limit < kTcHeader + t.stages * stage + 8 * static_cast<size_t>(kTcRawBytes)) return t;
+  t.raw_slots = static_cast<int>(std::min<size_t>(kTcMaxRaw, (smem_limit - kTcHeader - t.stages * stage - 1023) / kTcRawBytes));
+  const size_t fixed = kTcHeader;
+  const size_t body = (static_cast<size_t>(t.raw_slots) * kTcRawBytes + 1023) / 1024 * 1024 + t.stages * stage;
   // more than half of the SM's shared memory: one CTA per SM (tensor memory is not shared)
-  t.smem = std::max(fixed + t.stages * stage, smem_limit / 2 + 4096);
-  t.smem = std::min(t.smem, smem_limit);
-  if (fixed + t.stages * stage > t.smem) return t;
+  t.smem = std::min(std::max(fixed + body, smem_limit / 2 + 4096), smem_limit);
+  if (fixed + body > t.smem) return t;
   tc_ensure_attrs();
   t.tiles = (rows + kTcRows - 1) / kTcRows;
   // split K over a cluster so that the grid covers the SMs
@@ -807,7 +830,7 @@ TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncol
   for (; S >= 1; S /= 2) {
     const size_t rows_per = (kTcRows + S - 1) / S;
     const size_t recv = (static_cast<size_t>(S) * rows_per * (t.Np + 4) + static_cast<size_t>(t.Np) * (rows_per + 1)) * 4;
-    if (recv > static_cast<size_t>(t.stages) * stage) continue;
+    if (recv > body) continue;
     if (tc_max_clusters(S, t.smem) >= 1) break;
   }
   if (S < 1) return t;
@@ -835,7 +858,7 @@ cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream) 
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
   const int use_tma = x_tensor_map(p, t.Np, &map) ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, map, use_tma, t.S, t.Np, t.stages, t.tmem_cols);
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, map, use_tma, t.S, t.Np, t.astages, t.stages, t.raw_slots, t.a_base);
 }
 
 }  // namespace bisco
