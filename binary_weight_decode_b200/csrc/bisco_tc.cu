@@ -2,9 +2,9 @@
 //
 // With many batch rows the product is a dense contraction: for each segment,
 //   D_seg[o][m] = sum_i A_seg[o][i] * B_seg[i][m].
-// The signs are expanded in shared memory into bf16 tiles and multiplied on the
-// 5th-generation tensor cores (tcgen05.mma, kind::f16, fp32 accumulators in tensor
-// memory):
+// The signs are expanded into bf16 tiles in tensor memory and multiplied on the
+// 5th-generation tensor cores (tcgen05.mma, kind::f16, A from tensor memory, B from
+// shared memory, fp32 accumulators in tensor memory):
 //   * a binary base k: A = +-c_k[i] (the column scale folded into the sign; exact in
 //     bf16 because the scales are bf16), B = X (exact for bf16 activations; fp32
 //     activations are split into bf16 high and low parts). Each base has its own
@@ -22,24 +22,24 @@
 //
 // Work decomposition: cluster c owns 128 output rows; CTA r of the cluster takes 1/S of
 // the (segment, 128-column K tile, part) steps, where a split segment (high and low bf16
-// parts) has two steps per K tile, one per part, into two column blocks of its
-// accumulator. A step's tiles live in a shared-memory stage, K-major with the 128-byte
-// swizzle: each tile is two blocks of 64 columns; a row of a block is 128 bytes, its
-// 16-byte chunks permuted by XOR with (row mod 8), and groups of 8 rows are 1024 bytes
-// apart. cp.async brings in the raw sign words and column scales two steps ahead (a
-// four-slot ring). A bf16 activation tile comes in through the tensor memory accelerator
-// (two 64-column boxes per step, written in the 128-byte swizzle by the copy engine and
-// counted in bytes on the stage's "full" mbarrier); fp32-valued B tiles are written by
-// the producers. The warps are specialised: 16 producer warps wait until a stage is
-// free, start its activation copy, expand the step's signs from the raw ring and mark
-// the stage full; one more warp waits for each full stage, issues the step's eight K=16
-// MMAs and commits them to the stage's "free" mbarrier, so expansion of later stages
-// overlaps the MMAs of earlier ones. Every waiter walks every stage in order, so one
-// pair of barriers per stage slot suffices.
+// parts) has two steps per K tile, one per part, both accumulated into the segment's
+// block. Four warp roles hand steps over on mbarriers (every waiter walks every step in
+// order, so one pair of barriers per ring slot suffices):
+//   * sign loader (1 warp): one 4-D tensor copy brings a step's 2 KB of packed sign words
+//     (four 32-row tiles) and a 1-D tensor copy its 128 column scales into a ring of
+//     shared-memory slots, tens of steps ahead (the first ones before the dependency
+//     wait: weights never depend on the previous kernel);
+//   * activation loader (1 warp): two tensor copies per step bring the bf16 activation
+//     tile (64-column boxes, written in the 128-byte swizzle the MMA descriptors expect)
+//     into a shared-memory stage once the MMAs that last read it are done;
+//   * producers (16 warps): thread (row r, quarter q) expands 32 columns of row r into 16
+//     tensor-memory columns of lane r (tcgen05.st), the A operand of the step; fp32-valued
+//     or unaligned B tiles are written by the producers too;
+//   * MMA issue (one thread): eight K=16 MMAs per step, committed to the "free" barriers
+//     of the step's A and B stages.
 // The S partial results meet in distributed shared memory and are added in CTA-rank
-// order.
-// A CTA takes more than half of an SM's shared memory, so no two CTAs (each holding up
-// to 512 tensor-memory columns) ever share an SM.
+// order. A CTA takes all 512 tensor-memory columns and more than half of an SM's shared
+// memory, so it is alone on its SM.
 
 #include <cooperative_groups.h>
 #include <cuda.h>  // CUtensorMap and the tensor-map encoder's argument types (no driver library is linked)
@@ -99,10 +99,21 @@ __device__ __forceinline__ void bar_arrive(uint64_t* b) {
 __device__ __forceinline__ void bar_expect_tx(uint64_t* b, unsigned bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes) : "memory");
 }
-// Arrives on b once all cp.async operations issued so far by this thread have completed
-// (the arrival is one of the phase's expected arrivals).
-__device__ __forceinline__ void bar_arrive_cp(uint64_t* b) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(saddr(b)) : "memory");
+// One box of a 1-D tensor map into this CTA's shared memory (completion counted in bytes
+// on bar); out-of-range elements read 0.
+__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* map, int x, uint64_t* bar) {
+  asm volatile("cp.async.bulk.tensor.1d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2}], [%3];" ::"r"(
+                   saddr(dst)),
+               "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(saddr(bar))
+               : "memory");
+}
+// One box of a 4-D tensor map, coordinates innermost first.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int x, int y, int z, int w, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+          saddr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(saddr(bar))
+      : "memory");
 }
 // One box of a 2-D tensor map into this CTA's shared memory; completion counted in
 // bytes on bar. Coordinates are (column, row) in elements; out-of-range elements read 0.
@@ -163,11 +174,6 @@ __device__ __forceinline__ unsigned tile_off(int row, int k8, int rows) {
   return (k8 >> 3) * static_cast<unsigned>(rows) * 128u + row * 128u + (((k8 & 7) ^ (row & 7)) << 4);
 }
 
-// 16-byte cp.async with zero fill past src_bytes (0..16).
-__device__ __forceinline__ void cp16(void* dst, const void* src, unsigned src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src), "r"(src_bytes) : "memory");
-}
-
 __device__ __forceinline__ unsigned pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const unsigned*>(&h);
@@ -186,6 +192,15 @@ struct TcSeg {
   const uint4* bits;
   const void* cscale;
   int nq, ncols, kind, cvec;
+};
+
+// Tensor maps of a launch's packed sign words and column scales, one per segment:
+// bits[s] views segment s's packed layout [tiles][quads][32 rows][4 words] as a 4-D
+// uint32 tensor (box: 4 words x 32 rows x 1 quad x 4 tiles = the 2 KB of one step);
+// cs[s] views its bf16 column scales as a 1-D tensor (box: 128 scales).
+struct TcMaps {
+  CUtensorMap bits[kMaxSeg];
+  CUtensorMap cs[kMaxSeg];
 };
 
 __device__ __forceinline__ TcSeg tc_seg(const PassParam& p, int s) {
@@ -389,7 +404,8 @@ __host__ __device__ __forceinline__ TcAcc tc_acc(int nseg, const int* seg_kind, 
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ PassParam p, const __grid_constant__ CUtensorMap tmap_x, const int use_tma, const int S,
+    tc_gemm_kernel(const __grid_constant__ PassParam p, const __grid_constant__ CUtensorMap tmap_x,
+                   const __grid_constant__ TcMaps maps, const int use_tma, const int cs_tma, const int S,
                    const int Np, const int nA, const int nB, const int R, const int a_base) {
   extern __shared__ __align__(1024) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -441,10 +457,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(b_free + s)) : "memory");
     }
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(saddr(all_done)) : "memory");
-    // raw_full: two arrivals per loader lane (its copies landed; its plain stores done);
-    // raw_free: every producer thread
+    // raw_full: the sign loader's lane 0 (with the tensor copies' byte count) and each of
+    // its 32 lanes once its plain stores are done; raw_free: every producer thread
     for (int s = 0; s < R; ++s) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_full + s)), "r"(64) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_full + s)), "r"(33) : "memory");
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(raw_free + s)), "r"(kTcProducers) : "memory");
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -465,7 +481,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   bool ok = true;
   unsigned touched = 0;  // bit b: accumulator block written by this CTA (same in every thread)
   const int n = st1 - st0;
-  const int tiles_here = min(4, (p.rows + 31) / 32 - o0 / 32);  // 32-row tiles of this block in the packed layout
   // accumulator blocks this CTA writes (every thread walks the steps)
   TcCursor cur;
   cur.init(si, nseg_all, st0);
@@ -474,49 +489,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   if (warp == kTcProducers / 32 + 1) {
     // ---------------- sign loader warp ----------------
-    // Raw sign words (32 rows x 16 bytes of each of the four row tiles of the packed
-    // layout; lane l copies row l of every tile, so a warp's copies are 512 contiguous
-    // bytes) and the step's 128 column scales go to raw slot i % R with cp.async (bulk
-    // copies issued back to back by one thread are served one after another), up to R
-    // steps ahead of the producers. The ring takes the shared memory the activation tiles
-    // leave (tens of slots): with a few slots in flight per SM the sign stream ran at
-    // 0.6 TB/s (bytes in flight / latency). Sign words never depend on the previous
-    // kernel, so the first R slots are requested before the dependency wait.
+    // The step's raw sign words (the four 32-row tiles of its 128 rows, 512 bytes each in
+    // the packed layout) arrive through one 4-D tensor copy and its 128 column scales
+    // through one 1-D tensor copy (16-byte aligned scales; otherwise lanes 0..15 load them)
+    // into raw slot i % R, up to R steps ahead of the producers. Rows past the layout and
+    // columns past the segment read 0. The ring takes the shared memory the activation
+    // tiles leave (tens of slots). Sign words never depend on the previous kernel, so the
+    // first R slots are requested before the dependency wait.
     for (int i = 0; i < n; ++i) {
       const int rs = i % R;
       if (i >= R && !tc_wait(raw_free + rs, static_cast<unsigned>(i / R - 1) & 1u)) ok = false;
       const TcSeg& g = si[cur.seg].g;
       unsigned char* dst = raw_ring + rs * kTcRawBytes;
       const bool bits = g.kind != kSegSal && g.bits != nullptr;
-      if (bits) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {  // row 32 t + lane; rows past the layout's tiles read 0
-          const bool in = t < tiles_here;
-          const uint4* src = g.bits + (static_cast<long long>(in ? o0 / 32 + t : 0) * g.nq + cur.kt) * 32 + lane;
-          cp16(dst + (t * 32 + lane) * 16, src, in ? 16u : 0u);
+      const bool cs_copy = bits && g.cscale != nullptr && ((cs_tma >> cur.seg) & 1);
+      if (lane == 0) {
+        const unsigned bytes = (bits ? kTcRows * 16u : 0u) + (cs_copy ? kTcK * 2u : 0u);
+        if (bytes > 0) {
+          bar_expect_tx(raw_full + rs, bytes);
+          if (bits) tma_load_4d(dst, &maps.bits[cur.seg], 0, 0, cur.kt, o0 / 32, raw_full + rs);
+          if (cs_copy) tma_load_1d(dst + kTcRows * 16, &maps.cs[cur.seg], cur.kt * kTcK, raw_full + rs);
+        } else {
+          bar_arrive(raw_full + rs);
         }
       }
-      if (lane < kTcK / 8) {
-        // column scales (bf16) for columns 8 lane .. + 7 of the K tile, zero past the segment
-        if (bits && g.cscale != nullptr) {
-          const int cc = cur.kt * kTcK + lane * 8;
-          const int valid = max(0, min(8, g.ncols - cc));
-          unsigned char* cd = dst + kTcRows * 16 + lane * 16;
-          const unsigned short* cs = reinterpret_cast<const unsigned short*>(g.cscale);
-          if (g.cvec) {  // 16-byte aligned scales: asynchronous copy with zero fill
-            cp16(cd, cs + (valid > 0 ? cc : 0), static_cast<unsigned>(valid * 2));
-          } else {       // unaligned (e.g. the second base of a layer with in % 8 != 0): plain loads
-            unsigned short v[8];
+      if (bits && g.cscale != nullptr && !cs_copy && lane < kTcK / 8) {
+        // unaligned scales (e.g. the second base of a layer with in % 8 != 0): plain loads
+        // of columns 8 lane .. + 7 of the K tile, zero past the segment
+        const int cc = cur.kt * kTcK + lane * 8;
+        const int valid = max(0, min(8, g.ncols - cc));
+        const unsigned short* cs = reinterpret_cast<const unsigned short*>(g.cscale);
+        unsigned short v[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = e < valid ? __ldg(cs + cc + e) : 0;
-            *reinterpret_cast<uint4*>(cd) =
-                make_uint4(v[0] | (static_cast<unsigned>(v[1]) << 16), v[2] | (static_cast<unsigned>(v[3]) << 16),
-                           v[4] | (static_cast<unsigned>(v[5]) << 16), v[6] | (static_cast<unsigned>(v[7]) << 16));
-          }
-        }
+        for (int e = 0; e < 8; ++e) v[e] = e < valid ? __ldg(cs + cc + e) : 0;
+        *reinterpret_cast<uint4*>(dst + kTcRows * 16 + lane * 16) =
+            make_uint4(v[0] | (static_cast<unsigned>(v[1]) << 16), v[2] | (static_cast<unsigned>(v[3]) << 16),
+                       v[4] | (static_cast<unsigned>(v[5]) << 16), v[6] | (static_cast<unsigned>(v[7]) << 16));
       }
-      bar_arrive_cp(raw_full + rs);  // once this lane's copies have landed
-      bar_arrive(raw_full + rs);     // this lane's plain stores (release)
+      bar_arrive(raw_full + rs);  // this lane's plain stores (release)
       cur.next(si);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -783,6 +793,39 @@ bool x_tensor_map(const PassParam& p, int Np, CUtensorMap* map) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor maps of the packed sign words (and, where 16-byte aligned, the bf16 column
+// scales) of every segment with signs. Bit s of *cs_mask: segment s's scales come through
+// cs[s]. False if a map cannot be encoded.
+bool sign_maps(const PassParam& p, TcMaps* m, int* cs_mask) {
+  *cs_mask = 0;
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return false;
+  const cuuint64_t tiles = static_cast<cuuint64_t>((p.rows + 31) / 32);
+  for (int s = 0; s < p.nseg; ++s) {
+    const SegParam& G = p.seg[s];
+    if (G.bits == nullptr) continue;
+    const cuuint64_t nq = static_cast<cuuint64_t>(G.nq);
+    const cuuint64_t dims[4] = {4, 32, nq, tiles};
+    const cuuint64_t strides[3] = {16, 512, nq * 512};
+    const cuuint32_t box[4] = {4, 32, 1, 4};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    if (enc(&m->bits[s], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<uint4*>(G.bits), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return false;
+    if (G.cscale != nullptr && G.cvec && G.cdt == BISCO_BF16) {
+      const cuuint64_t cdims[1] = {static_cast<cuuint64_t>(G.ncols)};
+      const cuuint32_t cbox[1] = {static_cast<cuuint32_t>(kTcK)};
+      const cuuint32_t ces[1] = {1};
+      if (enc(&m->cs[s], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 1, const_cast<void*>(G.cscale), cdims, nullptr, cbox, ces,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+        *cs_mask |= 1 << s;
+    }
+  }
+  return true;
+}
+
 }  // namespace
 
 cudaError_t tc_ensure_attrs() {
@@ -858,7 +901,12 @@ cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream) 
   CUtensorMap map;
   std::memset(&map, 0, sizeof(map));
   const int use_tma = x_tensor_map(p, t.Np, &map) ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, map, use_tma, t.S, t.Np, t.astages, t.stages, t.raw_slots, t.a_base);
+  TcMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  int cs_mask = 0;
+  if (!sign_maps(p, &maps, &cs_mask)) return cudaErrorNotSupported;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel, p, map, maps, use_tma, cs_mask, t.S, t.Np, t.astages, t.stages, t.raw_slots,
+                            t.a_base);
 }
 
 }  // namespace bisco
