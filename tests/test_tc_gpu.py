@@ -30,7 +30,9 @@ CASES = [
     (300, 700, 2, 24, 0.02, 33, "bf16", "f32"),     # correction + salient
     (640, 1000, 1, 96, 0.01, 64, "bf16", "bf16"),
     (512, 1024, 2, 0, 0.0, 128, "bf16", "f32"),
-    (384, 640, 3, 40, 0.0, 130, "bf16", "f32"),     # 128 on the tensor cores + 2 on the LUT path
+    # three bases + correction at 128 rows: four accumulator blocks of 128 columns leave too
+    # little tensor memory for the sign stages, so the call runs on lookup-table chunks
+    (384, 640, 3, 40, 0.0, 130, "bf16", "f32"),
     (160, 384, 2, 8, 0.03, 150, "bf16", "f32"),     # 128 + 22 (lookup-table chunks of 8, 8, 6)
     (257, 129, 4, 0, 0.0, 40, "bf16", "f32"),       # four bases
     (192, 512, 2, 17, 0.0, 48, "f32", "f32"),       # fp32 activations: split on the bases
