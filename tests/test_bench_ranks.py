@@ -70,3 +70,28 @@ def test_max_without_process_group_is_identity():
 ])
 def test_launch_schedule(M, rank, bf16, expected):
     assert _bench().launches_per_gemv(M, rank, bf16) == expected
+
+
+def test_reference_arm_prints_one_contract_line():
+    # bench.py --impl reference times the oracle on the host cores (no GPU needed) and
+    # prints one JSON line with the base contract's keys, the same metric and config as
+    # the CUDA arm, and an e2e entry that moves no bytes across PCIe.
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference"
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["metric"] == "M=1 binary-GEMV effective HBM GB/s" and d["unit"] == "GB/s"
+    assert d["config"]["workload"].startswith("attn4096") and d["config"]["M"] == 1
+    assert d["steps"] == 1 and d["warmup"] == 1 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
