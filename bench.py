@@ -110,7 +110,10 @@ def max_over_ranks(value, dist, device):
 def launches_per_gemv(M, rank, scale_bf16, tc_min=32, tc_max=128, lut_max=8):
     """Kernel launches of one bisco_gemv call: the library's batch-chunk schedule
     (tensor-core chunks of up to 128 rows from 32 rows up when the scales are bf16,
-    lookup-table chunks of up to 8 rows otherwise), one launch per pass per chunk."""
+    lookup-table chunks of up to 8 rows otherwise), one launch per pass per chunk.
+    The tensor-core plan also needs its accumulators to leave room in tensor memory
+    (at most three blocks at 128 rows); every bench workload has at most two bases
+    plus one correction/salient block, so the schedule above is the one that runs."""
     chunks, rem = 0, M
     while rem > 0:
         take = min(rem, tc_max) if (scale_bf16 and rem >= tc_min) else min(rem, lut_max)
