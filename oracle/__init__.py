@@ -11,6 +11,7 @@ from .bisco_oracle import (  # noqa: F401
     correction_z,
     decode_values,
     dense_correction_storage_bits,
+    fluxbin_average_bit_width,
     fp4_weight_bits,
     gemv,
     gemv_rows,

@@ -204,6 +204,21 @@ def fp4_weight_bits(out, in_, bits_per_weight=4.0):
     return out * in_ * bits_per_weight
 
 
+def fluxbin_average_bit_width(rows, cols, Kb, Ks, g, s, scale_bits=16):
+    """Effective average bit-width of a FluxBin-style layer with grouped row scales and a
+    binary salient refinement ("FluxBin", Sec. C.2 Storage Consumption Analysis): Kb global
+    sign bits per weight; Ks refinement sign bits on the s salient columns of every group
+    of g columns; one row scale per (row, group) for each of the Kb + Ks bases; one column
+    scale per column of each base (the salient bases cover rows x cols*s/g); one index per
+    salient column; every scale and index in `scale_bits` bits. Bits over rows*cols."""
+    n_sal = cols * s / g
+    bits = Kb * rows * cols + Ks * rows * n_sal                 # signs
+    bits += (Kb + Ks) * rows * (cols / g) * scale_bits          # grouped row scales
+    bits += (Kb * cols + Ks * n_sal) * scale_bits               # column scales
+    bits += n_sal * scale_bits                                  # salient column indices
+    return bits / (rows * cols)
+
+
 def _dtype_bytes(dtype):
     return {"f32": 4, "bf16": 2}[dtype]
 

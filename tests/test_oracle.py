@@ -321,6 +321,22 @@ def test_storage_arithmetic_matches_the_page():
     assert fp4_mib / mib128 == g["read_ratio_approx"]
 
 
+@pytest.mark.parametrize("rows,cols", [(4096, 4096), (11008, 4096), (4096, 11008)])
+def test_fluxbin_average_bit_width_matches_the_page(rows, cols):
+    # grouped row scales and binary salient refinement: the page prints the resulting
+    # bit-widths (rounded) for three group/salient settings of its two-base configuration
+    g = golden("fluxbin_abw.json")
+    for c in g["cases"]:
+        abw = oracle.fluxbin_average_bit_width(rows, cols, g["Kb"], g["Ks"], c["g"], c["s"])
+        assert abw == pytest.approx(c["abw_approx"], abs=0.015), c
+        if "salient_ratio" in c:
+            assert c["s"] / c["g"] == c["salient_ratio"]
+    # the grouped row scales and the refinement are visible at the page's precision: without
+    # the refinement's row scales the typical configuration would read 2.38 bits, without
+    # any row scale 2.13, without the refinement bases (Ks = 0) 2.26
+    assert oracle.fluxbin_average_bit_width(rows, cols, 2, 0, 128, 8) == pytest.approx(2.26, abs=0.01)
+
+
 def test_algorithmic_bytes_counts_each_payload():
     L = Layer(out=4096, in_=4096, K=2, scale_dtype="bf16", bits=None, row_scale=None, col_scale=None)
     # signs 2*4096*4096/8, scales 2*(4096+4096)*2 B, x 4096*2 B, y 4096*2 B
