@@ -161,6 +161,10 @@ class DeviceLayer:
                 return torch.from_numpy(a.view(np.int32)).to(device)
             return torch.from_numpy(a).to(device)
 
+        if getattr(host, "group", 0):
+            # bisco_layer carries one row scale per (base, row); grouped row scales are not
+            # part of the C ABI yet
+            raise NotImplementedError("grouped row scales are not supported by libbisco")
         self.host = host
         self.out, self.in_, self.K = host.out, host.in_, host.K
         self.rank, self.n_sal = host.rank, host.n_sal

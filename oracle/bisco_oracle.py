@@ -119,16 +119,23 @@ def decode_values(a, dtype):
 # ----------------------------------------------------------------------------
 
 def _binary_part_rows(layer, rows):
-    """sum_k diag(r_k) B_k diag(c_k), restricted to output rows `rows`."""
+    """sum_k diag(r_k) B_k diag(c_k), restricted to output rows `rows`.
+
+    With grouped row scales (layer.group = g > 0; "FluxBin", Sec. 3.1: one row scale per
+    weight group, and Sec. 4: g is the group size of the row-wise scale) the row scale of
+    entry (o, i) is r_k[o][i // g]."""
     W = np.zeros((len(rows), layer.in_), dtype=np.float64)
     if layer.K == 0:
         return W
-    R = decode_values(layer.row_scale, layer.scale_dtype).reshape(layer.K, layer.out)
+    g = getattr(layer, "group", 0)
+    ng = -(-layer.in_ // g) if g else 1
+    R = decode_values(layer.row_scale, layer.scale_dtype).reshape(layer.K, layer.out, ng)
     C = decode_values(layer.col_scale, layer.scale_dtype).reshape(layer.K, layer.in_)
+    col_group = np.arange(layer.in_) // g if g else np.zeros(layer.in_, dtype=np.int64)
     bits = np.asarray(layer.bits).reshape(layer.K, -1)
     for k in range(layer.K):
         S = unpack_bit_rows(bits[k], layer.out, layer.in_, rows)
-        W += R[k, rows][:, None] * S * C[k][None, :]
+        W += R[k][rows][:, col_group] * S * C[k][None, :]
     return W
 
 

@@ -73,7 +73,7 @@ class Layer:
     K: int
     scale_dtype: str                  # "f32" or "bf16"
     bits: np.ndarray                  # uint32 [K, packed_words(out, in)]
-    row_scale: np.ndarray             # [K, out] float32 or uint16 (bf16 bits)
+    row_scale: np.ndarray             # [K, out] (or [K, out, ceil(in/group)]) float32 or uint16 (bf16 bits)
     col_scale: np.ndarray             # [K, in]
     rank: int = 0
     v_bits: Optional[np.ndarray] = None    # uint32 [packed_words(rank, in)]
@@ -85,6 +85,9 @@ class Layer:
     sal_scale: Optional[np.ndarray] = None  # float32 [n_sal]
     name: str = ""
     extra: dict = field(default_factory=dict)
+    # 0: one row scale per (base, row); g > 0: one per (base, row, group of g input
+    # columns), row_scale [K, out, ceil(in/g)] (grouped row scales: oracle only so far)
+    group: int = 0
 
     @property
     def sal_stride(self) -> int:
@@ -108,12 +111,13 @@ def make_activations(seed: int, key: Sequence[int], M: int, n: int, dtype: str,
 
 def make_layer(seed: int, key: Sequence[int], out: int, in_: int, K: int, scale_dtype: str,
                rank: int = 0, sal_frac: float = 0.0, x_for_salience: Optional[np.ndarray] = None,
-               x_dtype: str = "bf16", name: str = "") -> Layer:
+               x_dtype: str = "bf16", name: str = "", group: int = 0) -> Layer:
     bits = random_sign_words(_rng(seed, key, T_BITS), K, out, in_)
-    row = _as_dtype(np.abs(_rng(seed, key, T_ROW).standard_normal((K, out))) * 0.02, scale_dtype)
+    rshape = (K, out, -(-in_ // group)) if group else (K, out)
+    row = _as_dtype(np.abs(_rng(seed, key, T_ROW).standard_normal(rshape)) * 0.02, scale_dtype)
     col = _as_dtype(np.abs(_rng(seed, key, T_COL).standard_normal((K, in_))) * 0.02, scale_dtype)
     L = Layer(out=out, in_=in_, K=K, scale_dtype=scale_dtype, bits=bits, row_scale=row,
-              col_scale=col, name=name)
+              col_scale=col, name=name, group=group)
     if rank > 0:
         L.rank = rank
         L.v_bits = random_sign_words(_rng(seed, key, T_V), 1, rank, in_)[0]

@@ -78,3 +78,11 @@ def test_gemv_rejects_bad_arguments_before_touching_the_device():
     assert bw._lib.bisco_gemv(L, None, 0, -1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG  # M < 0
     assert bw._lib.bisco_gemv(L, None, 0, 0, None, 0, None, 0, None) == bw.BISCO_OK                # M == 0
     assert bw.bisco_status_string(bw.BISCO_ERR_WORKSPACE) == "BISCO_ERR_WORKSPACE"
+
+
+def test_grouped_row_scales_are_refused_by_the_binding():
+    # the C ABI carries one row scale per (base, row): a grouped layer must not be uploaded
+    from synth import make_layer
+    L = make_layer(0, (8,), 64, 256, 2, "bf16", group=128)
+    with pytest.raises(NotImplementedError):
+        bw.DeviceLayer(L)

@@ -57,12 +57,13 @@ def f32(a):
 
 
 def mk(out, in_, K=0, signs=None, row=None, col=None, rank=0, u=None, v=None, alpha=None,
-       sal_idx=None, sal_q=None, sal_scale=None):
-    """Layer with fp32 scales built through the independent packer."""
+       sal_idx=None, sal_q=None, sal_scale=None, group=0):
+    """Layer with fp32 scales built through the independent packer (row: [K, out], or
+    [K, out, groups] with grouped row scales)."""
     bits = np.stack([py_pack(signs[k]) for k in range(K)]) if K else np.zeros((0, 0), np.uint32)
     L = Layer(out=out, in_=in_, K=K, scale_dtype="f32", bits=bits,
               row_scale=f32(row if K else np.zeros((0, out))),
-              col_scale=f32(col if K else np.zeros((0, in_))))
+              col_scale=f32(col if K else np.zeros((0, in_))), group=group)
     if rank:
         L.rank = rank
         L.v_bits = py_pack(v)                               # [rank][in]
@@ -239,6 +240,63 @@ def test_terms_add():
                n_sal=3, sal_idx=L.sal_idx, sal_q=L.sal_q, sal_scale=L.sal_scale)
     parts = oracle.gemv(Lb, X, "f32") + oracle.gemv(Lc, X, "f32") + oracle.gemv(Ls, X, "f32")
     assert np.allclose(full, parts, rtol=1e-12, atol=1e-18)
+
+
+# --- grouped row scales (one row scale per group of g input columns) ------------
+
+def test_grouped_all_plus_one_is_a_sum_of_group_sums():
+    # all signs +1: y[m][o] = sum_k sum_G r_k[o][G] * sum_{i in group G} c_k[i] x[m][i]
+    rng = np.random.default_rng(11)
+    out, in_, K, g = 9, 300, 2, 128          # groups of 128, 128 and a ragged 44
+    ng = -(-in_ // g)
+    row = np.abs(rng.standard_normal((K, out, ng))) * 0.02 + 0.001
+    col = np.abs(rng.standard_normal((K, in_))) * 0.02
+    L = mk(out, in_, K=K, signs=[[[1] * in_] * out] * K, row=row, col=col, group=g)
+    X = f32(rng.standard_normal((2, in_)))
+    y = oracle.gemv(L, X, "f32")
+    r64, c64, x64 = f32(row).astype(float), f32(col).astype(float), X.astype(float)
+    expect = np.zeros((2, out))
+    for k in range(K):
+        for G in range(ng):
+            cols = slice(G * g, min(in_, (G + 1) * g))
+            expect += np.outer(x64[:, cols] @ c64[k, cols], r64[k, :, G])
+    assert np.allclose(y, expect, rtol=1e-12, atol=1e-15)
+
+
+def test_grouped_scales_equal_across_groups_match_one_scale_per_row():
+    rng = np.random.default_rng(12)
+    out, in_, K, g = 7, 200, 2, 64
+    signs = rng.choice([-1, 1], size=(K, out, in_)).tolist()
+    row = np.abs(rng.standard_normal((K, out))) + 0.1
+    col = np.abs(rng.standard_normal((K, in_))) + 0.1
+    X = f32(rng.standard_normal((3, in_)))
+    flat = oracle.gemv(mk(out, in_, K, signs, row, col), X, "f32")
+    grouped = oracle.gemv(mk(out, in_, K, signs, np.repeat(row[:, :, None], 4, axis=2), col, group=g), X, "f32")
+    assert np.allclose(grouped, flat, rtol=1e-13, atol=1e-16)
+
+
+@pytest.mark.parametrize("out,in_,K,g", [(1, 4, 1, 2), (2, 4, 1, 2), (1, 4, 2, 2), (2, 3, 1, 2), (1, 5, 1, 3)])
+def test_grouped_brute_force_all_sign_patterns(out, in_, K, g):
+    """Every sign pattern with a different row scale per group: the product equals the
+    sign-add identity applied group by group, bits read with plain integer shifts."""
+    rng = np.random.default_rng(out * 1000 + in_ * 100 + K * 10 + g)
+    ng = -(-in_ // g)
+    row = f32(rng.uniform(0.5, 2.0, size=(K, out, ng)))
+    col = f32(rng.uniform(0.5, 2.0, size=(K, in_)))
+    x = f32(rng.standard_normal((1, in_)))
+    for pattern in itertools.product([-1, 1], repeat=K * out * in_):
+        S = np.array(pattern).reshape(K, out, in_)
+        L = mk(out, in_, K, S.tolist(), row, col, group=g)
+        y = oracle.gemv(L, x, "f32")[0]
+        for o in range(out):
+            expect = 0.0
+            for k in range(K):
+                for G in range(ng):
+                    cols = range(G * g, min(in_, (G + 1) * g))
+                    a = {i: float(col[k, i]) * float(x[0, i]) for i in cols}
+                    set_sum = sum(a[i] for i in cols if py_bit(L.bits[k], out, in_, o, i))
+                    expect += float(row[k, o, G]) * (2.0 * set_sum - sum(a.values()))
+            assert y[o] == pytest.approx(expect, rel=1e-12, abs=1e-15)
 
 
 # --- brute force on tiny shapes -----------------------------------------------

@@ -23,6 +23,8 @@ PINS = [
     lambda: P.test_single_bit_positions(33, 129),
     lambda: P.test_oracle_pack_matches_independent_packer(45, 200),
     P.test_bf16_decode_by_definition,
+    P.test_grouped_all_plus_one_is_a_sum_of_group_sums,
+    lambda: P.test_grouped_brute_force_all_sign_patterns(2, 4, 1, 2),
 ]
 
 
@@ -81,6 +83,32 @@ def _binary_col_scale_of_base0(layer, rows):
     return W
 
 
+def _binary_grouped(layer, rows, group_of):
+    """Binary part with the row-scale group of column i given by group_of(i, g)."""
+    if layer.K == 0:
+        return np.zeros((len(rows), layer.in_))
+    g = getattr(layer, "group", 0)
+    ng = -(-layer.in_ // g) if g else 1
+    R = O.decode_values(layer.row_scale, layer.scale_dtype).reshape(layer.K, layer.out, ng)
+    C = O.decode_values(layer.col_scale, layer.scale_dtype).reshape(layer.K, layer.in_)
+    cols = np.arange(layer.in_)
+    grp = np.minimum(group_of(cols, g), ng - 1) if g else np.zeros(layer.in_, dtype=np.int64)
+    bits = np.asarray(layer.bits).reshape(layer.K, -1)
+    W = np.zeros((len(rows), layer.in_))
+    for k in range(layer.K):
+        S = O.unpack_bit_matrix(bits[k], layer.out, layer.in_)[rows]
+        W += R[k][rows][:, grp] * S * C[k][None, :]
+    return W
+
+
+def _binary_group_modulo(layer, rows):
+    return _binary_grouped(layer, rows, lambda i, g: i % g)
+
+
+def _binary_group_ignored(layer, rows):
+    return _binary_grouped(layer, rows, lambda i, g: np.zeros_like(i))
+
+
 def _correction_alpha_dropped(layer, rows):
     if not layer.rank:
         return 0.0
@@ -133,6 +161,8 @@ MUTATIONS = {
     "bits read MSB first": ("unpack_bit_matrix", _unpack_msb_first),
     "tile/quad axes swapped": ("unpack_bit_matrix", _unpack_tile_quad_swapped),
     "second base dropped": ("_binary_part_rows", _binary_first_base_only),
+    "row-scale group taken as column mod g": ("_binary_part_rows", _binary_group_modulo),
+    "row-scale groups ignored": ("_binary_part_rows", _binary_group_ignored),
     "column scale of base 0 reused": ("_binary_part_rows", _binary_col_scale_of_base0),
     "alpha dropped": ("_correction_part_rows", _correction_alpha_dropped),
     "u read transposed": ("_correction_part_rows", _correction_u_read_transposed),

@@ -55,3 +55,12 @@ def test_salient_recipe_cfg3_small_batch():
 def test_config_table():
     assert [s.in_ for s in CONFIGS[3]["specs"]] == [4096, 11008]
     assert len(CONFIGS[5]["specs"]) == 224
+
+
+def test_grouped_row_scales_shape_and_key():
+    # one row scale per (base, row, group of g input columns); same stream as ungrouped
+    L = make_layer(0, (9,), 40, 300, 2, "bf16", group=128)
+    assert L.group == 128 and L.row_scale.shape == (2, 40, 3) and L.row_scale.dtype == np.uint16
+    L0 = make_layer(0, (9,), 40, 300, 2, "bf16")
+    assert L0.group == 0 and L0.row_scale.shape == (2, 40)
+    assert np.array_equal(L.bits, L0.bits) and np.array_equal(L.col_scale, L0.col_scale)
