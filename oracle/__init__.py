@@ -7,6 +7,7 @@ the CUDA library (``binary_weight_decode_b200``) and neither imports the other.
 
 from .bisco_oracle import (  # noqa: F401
     algorithmic_bytes,
+    biloco_decompose,
     binary_correction_storage_bits,
     correction_z,
     decode_values,

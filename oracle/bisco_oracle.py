@@ -192,6 +192,49 @@ def correction_z(layer, X, x_dtype):
 
 
 # ----------------------------------------------------------------------------
+# binary low-rank decomposition (offline; the correction's sign vectors and alpha)
+# ----------------------------------------------------------------------------
+
+def _sign(a):
+    """+1 / -1 elementwise; a zero takes +1."""
+    return np.where(np.asarray(a) >= 0, 1.0, -1.0)
+
+
+def biloco_decompose(W, v0, rounds=5):
+    """Greedy binary rank-one components of W, then a joint refit of their coefficients
+    ("BiLoCo: Binary Low-Rank Corrections for Post-Training Quantization", "Finding the
+    sign vectors"): starting from the residual R = W, for each component j the sign
+    vectors alternate u = sign(R v), v = sign(R^T u) for `rounds` rounds from the starting
+    signs v0[j] (the random start is an input), alpha_j = u^T R v / (rows * cols) is the
+    error-minimising coefficient of the sign pair, and alpha_j u v^T leaves the residual.
+    The refit solves the least-squares problem for all coefficients at once (the normal
+    equations G alpha = b with G_ij = (u_i . u_j)(v_i . v_j), b_j = u_j^T W v_j).
+
+    Returns U [rows][R], V [R][cols] (entries +-1), the greedy and the refit coefficients.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    rows, cols = W.shape
+    v0 = np.asarray(v0, dtype=np.float64)
+    rank = v0.shape[0]
+    Rs = W.copy()
+    U = np.zeros((rows, rank))
+    V = np.zeros((rank, cols))
+    greedy = np.zeros(rank)
+    for j in range(rank):
+        v = _sign(v0[j])
+        for _ in range(rounds):
+            u = _sign(Rs @ v)
+            v = _sign(Rs.T @ u)
+        a = float(u @ Rs @ v) / (rows * cols)
+        Rs -= a * np.outer(u, v)
+        U[:, j], V[j], greedy[j] = u, v, a
+    G = (U.T @ U) * (V @ V.T)
+    b = np.array([U[:, j] @ W @ V[j] for j in range(rank)])
+    refit = np.linalg.lstsq(G, b, rcond=None)[0]
+    return U, V, greedy, refit
+
+
+# ----------------------------------------------------------------------------
 # storage and byte accounting
 # ----------------------------------------------------------------------------
 

@@ -149,6 +149,50 @@ def test_toy_greedy_coefficients_leave_the_printed_residual():
     assert sse == pytest.approx(g["greedy_residual_sse"], rel=1e-12)
 
 
+def test_biloco_decomposition_reproduces_the_page_toy():
+    # the page's 3x2 walk-through: both greedy components start from v = (+, +)
+    g = golden("toy_decomposition.json")
+    W = np.array(g["W"], dtype=np.float64)
+    U, V, greedy, refit = oracle.biloco_decompose(W, [[1, 1], [1, 1]])
+    for j, c in enumerate(g["components"]):
+        assert np.array_equal(U[:, j], c["u"]) and np.array_equal(V[j], c["v"])
+    assert greedy[0] == g["greedy_alpha_rational"][0][0] / g["greedy_alpha_rational"][0][1]
+    assert greedy[1] == pytest.approx(g["greedy_alpha_rational"][1][0] / g["greedy_alpha_rational"][1][1], rel=1e-15)
+    assert np.array_equal(W - greedy[0] * np.outer(U[:, 0], V[0]), np.array(g["greedy_residual_after_1"], float))
+    sse = float(np.sum((W - (U * greedy) @ V) ** 2))
+    assert sse == pytest.approx(g["greedy_residual_sse"], rel=1e-12)
+    assert np.allclose(refit, g["refit_alpha"], rtol=0, atol=1e-12)
+    # the refit components, run through the correction path of the oracle, rebuild W exactly
+    L = mk(3, 2, rank=2, u=U.astype(int).tolist(), v=V.astype(int).tolist(), alpha=refit)
+    assert np.allclose(oracle.reconstruct(L), W, rtol=0, atol=1e-6)
+
+
+def test_biloco_recovers_an_exact_sign_rank_one_matrix():
+    rng = np.random.default_rng(21)
+    u, v = rng.choice([-1.0, 1.0], size=9), rng.choice([-1.0, 1.0], size=13)
+    W = 3.0 * np.outer(u, v)
+    U, V, greedy, refit = oracle.biloco_decompose(W, rng.choice([-1, 1], size=(1, 13)))
+    assert abs(greedy[0]) == 3.0 and abs(refit[0]) == pytest.approx(3.0, rel=1e-15)
+    assert np.array_equal(greedy[0] * np.outer(U[:, 0], V[0]), W)
+
+
+def test_biloco_refit_is_the_least_squares_optimum():
+    rng = np.random.default_rng(22)
+    W = rng.standard_normal((6, 11))
+    U, V, greedy, refit = oracle.biloco_decompose(W, rng.choice([-1, 1], size=(3, 11)))
+    err = lambda a: float(np.sum((W - (U * a) @ V) ** 2))  # noqa: E731
+    assert err(refit) <= err(greedy) + 1e-12
+    # first-order optimality: the residual is orthogonal to every component, and moving
+    # any coefficient either way raises the error
+    res = W - (U * refit) @ V
+    for j in range(3):
+        assert abs(float(U[:, j] @ res @ V[j])) < 1e-10
+        for d in (-1e-3, 1e-3):
+            a = refit.copy()
+            a[j] += d
+            assert err(a) > err(refit)
+
+
 # --- closed forms and invariants ---------------------------------------------
 
 def _rand_layer(rng, out, in_, K, rank=0, n_sal=0):

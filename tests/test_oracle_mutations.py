@@ -24,6 +24,7 @@ PINS = [
     lambda: P.test_oracle_pack_matches_independent_packer(45, 200),
     P.test_bf16_decode_by_definition,
     P.test_grouped_all_plus_one_is_a_sum_of_group_sums,
+    P.test_biloco_decomposition_reproduces_the_page_toy,
     lambda: P.test_grouped_brute_force_all_sign_patterns(2, 4, 1, 2),
 ]
 
@@ -109,6 +110,19 @@ def _binary_group_ignored(layer, rows):
     return _binary_grouped(layer, rows, lambda i, g: np.zeros_like(i))
 
 
+_orig_decompose = O.biloco_decompose
+
+
+def _decompose_alpha_over_rows(W, v0, rounds=5):
+    U, V, greedy, refit = _orig_decompose(W, v0, rounds)
+    return U, V, greedy * np.asarray(W).shape[1], refit   # u^T R v / rows instead of / (rows*cols)
+
+
+def _decompose_refit_skipped(W, v0, rounds=5):
+    U, V, greedy, _ = _orig_decompose(W, v0, rounds)
+    return U, V, greedy, greedy.copy()
+
+
 def _correction_alpha_dropped(layer, rows):
     if not layer.rank:
         return 0.0
@@ -169,6 +183,8 @@ MUTATIONS = {
     "salient term dropped": ("_salient_part_rows", _salient_dropped),
     "salient column index ignored": ("_salient_part_rows", _salient_wrong_column),
     "W not transposed": ("gemv_rows", _gemv_untransposed),
+    "decomposition coefficient over rows only": ("biloco_decompose", _decompose_alpha_over_rows),
+    "decomposition refit skipped": ("biloco_decompose", _decompose_refit_skipped),
     "bf16 widened with wrong shift": ("decode_values", _bf16_wrong_shift),
 }
 
