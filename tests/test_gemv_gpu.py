@@ -234,3 +234,16 @@ def test_graph_bench_matches_direct_call():
     Y = run(L, X, "bf16", "f32", ws=ws, dl=dl)
     assert np.array_equal(Yg[0].cpu().numpy().astype(np.float64), Y)
     assert np.array_equal(Yg[1].cpu().numpy().astype(np.float64), Y)
+
+
+# ---- row shards: each shard's product is the full product's column slice -----
+
+@pytest.mark.parametrize("world,M", [(3, 1), (2, 40)])
+def test_row_shards_on_the_device(world, M):
+    # every shard runs through bisco_gemv on the same GPU, one after another (no collective):
+    # their outputs side by side must meet the bar against the whole layer's oracle product
+    from binary_weight_decode_b200 import shard
+    X = make_activations(0, (640, M), M, 300, "bf16")
+    L = make_layer(0, (640, M), 200, 300, 2, "bf16", rank=24, sal_frac=0.02, x_for_salience=X, x_dtype="bf16")
+    parts = [run(shard.shard_rows(L, r, world), X, "bf16") for r in range(world)]
+    check(np.concatenate(parts, axis=1), oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
