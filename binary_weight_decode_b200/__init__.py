@@ -24,9 +24,14 @@ _lib = ctypes.CDLL(LIB_PATH)
 BISCO_OK, BISCO_ERR_INVALID_ARG, BISCO_ERR_UNSUPPORTED, BISCO_ERR_CUDA, BISCO_ERR_TIMEOUT, BISCO_ERR_WORKSPACE = range(6)
 BISCO_F32, BISCO_BF16 = 0, 1
 
+BISCO_PATH_AUTO, BISCO_PATH_LOOKUP_TABLE, BISCO_PATH_SMALL_BATCH_ONLY = 0, 1, 2
+(BISCO_KERNEL_LUT_WARP, BISCO_KERNEL_LUT_STREAM, BISCO_KERNEL_LUT_ROWS, BISCO_KERNEL_INTEGER_MMA,
+ BISCO_KERNEL_TENSOR_CORE) = 1, 2, 3, 4, 5
+
 EXPORTED = [
     "bisco_packed_words", "bisco_pack", "bisco_unpack", "bisco_workspace_size", "bisco_workspace_init",
     "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string", "bisco_gemv_noalloc",
+    "bisco_set_path_policy", "bisco_plan_kernels", "bisco_debug_set_wait_test",
 ]
 
 
@@ -79,6 +84,13 @@ _lib.bisco_bench.argtypes = [ctypes.POINTER(bisco_bench_args), ctypes.POINTER(bi
 _lib.bisco_bench.restype = ctypes.c_int
 _lib.bisco_status_string.argtypes = [ctypes.c_int]
 _lib.bisco_status_string.restype = ctypes.c_char_p
+_lib.bisco_set_path_policy.argtypes = [ctypes.c_int32]
+_lib.bisco_set_path_policy.restype = ctypes.c_int
+_lib.bisco_plan_kernels.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_size_t,
+                                    ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+_lib.bisco_plan_kernels.restype = ctypes.c_int32
+_lib.bisco_debug_set_wait_test.argtypes = [ctypes.c_int32, ctypes.c_uint64]
+_lib.bisco_debug_set_wait_test.restype = ctypes.c_int
 
 
 class BiscoError(RuntimeError):
@@ -250,3 +262,26 @@ def bisco_bench(layers, X, Y, ws, warmup: int = 3, reps: int = 10, stream=None) 
     _check(_lib.bisco_bench(ctypes.byref(args), ctypes.byref(res)), "bisco_bench")
     return {"us_per_gemv": res.us_per_gemv, "us_per_replay": res.us_per_replay,
             "kernels_per_gemv": res.kernels_per_gemv}
+
+
+def bisco_set_path_policy(policy: int):
+    """Process-wide choice of kernel family (BISCO_PATH_*); see include/bisco.h."""
+    _check(_lib.bisco_set_path_policy(int(policy)), "bisco_set_path_policy")
+
+
+def bisco_plan_kernels(layer, M: int, x_dtype: int, ws_bytes: int) -> list:
+    """Kernel kinds (BISCO_KERNEL_*) that bisco_gemv would launch, in order."""
+    cap = 64
+    buf = (ctypes.c_int32 * cap)()
+    n = int(_lib.bisco_plan_kernels(ctypes.byref(_desc(layer)), M, x_dtype, ws_bytes, buf, cap))
+    if n < 0:
+        raise BiscoError(BISCO_ERR_INVALID_ARG, "bisco_plan_kernels")
+    if n > cap:
+        buf = (ctypes.c_int32 * n)()
+        n = int(_lib.bisco_plan_kernels(ctypes.byref(_desc(layer)), M, x_dtype, ws_bytes, buf, n))
+    return [int(buf[i]) for i in range(n)]
+
+
+def bisco_debug_set_wait_test(skip_tile: int, wait_ns: int = 0):
+    """Test hook for the integer kernel's bounded waits (skip_tile = -1 turns it off)."""
+    _check(_lib.bisco_debug_set_wait_test(int(skip_tile), int(wait_ns)), "bisco_debug_set_wait_test")

@@ -8,13 +8,15 @@
 // after griddepcontrol.wait, i.e. after pass Z completed.
 //
 // The batch is cut into chunks: up to 128 rows per launch on the tensor-core path
-// when a chunk has at least 16 rows (and the scales are bf16, so that folding a column
-// scale into the expanded signs is exact), otherwise up to 8 rows per launch on the
-// lookup-table kernels.
+// (tcgen05) when a chunk has at least 32 rows (and the scales are bf16, so that folding
+// a column scale into the expanded signs is exact), otherwise up to 8 rows per launch on
+// the integer tensor-core kernel (mma.sync, bisco_imma.cu) when its shared-memory plan
+// fits, else on the lookup-table kernels.
 
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -26,6 +28,12 @@ using namespace bisco;
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// Path policy (bisco_set_path_policy) and the integer kernel's test hooks
+// (bisco_debug_set_wait_test); both are process-wide.
+std::atomic<int> g_policy{BISCO_PATH_AUTO};
+std::atomic<int> g_dbg_skip_tile{-1};
+std::atomic<unsigned long long> g_dbg_wait_ns{0};
 
 int cached_sms(int dev) {
   static int sms[kMaxDevices] = {0};
@@ -84,7 +92,8 @@ SegList segs_y(const bisco_layer* L) {
 }
 
 struct Layout {
-  Plan pz, py;
+  Plan pz, py;          // lookup-table plans
+  ImmaPlan iz, iy;      // integer tensor-core plans (C == 0: none fits)
   bool has_z;
   size_t off_z, total;
 };
@@ -96,9 +105,11 @@ Layout layout_for(const bisco_layer* L, int MB, int dev) {
   lo.has_z = L->rank > 0;
   const SegList sy = segs_y(L);
   lo.py = make_plan(L->out, sy.units, sy.unit0, sy.nseg, MB, L->n_sal, sms, lim);
+  lo.iy = make_imma_plan(L->out, sy.units, sy.unit0, sy.nseg, MB, L->n_sal, lim);
   if (lo.has_z) {
     const int z0 = 0;
     lo.pz = make_plan(L->rank, quads(L->in), &z0, 1, MB, 0, sms, lim);
+    lo.iz = make_imma_plan(L->rank, quads(L->in), &z0, 1, MB, 0, lim);
   }
   lo.off_z = kStatusBytes;
   lo.total = lo.off_z + align256(lo.has_z ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
@@ -141,9 +152,16 @@ bool plans_fit(const Layout& lo, size_t lim) {
   return lo.py.smem <= lim && (!lo.has_z || lo.pz.smem <= lim);
 }
 
+bool imma_fits(const Layout& lo) { return lo.iy.C > 0 && (!lo.has_z || lo.iz.C > 0); }
+
 void fill_plan(PassParam& P, const Plan& pl) {
   P.C = pl.C; P.ncl = pl.ncl; P.max_tiles = pl.max_tiles; P.max_units = pl.max_units;
   P.max_lseg = pl.max_lseg; P.col_stride_bytes = pl.col_stride_bytes;
+}
+
+void fill_imma(PassParam& P, const ImmaPlan& pl) {
+  P.C = pl.C; P.ncl = pl.ncl; P.max_tiles = pl.max_tiles; P.max_units = pl.max_units;
+  P.max_lseg = pl.max_lseg; P.col_stride_bytes = 0;
 }
 
 
@@ -236,8 +254,9 @@ void pass_y(const bisco_layer* L, PassParam& py, const void* Xc, int32_t x_dtype
 // One batch chunk and how it runs.
 struct Chunk {
   int m0, Mc;
-  bool tc;
-  Layout lo;       // lookup-table plans (tc == false)
+  bool tc;         // tcgen05 tensor-core kernel
+  bool imma;       // integer tensor-core kernel (mma.sync); else the lookup-table kernels
+  Layout lo;       // lookup-table and integer plans (tc == false)
   TcPlan tz, ty;   // tensor-core plans (tc == true)
 };
 
@@ -290,7 +309,9 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
     const size_t fit = (ws_bytes - kStatusBytes) / (static_cast<size_t>(L->rank) * 4);
     tc_rows = static_cast<int>(std::min<size_t>(kTcMaxBatch, fit / 16 * 16));
   }
-  const bool tc_ok = (L->num_bases == 0 || L->scale_dtype == BISCO_BF16) && tc_rows >= kTcMinBatch;
+  const int policy = g_policy.load();
+  const bool tc_ok = (L->num_bases == 0 || L->scale_dtype == BISCO_BF16) && tc_rows >= kTcMinBatch &&
+                     policy != BISCO_PATH_SMALL_BATCH_ONLY;
   for (int m0 = 0; m0 < M;) {
     Chunk ch{};
     ch.m0 = m0;
@@ -302,7 +323,9 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
     if (!ch.tc) {
       ch.Mc = std::min(kMaxBatchChunk, rem);
       ch.lo = cached_layout(L, batch_block(ch.Mc), dev);
-      if (!plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
+      // single-row chunks stay on the lookup-table kernels, which are faster there today
+      ch.imma = policy != BISCO_PATH_LOOKUP_TABLE && batch_block(ch.Mc) >= 2 && imma_fits(ch.lo);
+      if (!ch.imma && !plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
     }
     out->push_back(ch);
     m0 += ch.Mc;
@@ -393,22 +416,85 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
 
   int* status = reinterpret_cast<int*>(wsb);
   float* zbuf = reinterpret_cast<float*>(wsb + kStatusBytes);
+  const ImmaDebug dbg{g_dbg_skip_tile.load(), g_dbg_wait_ns.load()};
   for (const Chunk& ch : chunks) {
     const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(ch.m0) * L->in * xb;
     void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(ch.m0) * L->out * yb;
     if (L->rank > 0) {
       PassParam pz{};
       pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);
-      if (!ch.tc) fill_plan(pz, ch.lo.pz);
-      const cudaError_t e = ch.tc ? launch_tc(pz, ch.tz, s) : launch_pass(pz, ch.lo.pz, s, true);
+      cudaError_t e;
+      if (ch.tc) {
+        e = launch_tc(pz, ch.tz, s);
+      } else if (ch.imma) {
+        fill_imma(pz, ch.lo.iz);
+        e = launch_imma(pz, ch.lo.iz, s, true, &dbg);
+      } else {
+        fill_plan(pz, ch.lo.pz);
+        e = launch_pass(pz, ch.lo.pz, s, true);
+      }
       if (e != cudaSuccess) return BISCO_ERR_CUDA;
     }
     PassParam py{};
     pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
-    if (!ch.tc) fill_plan(py, ch.lo.py);
-    const cudaError_t e = ch.tc ? launch_tc(py, ch.ty, s) : launch_pass(py, ch.lo.py, s, true);
+    cudaError_t e;
+    if (ch.tc) {
+      e = launch_tc(py, ch.ty, s);
+    } else if (ch.imma) {
+      fill_imma(py, ch.lo.iy);
+      e = launch_imma(py, ch.lo.iy, s, true, &dbg);
+    } else {
+      fill_plan(py, ch.lo.py);
+      e = launch_pass(py, ch.lo.py, s, true);
+    }
     if (e != cudaSuccess) return BISCO_ERR_CUDA;
   }
+  return BISCO_OK;
+}
+
+bisco_status bisco_set_path_policy(int32_t policy) {
+  if (policy != BISCO_PATH_AUTO && policy != BISCO_PATH_LOOKUP_TABLE && policy != BISCO_PATH_SMALL_BATCH_ONLY)
+    return BISCO_ERR_INVALID_ARG;
+  g_policy.store(policy);
+  return BISCO_OK;
+}
+
+int32_t bisco_plan_kernels(const bisco_layer* L, int32_t M, int32_t x_dtype, size_t ws_bytes, int32_t* kinds,
+                           int32_t max_kinds) {
+  if (validate_layer(L) != BISCO_OK || M < 0 || !dtype_ok(x_dtype) || max_kinds < 0 || (max_kinds > 0 && !kinds))
+    return -1;
+  if (M == 0) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (ws_bytes < ws_need(L, M)) return -1;
+  std::vector<Chunk> chunks;
+  if (plan_chunks(L, M, x_dtype, ws_bytes, dev, &chunks) != BISCO_OK) return -1;
+  int n = 0;
+  auto put = [&](int32_t k) {
+    if (n < max_kinds) kinds[n] = k;
+    ++n;
+  };
+  for (const Chunk& ch : chunks) {
+    const int passes = L->rank > 0 ? 2 : 1;
+    for (int ps = 0; ps < passes; ++ps) {
+      const bool is_z = L->rank > 0 && ps == 0;
+      if (ch.tc) {
+        put(BISCO_KERNEL_TENSOR_CORE);
+      } else if (ch.imma) {
+        put(BISCO_KERNEL_INTEGER_MMA);
+      } else {
+        const Plan& pl = is_z ? ch.lo.pz : ch.lo.py;
+        put(pl.kind == 2 ? BISCO_KERNEL_LUT_STREAM : pl.kind == 0 ? BISCO_KERNEL_LUT_WARP : BISCO_KERNEL_LUT_ROWS);
+      }
+    }
+  }
+  return n;
+}
+
+bisco_status bisco_debug_set_wait_test(int32_t skip_tile, uint64_t wait_ns) {
+  if (skip_tile < -1) return BISCO_ERR_INVALID_ARG;
+  g_dbg_skip_tile.store(skip_tile);
+  g_dbg_wait_ns.store(wait_ns);
   return BISCO_OK;
 }
 
@@ -435,13 +521,9 @@ bisco_status bisco_bench(const bisco_bench_args* a, bisco_bench_result* r) {
     if (a->ws_bytes < ws_need(&a->layers[i], a->M)) return BISCO_ERR_WORKSPACE;
 
   if (ensure_kernel_attrs() != cudaSuccess || tc_ensure_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
-  int launches = 0;
-  {
-    std::vector<Chunk> chunks;
-    const bisco_status st = plan_chunks(&a->layers[0], a->M, a->x_dtype, a->ws_bytes, dev, &chunks);
-    if (st != BISCO_OK) return st;
-    launches = static_cast<int>(chunks.size()) * (a->layers[0].rank > 0 ? 2 : 1);
-  }
+  const int launches = bisco_plan_kernels(&a->layers[0], a->M, a->x_dtype, a->ws_bytes, nullptr, 0);
+  if (launches < 0) return BISCO_ERR_UNSUPPORTED;
+  if (imma_ensure_attrs() != cudaSuccess) return BISCO_ERR_CUDA;
   cudaStream_t user = static_cast<cudaStream_t>(a->stream);
   cudaStream_t cs = nullptr;
   cudaGraph_t graph = nullptr;

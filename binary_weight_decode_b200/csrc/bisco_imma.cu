@@ -1,0 +1,821 @@
+// Binary-weight decode GEMV for batches of up to 8 rows per launch on the integer
+// tensor cores (mma.sync, s8 x s8 -> s32), sm_100a.
+//
+// Per output row o and batch row m the kernel computes
+//   y[m][o] = sum_seg rs_seg[o] * sum_i sign_seg[o][i] * v_seg[m][i]   (+ salient term)
+// where a "segment" is one packed sign matrix: a binary base B_k with v = c_k (.) x and
+// rs = r_k ("FluxBin", Sec. 3.1, decoupled row-column binary bases; the column scale is
+// folded into the activation as in Sec. 3.2, Stage 1), the correction's V with v = x and
+// rs = alpha, or its U^T with v = z ("BiLoCo", "The core idea": alpha * u * (v . x)).
+// A stored bit b means the sign (2b - 1) (FluxBin Sec. 3.2).
+//
+// Formulation. With bits b_i in {0, 1},
+//   sum_i (2 b_i - 1) v_i = 2 * sum_i b_i v_i - sum_i v_i,
+// so the tensor cores only ever multiply by the bits themselves. The activations of a
+// segment are written exactly in fixed point relative to the largest magnitude among
+// the CTA's columns of that segment: V_i = round(v_i * 2^s) with |V_i| <= 2^22, and V_i
+// is split into three signed 8-bit digits, V_i = d0 * 2^16 + d1 * 2^8 + d2. Every pair
+// (batch row, digit) is one column ("slot") of the MMA's B operand: n = 3 m + digit, so
+// one 8-column MMA holds two batch rows, and up to 8 batch rows take three.
+//
+// The A operand never leaves the registers. A lane holds the 32-bit sign words of its
+// rows; (word & (0x01010101 << b)) is four bytes with values {0, 2^b} at columns
+// b, b+8, b+16, b+24 of the word, and the same mask on (word >> 4) gives columns
+// b+4, b+12, b+20, b+28. One m16n8k32 MMA per mask b (b = 0..3) covers a 16-row x
+// 128-column block; each b has its own accumulator (its products carry the factor 2^b),
+// and sum_b (D_b >> b) is exact. The MMA's k index is a permutation of the columns
+// (the B fragments are written in the same permutation), which is what lets one
+// logic op per register extract the bits.
+//
+// Work decomposition. Clusters of C CTAs (one CTA per SM). A cluster owns a range of
+// 32-row tiles; CTA r of the cluster owns 1/C of the units (128-column quads over all
+// segments). Before griddepcontrol.wait (programmatic dependent launch) the CTA starts
+// bulk copies of all its sign words into shared memory (one copy per row tile and
+// segment run, completion counted on one mbarrier per tile) and stages its column and
+// row scales: none of this depends on the previous kernel. After the wait it stages the
+// activations, finds the per-segment scale, writes the B fragments, and the 16 warps
+// run through the (row block, unit) items of the CTA in equal contiguous ranges. Row
+// partial sums meet in shared memory (warp order), then in the owning CTA of the
+// cluster through distributed shared memory (CTA-rank order): results are
+// deterministic.
+
+#include <cooperative_groups.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+#include <utility>
+
+#include "bisco_device.cuh"
+#include "bisco_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace bisco {
+
+namespace {
+
+constexpr int kIW = 8;                  // warps per CTA
+constexpr int kIT = kIW * 32;           // threads per CTA
+constexpr int kMaxSlots = 24;           // 3 digits x 8 batch rows
+constexpr unsigned kByteMask = 0x01010101u;
+
+__host__ __device__ constexpr int groups_of(int MB) { return (3 * MB + 7) / 8; }
+__host__ __device__ constexpr int block_rows(int MB) { return groups_of(MB) == 1 ? 32 : 16; }
+
+// Shared-memory carve-up (sizes from the plan; every region 16-byte aligned).
+struct ISmem {
+  uint64_t* bar;           // [max_tiles]                 sign words of a row tile landed
+  int* useg;               // [max_units]                 local segment of a unit
+  int* lsstart;            // [max_lseg]                  start (local unit index) of a local segment
+  int* lsend;              // [max_lseg]                  end (local unit index) of a local segment
+  int* lsbits;             // [max_lseg]                  1 if the segment has sign bits
+  unsigned* xmax;          // [max_lseg][MB]              max |v| (float bits) over the CTA's columns
+  unsigned long long* vsum;  // [max_lseg][MB]            sum of the fixed-point values V (two's complement)
+  int* flags;              // [4]                         [0]: a wait timed out
+  float* wsl;              // [max_lseg][kMaxSlots][2]    slot weight 2^(17 - 8 digit - s) as two factors
+  float* ssf;              // [max_lseg][MB]              sum of the CTA's quantised v per segment
+  unsigned char* ring;     // [max_tiles][max_units][512] sign words
+  float* xt;               // [max_units][MB][128]        activations times column scales
+  uint4* bfr;              // [max_units][NG][32][2]      B fragments, 8 words per lane
+  float* cs;               // [max_units][128]            column scales (0 past the segment's columns)
+  float* rsc;              // [max_lseg][max_tiles * 32]  row scales
+  float* recv;             // [C][kc][msh][MB]            row partial sums pushed by the warps of the cluster
+  float* xs;               // [MB][nsp]                   salient activations x[idx_t] * s_t
+};
+
+__host__ __device__ __forceinline__ size_t a16(size_t n) { return (n + 15) & ~size_t(15); }
+
+__host__ __device__ __forceinline__ int msh_of(int max_tiles, int C) { return ((max_tiles * 32 + C - 1) / C + 3) & ~3; }
+
+__host__ __device__ __forceinline__ size_t ismem_bytes(int MB, int C, int max_tiles, int max_units, int max_lseg,
+                                                       int nbw, int n_sal) {
+  const int NG = groups_of(MB), RB = block_rows(MB);
+  const int nsp = (n_sal + 3) & ~3;
+  size_t n = 0;
+  n += a16(static_cast<size_t>(max_tiles) * 8);
+  n += a16(static_cast<size_t>(max_units) * 4);
+  n += 3 * a16(static_cast<size_t>(max_lseg) * 4);
+  n += a16(static_cast<size_t>(max_lseg) * MB * 4);
+  n += a16(static_cast<size_t>(max_lseg) * MB * 8);
+  n += 16;
+  n += a16(static_cast<size_t>(max_lseg) * kMaxSlots * 2 * 4);
+  n += a16(static_cast<size_t>(max_lseg) * MB * 4);
+  n += static_cast<size_t>(max_tiles) * max_units * 512;
+  n += static_cast<size_t>(max_units) * MB * 512;
+  n += static_cast<size_t>(max_units) * NG * 1024;
+  n += static_cast<size_t>(max_units) * 512;
+  n += static_cast<size_t>(max_lseg) * max_tiles * 128;
+  n += a16(static_cast<size_t>(C) * nbw * msh_of(max_tiles, C) * MB * 4);
+  n += a16(static_cast<size_t>(MB) * nsp * 4);
+  return n;
+}
+
+__device__ __forceinline__ ISmem icarve(unsigned char* smem, const PassParam& p, int MB, int nbw) {
+  const int NG = groups_of(MB), RB = block_rows(MB);
+  const int nsp = (p.n_sal + 3) & ~3;
+  ISmem s;
+  unsigned char* q = smem;
+  s.bar = reinterpret_cast<uint64_t*>(q);            q += a16(static_cast<size_t>(p.max_tiles) * 8);
+  s.useg = reinterpret_cast<int*>(q);                q += a16(static_cast<size_t>(p.max_units) * 4);
+  s.lsstart = reinterpret_cast<int*>(q);             q += a16(static_cast<size_t>(p.max_lseg) * 4);
+  s.lsend = reinterpret_cast<int*>(q);               q += a16(static_cast<size_t>(p.max_lseg) * 4);
+  s.lsbits = reinterpret_cast<int*>(q);              q += a16(static_cast<size_t>(p.max_lseg) * 4);
+  s.xmax = reinterpret_cast<unsigned*>(q);           q += a16(static_cast<size_t>(p.max_lseg) * MB * 4);
+  s.vsum = reinterpret_cast<unsigned long long*>(q); q += a16(static_cast<size_t>(p.max_lseg) * MB * 8);
+  s.flags = reinterpret_cast<int*>(q);               q += 16;
+  s.wsl = reinterpret_cast<float*>(q);               q += a16(static_cast<size_t>(p.max_lseg) * kMaxSlots * 2 * 4);
+  s.ssf = reinterpret_cast<float*>(q);               q += a16(static_cast<size_t>(p.max_lseg) * MB * 4);
+  s.ring = q;                                        q += static_cast<size_t>(p.max_tiles) * p.max_units * 512;
+  s.xt = reinterpret_cast<float*>(q);                q += static_cast<size_t>(p.max_units) * MB * 512;
+  s.bfr = reinterpret_cast<uint4*>(q);               q += static_cast<size_t>(p.max_units) * NG * 1024;
+  s.cs = reinterpret_cast<float*>(q);                q += static_cast<size_t>(p.max_units) * 512;
+  s.rsc = reinterpret_cast<float*>(q);               q += static_cast<size_t>(p.max_lseg) * p.max_tiles * 128;
+  s.recv = reinterpret_cast<float*>(q);              q += a16(static_cast<size_t>(p.C) * nbw * msh_of(p.max_tiles, p.C) * MB * 4);
+  s.xs = reinterpret_cast<float*>(q);
+  (void)nsp;
+  return s;
+}
+
+__device__ __forceinline__ int seg_of_unit(const PassParam& p, int u) {
+  int s = 0;
+#pragma unroll
+  for (int k = 1; k < kMaxSeg; ++k)
+    if (k < p.nseg && u >= p.seg[k].unit0) s = k;
+  return s;
+}
+
+__device__ __forceinline__ int share_begin_i(int d, int R, int C) { return d * R / C; }
+__device__ __forceinline__ int share_owner_i(int r, int R, int C) { return ((r + 1) * C - 1) / R; }
+
+// Fixed-point exponent of a segment: V = round(v * 2^s) keeps |V| <= 2^22 for every
+// |v| <= vmax. vmax == 0 gives s = 0 (every V is 0).
+__device__ __forceinline__ int fixed_shift(float vmax) {
+  if (!(vmax > 0.f)) return 0;
+  int e;
+  frexpf(vmax, &e);  // vmax = f * 2^e, f in [0.5, 1)
+  return 22 - e;
+}
+// 2^k for any integer k in [-252, 252], as the product of two representable factors.
+__device__ __forceinline__ void pow2_pair(int k, float& f1, float& f2) {
+  const int k1 = max(-126, min(127, k));
+  const int k2 = max(-126, min(127, k - k1));
+  f1 = __int_as_float((k1 + 127) << 23);
+  f2 = __int_as_float((k2 + 127) << 23);
+}
+
+// A holds the masked sign bytes, values 0 or 2^b <= 8, so the signed 8-bit type is exact.
+__device__ __forceinline__ void mma_s8s8(int (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3, unsigned b0,
+                                         unsigned b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The low byte of x, sign-extended.
+__device__ __forceinline__ int sext8(int x) { return static_cast<int>(static_cast<signed char>(x & 0xFF)); }
+
+template <int MB>
+__global__ void __launch_bounds__(kIT, 2)
+    imma_gemv_kernel(const __grid_constant__ PassParam p, const int nbw, const int dbg_skip_tile,
+                     const unsigned long long wait_ns) {
+  constexpr int NG = groups_of(MB);
+  constexpr int RB = block_rows(MB);   // rows per work item
+  constexpr int RH = RB / 16;          // 16-row MMA blocks per item
+  constexpr int BPT = 32 / RB;         // items (row blocks) per row tile
+  extern __shared__ __align__(128) unsigned char smem[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int ci = blockIdx.x / p.C;
+  const int t0 = ci * p.tiles / p.ncl, t1 = (ci + 1) * p.tiles / p.ncl, nt = t1 - t0;
+  const int u0 = rank * p.units / p.C, u1 = (rank + 1) * p.units / p.C, nu = u1 - u0;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g8 = lane >> 2, tq = lane & 3;
+  const int nsp = (p.n_sal + 3) & ~3;
+  const int seg_first = nu > 0 ? seg_of_unit(p, u0) : 0;
+  const int nls = nu > 0 ? seg_of_unit(p, u1 - 1) - seg_first + 1 : 0;
+  const ISmem S = icarve(smem, p, MB, nbw);
+  const int rows_c = nt * 32;
+  const int msh = msh_of(p.max_tiles, p.C);
+
+  // ---- set-up: barriers, unit table, counters ----
+  for (int i = threadIdx.x; i < nt; i += kIT) dev::mbar_init(S.bar + i, 1);
+  for (int ul = threadIdx.x; ul < nu; ul += kIT) {
+    const int sg = seg_of_unit(p, u0 + ul);
+    S.useg[ul] = sg - seg_first;
+  }
+  for (int ls = threadIdx.x; ls < nls; ls += kIT) {
+    const SegParam& G = p.seg[seg_first + ls];
+    S.lsstart[ls] = max(u0, G.unit0) - u0;
+    S.lsend[ls] = min(u1, G.unit0 + G.nq) - u0;
+    S.lsbits[ls] = G.bits != nullptr ? 1 : 0;
+  }
+  for (int i = threadIdx.x; i < nls * MB; i += kIT) { S.xmax[i] = 0u; S.vsum[i] = 0ull; }
+  if (threadIdx.x == 0) S.flags[0] = 0;
+  for (int i = threadIdx.x; i < p.C * nbw * msh * MB; i += kIT) S.recv[i] = 0.f;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __syncthreads();
+  // Peers write into this CTA's shared memory at the end; the split barrier tells them
+  // that every CTA of the cluster is running before any such write happens.
+  auto started = cluster.barrier_arrive();
+
+  // ---- sign words: one bulk copy per (row tile, segment run), issued by many warps ----
+  if (lane == 0) {
+    for (int tl = warp; tl < nt; tl += kIW) {
+      const int t = t0 + tl;
+      unsigned bytes = 0;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSeg; ++sg) {
+        if (sg >= p.nseg) break;
+        const SegParam& G = p.seg[sg];
+        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
+        if (G.bits != nullptr && b > a) bytes += static_cast<unsigned>(b - a) * 512u;
+      }
+      if (tl == dbg_skip_tile) continue;  // test hook: this tile's copies never start
+      dev::mbar_arrive_tx(S.bar + tl, bytes);
+      unsigned char* dst = S.ring + static_cast<size_t>(tl) * nu * 512;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSeg; ++sg) {
+        if (sg >= p.nseg) break;
+        const SegParam& G = p.seg[sg];
+        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
+        if (G.bits != nullptr && b > a)
+          dev::bulk_copy(dst + static_cast<size_t>(a - u0) * 512,
+                         G.bits + (static_cast<long long>(t) * G.nq + (a - G.unit0)) * 32,
+                         static_cast<unsigned>(b - a) * 512u, S.bar + tl);
+      }
+    }
+  }
+
+  // ---- column and row scales (weights only: before the dependency wait) ----
+  {
+    const int n_cs = nu * 16, n_rs = nls * nt * 4;
+    for (int ch = threadIdx.x; ch < n_cs + n_rs; ch += kIT) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      float* d;
+      if (ch < n_cs) {
+        const int ul = ch >> 4, j0 = (ch & 15) * 8;
+        const int u = u0 + ul;
+        const SegParam& G = p.seg[seg_of_unit(p, u)];
+        const int cc = (u - G.unit0) * 128 + j0;
+        const int valid = G.xsrc == 2 ? 0 : max(0, min(8, G.ncols - cc));
+        if (G.cscale == nullptr) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = j < valid ? 1.f : 0.f;
+        } else if (valid > 0) {
+          dev::load8_ro(G.cscale, cc, G.cdt, valid, G.cvec != 0, v);
+        }
+        d = S.cs + ch * 8;
+      } else {
+        const int rc = ch - n_cs;
+        const int ls = rc / (nt * 4), r8 = (rc - ls * nt * 4) * 8;
+        const SegParam& G = p.seg[seg_first + ls];
+        const int o = t0 * 32 + r8;
+        const int valid = max(0, min(8, p.rows - o));
+        if (G.rscale == nullptr) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = j < valid ? 1.f : 0.f;
+        } else if (valid > 0) {
+          dev::load8_ro(G.rscale, o, G.rdt, valid, G.rvec != 0, v);
+        }
+        d = S.rsc + ls * p.max_tiles * 32 + r8;
+      }
+      reinterpret_cast<float4*>(d)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+  __syncthreads();  // column scales visible
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- activations: v = xin * c per (unit, batch row) in column order, 16-byte loads of
+  //      8 consecutive columns, and the maximum |v| per (segment, batch row) ----
+  {
+    const int total = nu * MB * 16;
+    for (int base = 0; base < total; base += kIT) {
+      const int ch = base + threadIdx.x;
+      float mx = 0.f;
+      int lsm = -1;
+      if (ch < total) {
+        const int ulm = ch >> 4, j0 = (ch & 15) * 8;
+        const int ul = ulm / MB, m = ulm - ul * MB;
+        const int u = u0 + ul;
+        const int sg = seg_of_unit(p, u);
+        const SegParam& G = p.seg[sg];
+        const int cc = (u - G.unit0) * 128 + j0;
+        const int valid = max(0, min(8, G.ncols - cc));
+        float xv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xv[j] = 0.f;
+        if (m < p.Mc && valid > 0 && G.xsrc != 2) {
+          if (G.xsrc == 0)
+            dev::load8_act(p.X, static_cast<long long>(m) * p.ldx + cc, p.xdt, valid, p.x_vec != 0, xv);
+          else
+            dev::load8_act(p.Z, static_cast<long long>(m) * p.ldz + cc, BISCO_F32, valid, p.z_vec != 0, xv);
+        }
+        const float* cv = S.cs + ul * 128 + j0;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          v[j] = xv[j] * cv[j];
+          mx = fmaxf(mx, fabsf(v[j]));
+        }
+        float4* d4 = reinterpret_cast<float4*>(S.xt + static_cast<size_t>(ulm) * 128 + j0);
+        d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+        d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+        lsm = (sg - seg_first) * MB + m;
+      }
+      // the 16 lanes of a half-warp share one (unit, batch row)
+#pragma unroll
+      for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if ((lane & 15) == 0 && lsm >= 0) atomicMax(S.xmax + lsm, __float_as_uint(mx));
+    }
+  }
+  // ---- salient activations (gathered and scaled) ----
+  for (int idx = threadIdx.x; idx < MB * p.n_sal; idx += kIT) {
+    const int m = idx / p.n_sal, t = idx - m * p.n_sal;
+    float v = 0.f;
+    const int cc = __ldg(p.sal_idx + t);
+    if (cc < 0 || cc >= p.xcols) {
+      atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+    } else if (m < p.Mc) {
+      const long long i = static_cast<long long>(m) * p.ldx + cc;
+      const float xv = p.xdt == BISCO_BF16
+                           ? __uint_as_float(static_cast<unsigned>(__ldcg(reinterpret_cast<const unsigned short*>(p.X) + i)) << 16)
+                           : __ldcg(reinterpret_cast<const float*>(p.X) + i);
+      v = xv * __ldg(p.sal_scale + t);
+    }
+    S.xs[m * nsp + t] = v;
+  }
+  __syncthreads();  // activations and their maxima complete
+
+  // ---- B fragments: task (unit, batch row, lane-in-group t, mask b, half r) writes the
+  //      words of slots 3m, 3m+1, 3m+2 for the 4 columns 32t + b + 4r + 8i (i = 0..3)
+  //      that MMA b pairs with lane t (register b0 for r = 0, b1 for r = 1) ----
+  {
+    const int total = nu * MB * 32;
+    for (int base = 0; base < total; base += kIT) {
+      const int ch = base + threadIdx.x;
+      long long vs = 0;
+      int lsm = -1;
+      if (ch < total) {
+        const int ulm = ch >> 5, tbr = ch & 31;
+        const int ul = ulm / MB, m = ulm - ul * MB;
+        const int t = tbr >> 3, b = (tbr >> 1) & 3, r = tbr & 1;
+        lsm = S.useg[ul] * MB + m;
+        const int s = fixed_shift(__uint_as_float(S.xmax[lsm]));
+        float f1, f2;
+        pow2_pair(s, f1, f2);
+        const float* xc = S.xt + static_cast<size_t>(ulm) * 128 + 32 * t + b + 4 * r;
+        int d[3][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int V = __float2int_rn((xc[8 * i] * f1) * f2);
+          vs += V;
+          const int d2 = sext8(V);
+          const int r1 = (V - d2) >> 8;
+          const int d1 = sext8(r1);
+          d[0][i] = (r1 - d1) >> 8;
+          d[1][i] = d1;
+          d[2][i] = d2;
+        }
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+          const int n = 3 * m + k;
+          const int g = n >> 3, L = (n & 7) * 4 + t;
+          unsigned* dst = reinterpret_cast<unsigned*>(S.bfr + (static_cast<size_t>(ul) * NG + g) * 64 + L * 2) + 2 * b + r;
+          *dst = __byte_perm(__byte_perm(d[k][0], d[k][1], 0x0040), __byte_perm(d[k][2], d[k][3], 0x0040), 0x5410);
+        }
+      }
+      // the 32 lanes of a warp share one (unit, batch row)
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) vs += __shfl_xor_sync(0xffffffffu, vs, o);
+      if (lane == 0 && lsm >= 0) atomicAdd(S.vsum + lsm, static_cast<unsigned long long>(vs));
+    }
+  }
+  __syncthreads();  // B fragments and sums complete
+  asm volatile("griddepcontrol.launch_dependents;");
+
+  const int nb = nt * BPT;
+  const int items = nb * nu;
+  const int i0 = warp * items / kIW, i1 = (warp + 1) * items / kIW;
+  // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v
+  // (visible after the __syncthreads below)
+  for (int i = threadIdx.x; i < nls * kMaxSlots; i += kIT) {
+    const int ls = i / kMaxSlots, n = i - ls * kMaxSlots;
+    const int m = n / 3, dg = n - 3 * m;
+    float f1 = 0.f, f2 = 0.f;
+    if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
+    S.wsl[2 * i] = f1;
+    S.wsl[2 * i + 1] = f2;
+  }
+  for (int i = threadIdx.x; i < nls * MB; i += kIT) {
+    float f1, f2;
+    pow2_pair(-fixed_shift(__uint_as_float(S.xmax[i])), f1, f2);
+    S.ssf[i] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[i]))) * f1) * f2;
+  }
+  __syncthreads();
+  // peers push into this CTA's receive buffer from here on: every CTA of the cluster
+  // must be running (and have zeroed its buffer) first
+  cluster.barrier_wait(std::move(started));
+
+  // ---- MMA loop over this warp's contiguous range of (row block, unit) items: per row
+  //      block, runs of units of one segment; inside a run the operands of the next unit
+  //      are loaded while the current unit's MMAs issue (two register sets, ping-pong).
+  //      When a warp has finished a row block it pushes the block's row partial sums
+  //      to the CTA that owns the rows (distributed shared memory) ----
+  bool ok = true;
+  {
+    int acc[RH][NG][4][4];
+#pragma unroll
+    for (int h = 0; h < RH; ++h)
+#pragma unroll
+      for (int g = 0; g < NG; ++g)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
+    int cur_tile = -1;
+    bool tile_ok = true;
+    int it = i0;
+    while (it < i1) {
+      const int bl = it / nu;
+      const int tl = bl / BPT;
+      const int ua = it - bl * nu;
+      const int ub = min(nu, i1 - bl * nu);  // this warp's units of block bl: [ua, ub)
+      if (tl != cur_tile) {
+        cur_tile = tl;
+        tile_ok = dev::mbar_wait(S.bar + tl, 0u, wait_ns);
+        if (!tile_ok) ok = false;
+      }
+      const unsigned* wbase = reinterpret_cast<const unsigned*>(S.ring + static_cast<size_t>(tl) * nu * 512) +
+                              ((bl % BPT) * RB + g8) * 4 + tq;
+      const uint4* bbase = S.bfr + lane * 2;
+      float pacc[RH][2][MB];
+#pragma unroll
+      for (int h = 0; h < RH; ++h)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int m = 0; m < MB; ++m) pacc[h][r][m] = 0.f;
+      int ur = ua;
+      while (ur < ub) {
+        const int ls = S.useg[ur];
+        const int ue = min(ub, S.lsend[ls]);
+        if (S.lsbits[ls] && tile_ok) {
+          auto load_b = [&](int ul, unsigned (&B)[NG][8]) {
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+              if (8 * g + g8 < 3 * MB) {
+                const uint4* src = bbase + (static_cast<size_t>(ul) * NG + g) * 64;
+                const uint4 q0 = src[0], q1 = src[1];
+                B[g][0] = q0.x; B[g][1] = q0.y; B[g][2] = q0.z; B[g][3] = q0.w;
+                B[g][4] = q1.x; B[g][5] = q1.y; B[g][6] = q1.z; B[g][7] = q1.w;
+              } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) B[g][k] = 0u;
+              }
+            }
+          };
+          auto load_w = [&](int ul, unsigned (&wv)[2 * RH]) {
+            const unsigned* ws = wbase + ul * 128;
+#pragma unroll
+            for (int k = 0; k < 2 * RH; ++k) wv[k] = ws[k * 32];
+          };
+          auto mma_unit = [&](const unsigned (&B)[NG][8], const unsigned (&wv)[2 * RH]) {
+#pragma unroll
+            for (int h = 0; h < RH; ++h) {
+              const unsigned w0 = wv[2 * h], w1 = wv[2 * h + 1];
+              const unsigned s0 = w0 >> 4, s1 = w1 >> 4;
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const unsigned mk = kByteMask << b;
+                const unsigned a0 = w0 & mk, a1 = w1 & mk, a2 = s0 & mk, a3 = s1 & mk;
+#pragma unroll
+                for (int g = 0; g < NG; ++g) mma_s8s8(acc[h][g][b], a0, a1, a2, a3, B[g][2 * b], B[g][2 * b + 1]);
+              }
+            }
+          };
+          if constexpr (NG <= 2) {
+            unsigned B0[NG][8], B1[NG][8], W0[2 * RH], W1[2 * RH];
+            load_b(ur, B0);
+            load_w(ur, W0);
+            int ul = ur;
+            for (; ul + 1 < ue; ul += 2) {
+              load_b(ul + 1, B1);
+              load_w(ul + 1, W1);
+              mma_unit(B0, W0);
+              if (ul + 2 < ue) {
+                load_b(ul + 2, B0);
+                load_w(ul + 2, W0);
+              }
+              mma_unit(B1, W1);
+            }
+            if (ul < ue) mma_unit(B0, W0);
+          } else {  // three slot groups: registers allow only the sign words to run ahead
+            unsigned B0[NG][8], W0[2 * RH], W1[2 * RH];
+            load_w(ur, W0);
+            int ul = ur;
+            for (; ul + 1 < ue; ul += 2) {
+              load_w(ul + 1, W1);
+              load_b(ul, B0);
+              mma_unit(B0, W0);
+              if (ul + 2 < ue) load_w(ul + 2, W0);
+              load_b(ul + 1, B0);
+              mma_unit(B0, W1);
+            }
+            if (ul < ue) {
+              load_b(ul, B0);
+              mma_unit(B0, W0);
+            }
+          }
+          // drain: D = sum_b (acc_b >> b) per slot, times the slot weight, summed over the
+          // slots of each batch row (the four lanes of a quad), times the row scale; the run
+          // that starts the CTA's range of the segment also subtracts r * sum_i v_i
+          float wlo[NG][2];
+#pragma unroll
+          for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const float2 wf = reinterpret_cast<const float2*>(S.wsl)[ls * kMaxSlots + 8 * g + 2 * tq + e];
+              wlo[g][e] = wf.x * wf.y;  // slot weights are powers of two: the product is exact
+            }
+          const bool first_run = ur == S.lsstart[ls];
+#pragma unroll
+          for (int h = 0; h < RH; ++h) {
+            float cv[2][MB];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+              for (int m = 0; m < MB; ++m) cv[r][m] = 0.f;
+#pragma unroll
+            for (int g = 0; g < NG; ++g) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int n = 8 * g + 2 * tq + (j & 1);
+                const int D = acc[h][g][0][j] + (acc[h][g][1][j] >> 1) + (acc[h][g][2][j] >> 2) + (acc[h][g][3][j] >> 3);
+                const float val = static_cast<float>(D) * wlo[g][j & 1];
+                const int m = n / 3;
+#pragma unroll
+                for (int mm = 0; mm < MB; ++mm) cv[j >> 1][mm] += (m == mm) ? val : 0.f;
+              }
+#pragma unroll
+              for (int b = 0; b < 4; ++b)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              const int row = (bl % BPT) * RB + 16 * h + g8 + 8 * r;  // row within the tile
+              const float rs = S.rsc[ls * p.max_tiles * 32 + tl * 32 + row];
+#pragma unroll
+              for (int mm = 0; mm < MB; ++mm) {
+                float v = cv[r][mm];
+                v += __shfl_xor_sync(0xffffffffu, v, 1);
+                v += __shfl_xor_sync(0xffffffffu, v, 2);
+                if (first_run) v -= S.ssf[ls * MB + mm];
+                pacc[h][r][mm] = fmaf(v, rs, pacc[h][r][mm]);
+              }
+            }
+          }
+        }
+        ur = ue;
+      }
+      // push the block's row partial sums: slot c = this warp's index among the warps
+      // whose item ranges touch block bl (they are consecutive)
+      int wfirst = warp;
+      while (wfirst > 0 && ((wfirst) * items / kIW) > bl * nu) --wfirst;
+      const int c = warp - wfirst;
+      if (tq == 0) {
+#pragma unroll
+        for (int h = 0; h < RH; ++h)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const int lr = bl * RB + 16 * h + g8 + 8 * r;  // row within the cluster's rows
+            const int dst = share_owner_i(lr, rows_c, p.C);
+            float* rp = cluster.map_shared_rank(S.recv, dst) +
+                        ((static_cast<size_t>(rank) * nbw + c) * msh + (lr - share_begin_i(dst, rows_c, p.C))) * MB;
+#pragma unroll
+            for (int mm = 0; mm < MB; ++mm) rp[mm] = pacc[h][r][mm];
+          }
+      }
+      it = bl * nu + ub;
+    }
+  }
+  if (!ok) {
+    atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
+    S.flags[0] = 1;
+  }
+  cluster.sync();  // all partial sums have landed
+  // After a timeout make sure no copy is still writing into shared memory before the
+  // CTA exits: wait, bounded, for every tile's copies.
+  if (S.flags[0] != 0 && threadIdx.x == 0)
+    for (int tl = 0; tl < nt; ++tl)
+      if (tl != dbg_skip_tile) dev::mbar_wait(S.bar + tl, 0u, wait_ns);
+
+  // ---- reduce this CTA's share of rows in CTA-rank order, add salient columns, store ----
+  const int r0 = share_begin_i(rank, rows_c, p.C), r1 = share_begin_i(rank + 1, rows_c, p.C);
+  for (int lr = r0 + threadIdx.x; lr < r1; lr += kIT) {
+    const int o = t0 * 32 + lr;
+    if (o >= p.rows) continue;
+    const int sr = lr - r0;
+    float sum[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) sum[m] = 0.f;
+    for (int src = 0; src < p.C * nbw; ++src) {  // (rank, contributor slot), fixed order
+#pragma unroll
+      for (int m = 0; m < MB; ++m) sum[m] += S.recv[(static_cast<size_t>(src) * msh + sr) * MB + m];
+    }
+    if (p.n_sal > 0) {
+      const int8_t* qrow = p.sal_q + static_cast<long long>(o) * p.sal_stride;
+      for (int tq2 = 0; tq2 < p.n_sal; tq2 += 16) {
+        const uint4 qq = __ldg(reinterpret_cast<const uint4*>(qrow + tq2));
+        const unsigned qw[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int tt = tq2 + k;
+          if (tt < p.n_sal) {
+            const float qv = static_cast<float>(static_cast<int8_t>((qw[k >> 2] >> (8 * (k & 3))) & 0xFF));
+#pragma unroll
+            for (int m = 0; m < MB; ++m) sum[m] = fmaf(qv, S.xs[m * nsp + tt], sum[m]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      if (m < p.Mc) {
+        if (p.ydt == BISCO_BF16)
+          reinterpret_cast<__nv_bfloat16*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = __float2bfloat16_rn(sum[m]);
+        else
+          reinterpret_cast<float*>(p.Y)[static_cast<long long>(m) * p.ldy + o] = sum[m];
+      }
+    }
+  }
+}
+
+template <int MB>
+int imma_clusters(int C, size_t smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C);
+  cfg.blockDim = dim3(kIT);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, imma_gemv_kernel<MB>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int imma_clusters_mb(int MB, int C, size_t smem) {
+  switch (MB) {
+    case 1: return imma_clusters<1>(C, smem);
+    case 2: return imma_clusters<2>(C, smem);
+    case 4: return imma_clusters<4>(C, smem);
+    case 8: return imma_clusters<8>(C, smem);
+    default: return 0;
+  }
+}
+
+int max_segments_per_cta_i(int units, int C, const int* seg_unit0, int nseg) {
+  auto seg_of = [&](int u) {
+    int s = 0;
+    for (int k = 1; k < nseg; ++k)
+      if (u >= seg_unit0[k]) s = k;
+    return s;
+  };
+  int m = 1;
+  for (int r = 0; r < C; ++r) {
+    const int a = r * units / C, b = (r + 1) * units / C;
+    if (b > a) m = std::max(m, seg_of(b - 1) - seg_of(a) + 1);
+  }
+  return m;
+}
+
+template <int MB>
+cudaError_t imma_set_attrs(size_t lim) {
+  cudaError_t e = cudaFuncSetAttribute(imma_gemv_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(lim));
+  return e;
+}
+
+}  // namespace
+
+cudaError_t imma_ensure_attrs() {
+  static std::once_flag once[64];
+  static cudaError_t err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::call_once(once[dev & 63], [&] {
+    const size_t lim = query_smem_limit();
+    cudaError_t r = imma_set_attrs<1>(lim);
+    if (r == cudaSuccess) r = imma_set_attrs<2>(lim);
+    if (r == cudaSuccess) r = imma_set_attrs<4>(lim);
+    if (r == cudaSuccess) r = imma_set_attrs<8>(lim);
+    err[dev & 63] = r;
+  });
+  return err[dev & 63];
+}
+
+// Plan: the cluster size C in {1, 2, 4, 8} that minimises a cycle estimate per SM --
+// tensor-core time of the largest CTA share (8 MMAs per 32 x 128 block and group of 8
+// slots, at the measured 0.42 m16n8k32 MMAs per clock and SM with 8 warps), the
+// B-fragment writes (about 200 lane operations per task of 8 columns and one batch row,
+// 64 lanes per clock for one CTA), a fixed cost for the cluster reduction, and a fixed
+// cost when the CTA takes more than half of the SM's shared memory (then the next
+// kernel's CTA cannot be resident beside it and start its copies early) -- among the
+// plans whose shared memory fits. The grid has at most one CTA of the launch per SM.
+// C = 0 in the result means no plan fits.
+ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, size_t smem_limit) {
+  ImmaPlan best{};
+  if (imma_ensure_attrs() != cudaSuccess) return best;
+  int dev = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+  // two CTAs per SM: each gets half of the SM's shared memory less the 1 KB the
+  // hardware reserves per CTA
+  const size_t half = per_sm > 0 ? static_cast<size_t>(per_sm) / 2 - 1024 : smem_limit / 2;
+  const int tiles = (rows + 31) / 32;
+  const int NG = groups_of(MB), RB = block_rows(MB);
+  double best_cost = -1;
+  for (int C = 1; C <= kMaxCluster; C *= 2) {
+    if (C > 1 && C > units) break;
+    const int max_units = (units + C - 1) / C;
+    const int max_lseg = max_segments_per_cta_i(units, C, seg_unit0, nseg);
+    // clusters that fit with one CTA of the launch per SM (the query asks for more
+    // than half of the SM's shared memory)
+    const size_t force = smem_limit / 2 + 1024;
+    int fit = imma_clusters_mb(MB, C, force);
+    if (fit <= 0) continue;
+    const int ncl = std::max(1, std::min(tiles, fit));
+    const int max_tiles = (tiles + ncl - 1) / ncl;
+    // contributor slots per row: warps own equal contiguous ranges of (row block, unit)
+    // items, so with at least kIW row blocks in every CTA a block is touched by at most
+    // two warps; otherwise by at most kIW
+    const int nb_min = (tiles / ncl) * (32 / RB);
+    const int nbw = nb_min >= kIW ? 2 : kIW;
+    const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, nbw, n_sal);
+    if (need > smem_limit) continue;
+    const bool coresident = need <= half;
+    const double mma = static_cast<double>(max_tiles) * max_units * 8.0 * NG / 0.42;
+    const double bfr = static_cast<double>(max_units) * MB * 16.0 * 200.0 / 64.0;
+    const double red = C > 1 ? 600.0 : 150.0;
+    const double cost = mma + bfr + red + (coresident ? 0.0 : 2500.0);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best.C = C;
+      best.ncl = ncl;
+      best.max_tiles = max_tiles;
+      best.max_units = max_units;
+      best.max_lseg = max_lseg;
+      best.nbw = nbw;
+      best.MB = MB;
+      best.smem = coresident ? need : std::max(need, force);
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_imma(const PassParam& p, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
+                        const ImmaDebug* dbg) {
+  const cudaError_t e = imma_ensure_attrs();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.ncl * plan.C);
+  cfg.blockDim = dim3(kIT);
+  cfg.dynamicSmemBytes = plan.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = plan.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  const int skip = dbg ? dbg->skip_tile : -1;
+  const unsigned long long wait_ns = dbg && dbg->wait_ns ? dbg->wait_ns : kDefaultWaitNs;
+  switch (plan.MB) {
+    case 1: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1>, p, plan.nbw, skip, wait_ns);
+    case 2: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2>, p, plan.nbw, skip, wait_ns);
+    case 4: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4>, p, plan.nbw, skip, wait_ns);
+    case 8: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8>, p, plan.nbw, skip, wait_ns);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace bisco

@@ -85,7 +85,28 @@ cudaError_t ensure_kernel_attrs();
 int query_num_sms();
 size_t query_smem_limit();
 
-// Tensor-core path (16..128 batch rows per launch): one launch per pass.
+// Integer tensor-core GEMV (mma.sync u8 x s8) for batch chunks of up to 8 rows.
+struct ImmaPlan {
+  int C, ncl;            // cluster size (K split) and clusters; C == 0: no plan fits
+  int max_tiles;         // 32-row tiles of the largest cluster share
+  int max_units;         // 128-column units of the largest CTA share
+  int max_lseg;          // segments a CTA's unit range touches, at most
+  int nbw;               // partial-sum slots per row and CTA (warps whose items touch one row block)
+  int MB;                // batch rows per launch (1, 2, 4 or 8)
+  size_t smem;
+};
+// Test hooks of the integer kernel: skip_tile >= 0 leaves that row tile's sign-word
+// copies unissued (its waiters give up after wait_ns and report BISCO_ERR_TIMEOUT).
+struct ImmaDebug {
+  int skip_tile;
+  unsigned long long wait_ns;
+};
+constexpr unsigned long long kDefaultWaitNs = 200000000ull;  // bound on every mbarrier wait (200 ms)
+ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, size_t smem_limit);
+cudaError_t launch_imma(const PassParam& p, const ImmaPlan& plan, cudaStream_t stream, bool pdl, const ImmaDebug* dbg);
+cudaError_t imma_ensure_attrs();
+
+// Tensor-core path (32..128 batch rows per launch): one launch per pass.
 constexpr int kTcMinBatch = 32;           // smallest batch chunk sent to the tensor cores
 constexpr int kTcMaxBatch = 128;          // batch rows per launch
 struct TcPlan {

@@ -1,13 +1,12 @@
 // bisco_gemv_noalloc: the GEMV entry point for callers that cannot allocate device memory.
 //
 // Some callers have no way to obtain a workspace buffer: a plug-in loaded into a host
-// application that owns every device allocation, code that runs while a stream is
-// being captured into a CUDA graph (where a fresh allocation would break the capture),
-// or a runtime whose device memory is fully reserved at start-up. For them this file
-// keeps the scratch space bisco_gemv needs (the device status word and, for layers with
-// a binary low-rank correction, the intermediate z of one batch chunk) in a fixed array
-// that lives in the library's own device image. Every GPU that loads the library holds
-// this array until the process exits.
+// application that owns every device allocation and hands the plug-in only its
+// operands, or a runtime whose device memory is fully reserved at start-up. For them
+// this file keeps the scratch space bisco_gemv needs (the device status word and, for
+// layers with a binary low-rank correction, the intermediate z of one batch chunk) in a
+// fixed array that lives in the library's own device image. Every GPU that loads the
+// library holds this array until the process exits.
 
 #include <cuda_runtime.h>
 
@@ -26,19 +25,26 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 
 // Device address of g_noalloc_scratch on each device. The symbol's name is only a
-// host-side handle, so the address is looked up once per device, with that device
-// current, and cached.
+// host-side handle, so the address is looked up with that device current and cached.
+// Only a successful lookup is cached: a failed one (e.g. a transient error) is retried
+// on the next call. A device reset (cudaDeviceReset) invalidates the cached address;
+// callers that reset a device must not call this entry point on it afterwards.
 void* scratch_address(int dev, cudaError_t* err) {
-  static std::once_flag once[kMaxDevices];
+  static std::mutex mu[kMaxDevices];
   static void* addr[kMaxDevices];
-  static cudaError_t status[kMaxDevices];
-  std::call_once(once[dev], [dev] {
-    void* p = nullptr;
-    status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    addr[dev] = status[dev] == cudaSuccess ? p : nullptr;
-  });
-  *err = status[dev];
-  return addr[dev];
+  std::lock_guard<std::mutex> g(mu[dev]);
+  if (addr[dev] != nullptr) {
+    *err = cudaSuccess;
+    return addr[dev];
+  }
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (*err != cudaSuccess) {
+    cudaGetLastError();  // clear the (non-sticky) error so that a retry starts clean
+    return nullptr;
+  }
+  addr[dev] = p;
+  return p;
 }
 
 }  // namespace

@@ -142,6 +142,52 @@ bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype
 bisco_status bisco_sync_status(void* stream, const void* ws);
 
 /*
+ * Which kernel family runs a batch chunk (process-wide; for tests and diagnostics).
+ *  BISCO_PATH_AUTO (default): chunks of 32..128 rows on the tcgen05 tensor-core kernel
+ *    (bf16 scales), chunks of 2..8 rows on the integer tensor-core kernel (mma.sync)
+ *    when its shared-memory plan fits, single rows and the rest on the lookup-table
+ *    kernels.
+ *  BISCO_PATH_LOOKUP_TABLE: as AUTO, but chunks of up to 8 rows always take the
+ *    lookup-table kernels (FluxBin Sec. 3.2, Stages 1-3, restated for B200).
+ *  BISCO_PATH_SMALL_BATCH_ONLY: as AUTO, but every chunk has at most 8 rows (no
+ *    tcgen05 kernel).
+ * Every path computes the same product within the documented tolerance.
+ * Returns BISCO_ERR_INVALID_ARG for an unknown policy.
+ */
+enum { BISCO_PATH_AUTO = 0, BISCO_PATH_LOOKUP_TABLE = 1, BISCO_PATH_SMALL_BATCH_ONLY = 2 };
+bisco_status bisco_set_path_policy(int32_t policy);
+
+/* Kernel kinds reported by bisco_plan_kernels. */
+enum {
+  BISCO_KERNEL_LUT_WARP = 1,      /* lookup tables, 16-warp CTAs, <= 2 batch rows        */
+  BISCO_KERNEL_LUT_STREAM = 2,    /* lookup tables, bulk-copy sign stream, <= 2 rows     */
+  BISCO_KERNEL_LUT_ROWS = 3,      /* lookup tables, warps own row tiles, 4 or 8 rows     */
+  BISCO_KERNEL_INTEGER_MMA = 4,   /* int8 tensor cores (mma.sync), <= 8 rows             */
+  BISCO_KERNEL_TENSOR_CORE = 5    /* tcgen05 tensor cores, 32..128 rows                  */
+};
+
+/*
+ * The kernel launches bisco_gemv would issue for this layer, batch M, activation dtype
+ * and workspace size under the current path policy, in launch order. Writes up to
+ * max_kinds entries of kinds (host array) and returns the number of launches, or -1 if
+ * the request is invalid or unsupported (same checks as bisco_gemv). Needs the device
+ * whose plans are queried to be current; launches nothing.
+ */
+int32_t bisco_plan_kernels(const bisco_layer* layer, int32_t M, int32_t x_dtype, size_t ws_bytes, int32_t* kinds,
+                           int32_t max_kinds);
+
+/*
+ * Test hook for the bounded device-side waits of the integer tensor-core kernel.
+ * With skip_tile >= 0, every later launch of that kernel leaves the sign-word copies of
+ * local row tile skip_tile of each CTA unissued, so the warps that wait for them give
+ * up after wait_ns nanoseconds (0: the default limit, 200 ms) and record
+ * BISCO_ERR_TIMEOUT in the workspace status word; no copy is in flight into that tile's
+ * shared memory when they give up. skip_tile = -1 restores normal operation.
+ * Process-wide; BISCO_ERR_INVALID_ARG for skip_tile < -1.
+ */
+bisco_status bisco_debug_set_wait_test(int32_t skip_tile, uint64_t wait_ns);
+
+/*
  * Largest correction rank bisco_gemv_noalloc accepts.
  */
 #define BISCO_NOALLOC_MAX_RANK 4096
@@ -151,8 +197,8 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  * papers: this is a deployment convenience of this library.)
  *
  * For callers that cannot allocate device memory -- e.g. a plug-in inside a host
- * application that owns all device allocations, or code running while a stream is
- * captured into a CUDA graph, where a new allocation would break the capture. The
+ * application that owns every device allocation and passes the plug-in only its
+ * operands, or a runtime that reserves all device memory at start-up. The
  * scratch space (status word and the correction's intermediate z for one batch chunk)
  * is a fixed array of 256 + 8 * 4096 * 4 bytes in the library's device image; every GPU
  * that loads the library keeps it until the process exits. This call allocates nothing.
@@ -160,7 +206,12 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  * Arguments and results are those of bisco_gemv, minus the workspace. Layers with
  * rank > BISCO_NOALLOC_MAX_RANK are rejected with BISCO_ERR_UNSUPPORTED.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
- * make that first call before any stream capture starts.
+ * make that first call before any stream capture starts. A failed lookup is not cached
+ * (the next call retries); a device reset invalidates the cached address.
+ * With the fixed array, z fits at most floor(8192 / rank) batch rows, so a batch chunk on
+ * the tcgen05 tensor-core kernel (32..128 rows) is limited to floor(8192 / rank / 16) * 16
+ * rows; layers with rank > 256 run every chunk on the small-batch kernels (correct, slower
+ * at large batch than bisco_gemv with its preferred workspace).
  * All calls share the one array: calls that may overlap on the GPU (different streams,
  * or different host threads) race with each other; order them on one stream.
  * Device-side errors are recorded in the shared array and cannot be read back through

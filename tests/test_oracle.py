@@ -448,6 +448,23 @@ def test_algorithmic_bytes_counts_each_payload():
     assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 4_243_456 + extra
 
 
+def test_algorithmic_bytes_salient_term():
+    # Llama-7B gate/up layer (out 11008, in 4096, two bases, bf16 scales) with 41 salient
+    # columns, batch 1, bf16 in and out, counted term by term by hand:
+    #   signs 2*11008*4096/8 = 11,272,192; scales 2*(11008+4096)*2 = 60,416;
+    #   salient int8 block 11008*41 = 451,328, fp32 scales 41*4 = 164, int32 indices 41*4 = 164;
+    #   x 4096*2 = 8,192; y 11008*2 = 22,016                         -> 11,814,472
+    L = Layer(out=11008, in_=4096, K=2, scale_dtype="bf16", bits=None, row_scale=None, col_scale=None, n_sal=41)
+    assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 11_814_472
+    # the down projection (out 4096, in 11008) with 111 salient columns:
+    #   11,272,192 + 60,416 + 4096*111 + 111*8 + 11008*2 + 4096*2 -> 11,818,360
+    L = Layer(out=4096, in_=11008, K=2, scale_dtype="bf16", bits=None, row_scale=None, col_scale=None, n_sal=111)
+    assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 11_818_360
+    # each salient column adds one int8 per output row plus its scale and its index
+    L.n_sal = 112
+    assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 11_818_360 + 4096 + 8
+
+
 @pytest.mark.parametrize("rows,cols", [(70, 300), (33, 129), (1, 5)])
 def test_row_decoder_matches_independent_packer(rows, cols):
     S = np.random.default_rng(7 * rows + cols).choice(np.array([-1, 1], np.int8), size=(rows, cols))

@@ -1,8 +1,8 @@
 """bisco_gemv_noalloc: the entry point for callers that cannot allocate device memory.
 
-Such callers (a plug-in whose host application owns every device allocation, or code
-running while a stream is captured into a graph, where a fresh allocation would break
-the capture) cannot hand bisco_gemv a workspace. bisco_gemv_noalloc uses a fixed
+Such callers (a plug-in whose host application owns every device allocation and
+passes it only its operands, or a runtime that reserves all device memory at start-up)
+cannot hand bisco_gemv a workspace. bisco_gemv_noalloc uses a fixed
 scratch array inside the library instead. This file checks, through the C ABI, that
 two calls in a row give what bisco_gemv gives with a caller-provided workspace, and
 that a rank above the array's limit is refused without touching the output.
