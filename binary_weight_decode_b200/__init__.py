@@ -24,7 +24,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 BISCO_OK, BISCO_ERR_INVALID_ARG, BISCO_ERR_UNSUPPORTED, BISCO_ERR_CUDA, BISCO_ERR_TIMEOUT, BISCO_ERR_WORKSPACE = range(6)
 BISCO_F32, BISCO_BF16 = 0, 1
 
-BISCO_PATH_AUTO, BISCO_PATH_LOOKUP_TABLE, BISCO_PATH_SMALL_BATCH_ONLY = 0, 1, 2
+BISCO_PATH_AUTO, BISCO_PATH_LOOKUP_TABLE, BISCO_PATH_SMALL_BATCH_ONLY, BISCO_PATH_INTEGER_MMA = 0, 1, 2, 3
 (BISCO_KERNEL_LUT_WARP, BISCO_KERNEL_LUT_STREAM, BISCO_KERNEL_LUT_ROWS, BISCO_KERNEL_INTEGER_MMA,
  BISCO_KERNEL_TENSOR_CORE) = 1, 2, 3, 4, 5
 

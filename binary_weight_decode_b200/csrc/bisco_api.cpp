@@ -324,7 +324,8 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
       ch.Mc = std::min(kMaxBatchChunk, rem);
       ch.lo = cached_layout(L, batch_block(ch.Mc), dev);
       // single-row chunks stay on the lookup-table kernels, which are faster there today
-      ch.imma = policy != BISCO_PATH_LOOKUP_TABLE && batch_block(ch.Mc) >= 2 && imma_fits(ch.lo);
+      ch.imma = policy != BISCO_PATH_LOOKUP_TABLE && imma_fits(ch.lo) &&
+                (batch_block(ch.Mc) >= 2 || policy == BISCO_PATH_INTEGER_MMA);
       if (!ch.imma && !plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
     }
     out->push_back(ch);
@@ -453,7 +454,8 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
 }
 
 bisco_status bisco_set_path_policy(int32_t policy) {
-  if (policy != BISCO_PATH_AUTO && policy != BISCO_PATH_LOOKUP_TABLE && policy != BISCO_PATH_SMALL_BATCH_ONLY)
+  if (policy != BISCO_PATH_AUTO && policy != BISCO_PATH_LOOKUP_TABLE && policy != BISCO_PATH_SMALL_BATCH_ONLY &&
+      policy != BISCO_PATH_INTEGER_MMA)
     return BISCO_ERR_INVALID_ARG;
   g_policy.store(policy);
   return BISCO_OK;

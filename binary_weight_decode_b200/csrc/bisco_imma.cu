@@ -74,7 +74,7 @@ struct ISmem {
   unsigned* xmax;          // [max_lseg][MB]              max |v| (float bits) over the CTA's columns
   unsigned long long* vsum;  // [max_lseg][MB]            sum of the fixed-point values V (two's complement)
   int* flags;              // [4]                         [0]: a wait timed out
-  float* wsl;              // [max_lseg][kMaxSlots][2]    slot weight 2^(17 - 8 digit - s) as two factors
+  float* wsl;              // [max_lseg][kMaxSlots]       slot weight 2^(17 - 8 digit - s)
   float* ssf;              // [max_lseg][MB]              sum of the CTA's quantised v per segment
   unsigned char* ring;     // [max_tiles][max_units][512] sign words
   float* xt;               // [max_units][MB][128]        activations times column scales
@@ -221,35 +221,8 @@ __global__ void __launch_bounds__(kIT, 2)
   // that every CTA of the cluster is running before any such write happens.
   auto started = cluster.barrier_arrive();
 
-  // ---- sign words: one bulk copy per (row tile, segment run), issued by many warps ----
-  if (lane == 0) {
-    for (int tl = warp; tl < nt; tl += kIW) {
-      const int t = t0 + tl;
-      unsigned bytes = 0;
-#pragma unroll
-      for (int sg = 0; sg < kMaxSeg; ++sg) {
-        if (sg >= p.nseg) break;
-        const SegParam& G = p.seg[sg];
-        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
-        if (G.bits != nullptr && b > a) bytes += static_cast<unsigned>(b - a) * 512u;
-      }
-      if (tl == dbg_skip_tile) continue;  // test hook: this tile's copies never start
-      dev::mbar_arrive_tx(S.bar + tl, bytes);
-      unsigned char* dst = S.ring + static_cast<size_t>(tl) * nu * 512;
-#pragma unroll
-      for (int sg = 0; sg < kMaxSeg; ++sg) {
-        if (sg >= p.nseg) break;
-        const SegParam& G = p.seg[sg];
-        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
-        if (G.bits != nullptr && b > a)
-          dev::bulk_copy(dst + static_cast<size_t>(a - u0) * 512,
-                         G.bits + (static_cast<long long>(t) * G.nq + (a - G.unit0)) * 32,
-                         static_cast<unsigned>(b - a) * 512u, S.bar + tl);
-      }
-    }
-  }
-
-  // ---- column and row scales (weights only: before the dependency wait) ----
+  // ---- column and row scales (weights only: before the dependency wait; issued ahead of
+  //      the sign-word copies so that they are not queued behind them) ----
   {
     const int n_cs = nu * 16, n_rs = nls * nt * 4;
     for (int ch = threadIdx.x; ch < n_cs + n_rs; ch += kIT) {
@@ -288,9 +261,36 @@ __global__ void __launch_bounds__(kIT, 2)
       reinterpret_cast<float4*>(d)[1] = make_float4(v[4], v[5], v[6], v[7]);
     }
   }
-  __syncthreads();  // column scales visible
+  // ---- sign words: one bulk copy per (row tile, segment run), issued by many warps ----
+  if (lane == 0) {
+    for (int tl = warp; tl < nt; tl += kIW) {
+      const int t = t0 + tl;
+      unsigned bytes = 0;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSeg; ++sg) {
+        if (sg >= p.nseg) break;
+        const SegParam& G = p.seg[sg];
+        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
+        if (G.bits != nullptr && b > a) bytes += static_cast<unsigned>(b - a) * 512u;
+      }
+      if (tl == dbg_skip_tile) continue;  // test hook: this tile's copies never start
+      dev::mbar_arrive_tx(S.bar + tl, bytes);
+      unsigned char* dst = S.ring + static_cast<size_t>(tl) * nu * 512;
+#pragma unroll
+      for (int sg = 0; sg < kMaxSeg; ++sg) {
+        if (sg >= p.nseg) break;
+        const SegParam& G = p.seg[sg];
+        const int a = max(u0, G.unit0), b = min(u1, G.unit0 + G.nq);
+        if (G.bits != nullptr && b > a)
+          dev::bulk_copy(dst + static_cast<size_t>(a - u0) * 512,
+                         G.bits + (static_cast<long long>(t) * G.nq + (a - G.unit0)) * 32,
+                         static_cast<unsigned>(b - a) * 512u, S.bar + tl);
+      }
+    }
+  }
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  __syncthreads();  // column scales visible
 
   // ---- activations: v = xin * c per (unit, batch row) in column order, 16-byte loads of
   //      8 consecutive columns, and the maximum |v| per (segment, batch row) ----
@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(kIT, 2)
     const int total = nu * MB * 32;
     for (int base = 0; base < total; base += kIT) {
       const int ch = base + threadIdx.x;
-      long long vs = 0;
+      int vs = 0;  // 4 values of |V| <= 2^22 per lane, 32 lanes: |sum| <= 2^29
       int lsm = -1;
       if (ch < total) {
         const int ulm = ch >> 5, tbr = ch & 31;
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kIT, 2)
       // the 32 lanes of a warp share one (unit, batch row)
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) vs += __shfl_xor_sync(0xffffffffu, vs, o);
-      if (lane == 0 && lsm >= 0) atomicAdd(S.vsum + lsm, static_cast<unsigned long long>(vs));
+      if (lane == 0 && lsm >= 0) atomicAdd(S.vsum + lsm, static_cast<unsigned long long>(static_cast<long long>(vs)));
     }
   }
   __syncthreads();  // B fragments and sums complete
@@ -403,25 +403,21 @@ __global__ void __launch_bounds__(kIT, 2)
   const int nb = nt * BPT;
   const int items = nb * nu;
   const int i0 = warp * items / kIW, i1 = (warp + 1) * items / kIW;
-  // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v
-  // (visible after the __syncthreads below)
-  for (int i = threadIdx.x; i < nls * kMaxSlots; i += kIT) {
-    const int ls = i / kMaxSlots, n = i - ls * kMaxSlots;
+  // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v, read
+  // by the drains below
+  if (threadIdx.x < nls * kMaxSlots) {
+    const int ls = threadIdx.x / kMaxSlots, n = threadIdx.x - ls * kMaxSlots;
     const int m = n / 3, dg = n - 3 * m;
     float f1 = 0.f, f2 = 0.f;
     if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
-    S.wsl[2 * i] = f1;
-    S.wsl[2 * i + 1] = f2;
-  }
-  for (int i = threadIdx.x; i < nls * MB; i += kIT) {
+    S.wsl[threadIdx.x] = f1 * f2;  // powers of two: the product is exact
+  } else if (threadIdx.x - nls * kMaxSlots < nls * MB) {
+    const int i = threadIdx.x - nls * kMaxSlots;
     float f1, f2;
     pow2_pair(-fixed_shift(__uint_as_float(S.xmax[i])), f1, f2);
     S.ssf[i] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[i]))) * f1) * f2;
   }
   __syncthreads();
-  // peers push into this CTA's receive buffer from here on: every CTA of the cluster
-  // must be running (and have zeroed its buffer) first
-  cluster.barrier_wait(std::move(started));
 
   // ---- MMA loop over this warp's contiguous range of (row block, unit) items: per row
   //      block, runs of units of one segment; inside a run the operands of the next unit
@@ -429,6 +425,7 @@ __global__ void __launch_bounds__(kIT, 2)
   //      When a warp has finished a row block it pushes the block's row partial sums
   //      to the CTA that owns the rows (distributed shared memory) ----
   bool ok = true;
+  bool waited = false;  // this thread has completed the cluster barrier started above
   {
     int acc[RH][NG][4][4];
 #pragma unroll
@@ -538,12 +535,11 @@ __global__ void __launch_bounds__(kIT, 2)
           // that starts the CTA's range of the segment also subtracts r * sum_i v_i
           float wlo[NG][2];
 #pragma unroll
-          for (int g = 0; g < NG; ++g)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const float2 wf = reinterpret_cast<const float2*>(S.wsl)[ls * kMaxSlots + 8 * g + 2 * tq + e];
-              wlo[g][e] = wf.x * wf.y;  // slot weights are powers of two: the product is exact
-            }
+          for (int g = 0; g < NG; ++g) {
+            const float2 wf = reinterpret_cast<const float2*>(S.wsl)[(ls * kMaxSlots + 8 * g + 2 * tq) >> 1];
+            wlo[g][0] = wf.x;
+            wlo[g][1] = wf.y;
+          }
           const bool first_run = ur == S.lsstart[ls];
 #pragma unroll
           for (int h = 0; h < RH; ++h) {
@@ -585,23 +581,48 @@ __global__ void __launch_bounds__(kIT, 2)
         }
         ur = ue;
       }
-      // push the block's row partial sums: slot c = this warp's index among the warps
-      // whose item ranges touch block bl (they are consecutive)
+      // push the block's row partial sums to the CTA that owns the rows, one store per
+      // lane: after the quad reduction every lane of a quad holds the same sums, so lane tq
+      // takes one (half, row) pair (32-row blocks) or one row and half the batch rows
+      // (16-row blocks). Slot c = this warp's index among the consecutive warps whose item
+      // ranges touch block bl.
+      if (!waited) {  // peers must be running and have zeroed their buffers
+        cluster.barrier_wait(std::move(started));
+        waited = true;
+      }
       int wfirst = warp;
       while (wfirst > 0 && ((wfirst) * items / kIW) > bl * nu) --wfirst;
       const int c = warp - wfirst;
-      if (tq == 0) {
+      {
+        constexpr int VPL = RH == 2 ? MB : MB / 2;  // values per lane
+        const int hh = RH == 2 ? (tq >> 1) : 0;
+        const int rr = tq & 1;
+        const int m0 = RH == 2 ? 0 : (tq >> 1) * (MB / 2);
+        float v[VPL];
 #pragma unroll
-        for (int h = 0; h < RH; ++h)
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int lr = bl * RB + 16 * h + g8 + 8 * r;  // row within the cluster's rows
-            const int dst = share_owner_i(lr, rows_c, p.C);
-            float* rp = cluster.map_shared_rank(S.recv, dst) +
-                        ((static_cast<size_t>(rank) * nbw + c) * msh + (lr - share_begin_i(dst, rows_c, p.C))) * MB;
-#pragma unroll
-            for (int mm = 0; mm < MB; ++mm) rp[mm] = pacc[h][r][mm];
+        for (int e = 0; e < VPL; ++e) {
+          if constexpr (RH == 2) {  // (hh, rr) from tq; all MB values
+            const float lo = rr ? pacc[0][1][e] : pacc[0][0][e];
+            const float hi = rr ? pacc[RH - 1][1][e] : pacc[RH - 1][0][e];
+            v[e] = hh ? hi : lo;
+          } else {  // rr from tq, batch rows e or MB/2 + e
+            const float a = rr ? pacc[0][1][e] : pacc[0][0][e];
+            const float b = rr ? pacc[0][1][(MB / 2 + e) % MB] : pacc[0][0][(MB / 2 + e) % MB];
+            v[e] = (tq >> 1) ? b : a;
           }
+        }
+        const int lr = bl * RB + 16 * hh + g8 + 8 * rr;  // row within the cluster's rows
+        const int dst = share_owner_i(lr, rows_c, p.C);
+        float* rp = cluster.map_shared_rank(S.recv, dst) +
+                    ((static_cast<size_t>(rank) * nbw + c) * msh + (lr - share_begin_i(dst, rows_c, p.C))) * MB + m0;
+        if constexpr (VPL == 1) {
+          rp[0] = v[0];
+        } else if constexpr (VPL == 2) {
+          *reinterpret_cast<float2*>(rp) = make_float2(v[0], v[1]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < VPL; e += 4) *reinterpret_cast<float4*>(rp + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
       }
       it = bl * nu + ub;
     }
@@ -610,6 +631,7 @@ __global__ void __launch_bounds__(kIT, 2)
     atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
     S.flags[0] = 1;
   }
+  if (!waited) cluster.barrier_wait(std::move(started));  // warps without items
   cluster.sync();  // all partial sums have landed
   // After a timeout make sure no copy is still writing into shared memory before the
   // CTA exits: wait, bounded, for every tile's copies.
@@ -732,12 +754,16 @@ cudaError_t imma_ensure_attrs() {
 
 // Plan: the cluster size C in {1, 2, 4, 8} that minimises a cycle estimate per SM --
 // tensor-core time of the largest CTA share (8 MMAs per 32 x 128 block and group of 8
-// slots, at the measured 0.42 m16n8k32 MMAs per clock and SM with 8 warps), the
-// B-fragment writes (about 200 lane operations per task of 8 columns and one batch row,
-// 64 lanes per clock for one CTA), a fixed cost for the cluster reduction, and a fixed
-// cost when the CTA takes more than half of the SM's shared memory (then the next
-// kernel's CTA cannot be resident beside it and start its copies early) -- among the
-// plans whose shared memory fits. The grid has at most one CTA of the launch per SM.
+// slots; a legacy m16n8k32 MMA holds its sub-partition's issue for about 10 cycles and
+// the masks add about half as much again: measured 237 cycles per 32 x 128 block and
+// warp with 8 warps per SM), the B-fragment writes (about 60 lane operations per task of
+// 4 columns and one batch row, 64 lanes per clock for one CTA), and a fixed cost for the
+// cluster reduction, plus a fixed cost when the CTA takes more than half of the SM's
+// shared memory (the next kernel's CTA then cannot be resident beside it) -- among the
+// plans whose shared memory fits. The grid holds as many CTAs as fit one per SM; with
+// half an SM or less per CTA the block scheduler still places two CTAs of one launch on
+// some SMs (measured: 120 CTAs on 98 SMs), which those SMs pay for, but exposing the next
+// kernel's prologue costs more.
 // C = 0 in the result means no plan fits.
 ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, size_t smem_limit) {
   ImmaPlan best{};
@@ -769,10 +795,14 @@ ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int
     const int nbw = nb_min >= kIW ? 2 : kIW;
     const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, nbw, n_sal);
     if (need > smem_limit) continue;
+    // kIW warps of a CTA work on kIW blocks at once: 237 / kIW cycles per block and SM
+    const double mma = static_cast<double>(max_tiles) * max_units * NG * 237.0 / kIW;
+    const double bfr = static_cast<double>(max_units) * MB * 32.0 * 60.0 / 64.0;
+    const double red = C > 1 ? 1500.0 : 300.0;
+    // a CTA of at most half an SM lets the next kernel's CTA (launched early) be resident
+    // beside it and run its prologue during this kernel; a larger one exposes that
+    // prologue (measured on the 4096 x 4096 layer: 6.85 us vs 8.08 us per GEMV)
     const bool coresident = need <= half;
-    const double mma = static_cast<double>(max_tiles) * max_units * 8.0 * NG / 0.42;
-    const double bfr = static_cast<double>(max_units) * MB * 16.0 * 200.0 / 64.0;
-    const double red = C > 1 ? 600.0 : 150.0;
     const double cost = mma + bfr + red + (coresident ? 0.0 : 2500.0);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;

@@ -151,10 +151,12 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  *    lookup-table kernels (FluxBin Sec. 3.2, Stages 1-3, restated for B200).
  *  BISCO_PATH_SMALL_BATCH_ONLY: as AUTO, but every chunk has at most 8 rows (no
  *    tcgen05 kernel).
+ *  BISCO_PATH_INTEGER_MMA: as AUTO, but chunks of up to 8 rows, single rows included,
+ *    take the integer tensor-core kernel whenever its plan fits.
  * Every path computes the same product within the documented tolerance.
  * Returns BISCO_ERR_INVALID_ARG for an unknown policy.
  */
-enum { BISCO_PATH_AUTO = 0, BISCO_PATH_LOOKUP_TABLE = 1, BISCO_PATH_SMALL_BATCH_ONLY = 2 };
+enum { BISCO_PATH_AUTO = 0, BISCO_PATH_LOOKUP_TABLE = 1, BISCO_PATH_SMALL_BATCH_ONLY = 2, BISCO_PATH_INTEGER_MMA = 3 };
 bisco_status bisco_set_path_policy(int32_t policy);
 
 /* Kernel kinds reported by bisco_plan_kernels. */

@@ -112,6 +112,41 @@ def test_lookup_table_kernels_elementwise(policy, case):
     check(run(L, X, xdt, "f32"), oracle.gemv(L, X, xdt), X, xdt, "f32")
 
 
+# ---- integer kernel on single batch rows (BISCO_PATH_INTEGER_MMA) ---------------
+
+INT_ONE_ROW = [
+    # out, in, K, scale_dtype, rank, sal_frac, x_dtype
+    (1, 1, 1, "f32", 0, 0.0, "f32"),
+    (33, 129, 2, "bf16", 0, 0.0, "bf16"),
+    (96, 385, 1, "bf16", 129, 0.0, "bf16"),
+    (300, 333, 0, "bf16", 5, 0.0, "bf16"),
+    (64, 256, 0, "bf16", 0, 0.05, "bf16"),
+    (1024, 1024, 2, "bf16", 64, 0.01, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", INT_ONE_ROW, ids=[f"{c[0]}x{c[1]}K{c[2]}R{c[4]}" for c in INT_ONE_ROW])
+def test_integer_kernel_one_row_elementwise(policy, case):
+    policy(bw.BISCO_PATH_INTEGER_MMA)
+    out, in_, K, sdt, rank, sal, xdt = case
+    key = (93, out, in_, K, rank)
+    X = make_activations(0, key, 1, in_, xdt)
+    L = make_layer(0, key, out, in_, K, sdt, rank=rank, sal_frac=sal, x_for_salience=X if sal else None, x_dtype=xdt)
+    assert set(kinds(L, 1, xdt)) == {bw.BISCO_KERNEL_INTEGER_MMA}
+    for ydt in ("f32", "bf16"):
+        check(run(L, X, xdt, ydt), oracle.gemv(L, X, xdt), X, xdt, ydt)
+
+
+@pytest.mark.parametrize("cfg,spec", [(2, 0), (3, 0), (3, 1), (4, 0)], ids=["cfg2", "cfg3_gate_up", "cfg3_down", "cfg4"])
+def test_integer_kernel_one_row_workloads_sampled(policy, cfg, spec):
+    policy(bw.BISCO_PATH_INTEGER_MMA)
+    L, X = build(cfg, spec, 1)
+    assert set(kinds(L, 1)) == {bw.BISCO_KERNEL_INTEGER_MMA}
+    Y = run(L, X, "bf16", "f32")
+    rows = sample_rows(L.out, 192, 3 + spec)
+    check(Y[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
+
+
 # ---- integer kernel: activation magnitudes and batch sizes ----------------------
 
 @pytest.mark.parametrize("scale_exp", [-100, -20, 0, 20, 100])
