@@ -426,7 +426,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);
       cudaError_t e;
       if (ch.tc) {
-        e = launch_tc(pz, ch.tz, s);
+        e = launch_tc(pz, ch.tz, s, &dbg);
       } else if (ch.imma) {
         fill_imma(pz, ch.lo.iz);
         e = launch_imma(pz, ch.lo.iz, s, true, &dbg);
@@ -440,7 +440,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
     pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
     cudaError_t e;
     if (ch.tc) {
-      e = launch_tc(py, ch.ty, s);
+      e = launch_tc(py, ch.ty, s, &dbg);
     } else if (ch.imma) {
       fill_imma(py, ch.lo.iy);
       e = launch_imma(py, ch.lo.iy, s, true, &dbg);

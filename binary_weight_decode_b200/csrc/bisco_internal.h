@@ -95,8 +95,10 @@ struct ImmaPlan {
   int MB;                // batch rows per launch (1, 2, 4 or 8)
   size_t smem;
 };
-// Test hooks of the integer kernel: skip_tile >= 0 leaves that row tile's sign-word
-// copies unissued (its waiters give up after wait_ns and report BISCO_ERR_TIMEOUT).
+// Test hooks of the bounded device-side waits: skip_tile >= 0 leaves sign-word copies
+// unissued (the integer kernel: those of local row tile skip_tile; the tcgen05 kernel:
+// those of each CTA's last step), so their waiters give up after wait_ns and report
+// BISCO_ERR_TIMEOUT.
 struct ImmaDebug {
   int skip_tile;
   unsigned long long wait_ns;
@@ -122,7 +124,7 @@ struct TcPlan {
 // seg_kind[s] is SegParam::xsrc of segment s; seg_ncols[s] its columns.
 TcPlan make_tc_plan(int rows, int nseg, const int* seg_kind, const int* seg_ncols, int n_sal, bool x_bf16, int Mc,
                     int num_sms, size_t smem_limit);
-cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream);
+cudaError_t launch_tc(const PassParam& p, const TcPlan& t, cudaStream_t stream, const ImmaDebug* dbg);
 cudaError_t tc_ensure_attrs();
 
 }  // namespace bisco

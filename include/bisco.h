@@ -179,13 +179,14 @@ int32_t bisco_plan_kernels(const bisco_layer* layer, int32_t M, int32_t x_dtype,
                            int32_t max_kinds);
 
 /*
- * Test hook for the bounded device-side waits of the integer tensor-core kernel.
- * With skip_tile >= 0, every later launch of that kernel leaves the sign-word copies of
- * local row tile skip_tile of each CTA unissued, so the warps that wait for them give
- * up after wait_ns nanoseconds (0: the default limit, 200 ms) and record
- * BISCO_ERR_TIMEOUT in the workspace status word; no copy is in flight into that tile's
- * shared memory when they give up. skip_tile = -1 restores normal operation.
- * Process-wide; BISCO_ERR_INVALID_ARG for skip_tile < -1.
+ * Test hook for the bounded device-side waits of the tensor-core kernels.
+ * With skip_tile >= 0, every later launch leaves some sign-word copies unissued: the
+ * integer tensor-core kernel those of local row tile skip_tile of each CTA, the tcgen05
+ * kernel those of each CTA's last step. The threads that wait for them give up after
+ * wait_ns nanoseconds (0: the default limit, 200 ms) and record BISCO_ERR_TIMEOUT in the
+ * workspace status word; no copy is in flight into the skipped shared memory when they
+ * give up, and the kernels still release their tensor memory. skip_tile = -1 restores
+ * normal operation. Process-wide; BISCO_ERR_INVALID_ARG for skip_tile < -1.
  */
 bisco_status bisco_debug_set_wait_test(int32_t skip_tile, uint64_t wait_ns);
 

@@ -208,3 +208,28 @@ def test_integer_kernel_wait_gives_up_and_reports_timeout():
     assert bw.bisco_sync_status(ws) == bw.BISCO_OK
     Y = Yd.cpu().numpy().astype(np.float64)
     check(Y, oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
+
+
+def test_tensor_core_kernel_wait_gives_up_and_reports_timeout():
+    # the tcgen05 kernel: the last step's sign-word copy of every CTA is never issued;
+    # the producers' bounded wait gives up after 1 ms, the kernel still reaches its
+    # tensor-memory release (the next launch allocates all 512 columns again), the status
+    # word reads BISCO_ERR_TIMEOUT, and after bisco_workspace_init the next call is correct
+    L, X = build(2, 0, 64)
+    dl = bw.DeviceLayer(L)
+    assert kinds(L, 64) == [bw.BISCO_KERNEL_TENSOR_CORE]
+    ws = bw.alloc_workspace([dl], 64)
+    Xd = to_dev_x(X, "bf16")
+    Yd = torch.empty((64, L.out), dtype=torch.float32, device="cuda")
+    try:
+        bw.bisco_debug_set_wait_test(0, 1_000_000)
+        bw.bisco_gemv(dl, Xd, Yd, ws)
+        assert bw.bisco_sync_status(ws) == bw.BISCO_ERR_TIMEOUT
+    finally:
+        bw.bisco_debug_set_wait_test(-1, 0)
+    bw.bisco_workspace_init(ws)
+    bw.bisco_gemv(dl, Xd, Yd, ws)
+    assert bw.bisco_sync_status(ws) == bw.BISCO_OK
+    rows = sample_rows(L.out, 128, 5)
+    Y = Yd.cpu().numpy().astype(np.float64)[:, rows]
+    check(Y, oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
