@@ -177,10 +177,17 @@ __device__ __forceinline__ void mma_s8s8(int (&c)[4], unsigned a0, unsigned a1, 
 // The low byte of x, sign-extended.
 __device__ __forceinline__ int sext8(int x) { return static_cast<int>(static_cast<signed char>(x & 0xFF)); }
 
-template <int MB>
+// One launch computes one pass (pz unused, ncl_z = 0), or -- the correction fused into
+// one launch -- both: the first ncl_z clusters compute z = alpha (.) (V x) (pass pz) into
+// the workspace and count their CTAs done on a ready counter; the other clusters compute
+// pass py, first the units that do not read z (the bases), then, after a bounded wait
+// for the counter, the U^T units. Every CTA of the grid is resident before the next
+// kernel on the stream can start, and the z producers wait for nothing but the
+// previous kernel, so the wait always ends; it is bounded anyway (BISCO_ERR_TIMEOUT).
+template <int MB, bool FUSED>
 __global__ void __launch_bounds__(kIT, 2)
-    imma_gemv_kernel(const __grid_constant__ PassParam p, const int nbw, const int dbg_skip_tile,
-                     const unsigned long long wait_ns) {
+    imma_gemv_kernel(const __grid_constant__ PassParam pz, const __grid_constant__ PassParam py, const int ncl_z,
+                     const int kc, const int dbg_skip_tile, const unsigned long long wait_ns) {
   constexpr int NG = groups_of(MB);
   constexpr int RB = block_rows(MB);   // rows per work item
   constexpr int RH = RB / 16;          // 16-row MMA blocks per item
@@ -188,7 +195,11 @@ __global__ void __launch_bounds__(kIT, 2)
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int ci = blockIdx.x / p.C;
+  const int ci_all = blockIdx.x / py.C;
+  constexpr bool fused = FUSED;
+  const bool role_z = FUSED && ci_all < ncl_z;
+  const PassParam& p = role_z ? pz : py;
+  const int ci = role_z ? ci_all : ci_all - ncl_z;
   const int t0 = ci * p.tiles / p.ncl, t1 = (ci + 1) * p.tiles / p.ncl, nt = t1 - t0;
   const int u0 = rank * p.units / p.C, u1 = (rank + 1) * p.units / p.C, nu = u1 - u0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -196,9 +207,11 @@ __global__ void __launch_bounds__(kIT, 2)
   const int nsp = (p.n_sal + 3) & ~3;
   const int seg_first = nu > 0 ? seg_of_unit(p, u0) : 0;
   const int nls = nu > 0 ? seg_of_unit(p, u1 - 1) - seg_first + 1 : 0;
-  const ISmem S = icarve(smem, p, MB, nbw);
+  const ISmem S = icarve(smem, p, MB, kc);
   const int rows_c = nt * 32;
   const int msh = msh_of(p.max_tiles, p.C);
+  int* const z_ready = p.status + 32;  // counters in the workspace's status region
+  int* const z_done = p.status + 33;
 
   // ---- set-up: barriers, unit table, counters ----
   for (int i = threadIdx.x; i < nt; i += kIT) dev::mbar_init(S.bar + i, 1);
@@ -213,8 +226,8 @@ __global__ void __launch_bounds__(kIT, 2)
     S.lsbits[ls] = G.bits != nullptr ? 1 : 0;
   }
   for (int i = threadIdx.x; i < nls * MB; i += kIT) { S.xmax[i] = 0u; S.vsum[i] = 0ull; }
-  if (threadIdx.x == 0) S.flags[0] = 0;
-  for (int i = threadIdx.x; i < p.C * nbw * msh * MB; i += kIT) S.recv[i] = 0.f;
+  if (threadIdx.x == 0) { S.flags[0] = 0; S.flags[1] = 0; }
+  for (int i = threadIdx.x; i < p.C * kc * msh * MB; i += kIT) S.recv[i] = 0.f;
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   __syncthreads();
   // Peers write into this CTA's shared memory at the end; the split barrier tells them
@@ -292,49 +305,6 @@ __global__ void __launch_bounds__(kIT, 2)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __syncthreads();  // column scales visible
 
-  // ---- activations: v = xin * c per (unit, batch row) in column order, 16-byte loads of
-  //      8 consecutive columns, and the maximum |v| per (segment, batch row) ----
-  {
-    const int total = nu * MB * 16;
-    for (int base = 0; base < total; base += kIT) {
-      const int ch = base + threadIdx.x;
-      float mx = 0.f;
-      int lsm = -1;
-      if (ch < total) {
-        const int ulm = ch >> 4, j0 = (ch & 15) * 8;
-        const int ul = ulm / MB, m = ulm - ul * MB;
-        const int u = u0 + ul;
-        const int sg = seg_of_unit(p, u);
-        const SegParam& G = p.seg[sg];
-        const int cc = (u - G.unit0) * 128 + j0;
-        const int valid = max(0, min(8, G.ncols - cc));
-        float xv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) xv[j] = 0.f;
-        if (m < p.Mc && valid > 0 && G.xsrc != 2) {
-          if (G.xsrc == 0)
-            dev::load8_act(p.X, static_cast<long long>(m) * p.ldx + cc, p.xdt, valid, p.x_vec != 0, xv);
-          else
-            dev::load8_act(p.Z, static_cast<long long>(m) * p.ldz + cc, BISCO_F32, valid, p.z_vec != 0, xv);
-        }
-        const float* cv = S.cs + ul * 128 + j0;
-        float v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v[j] = xv[j] * cv[j];
-          mx = fmaxf(mx, fabsf(v[j]));
-        }
-        float4* d4 = reinterpret_cast<float4*>(S.xt + static_cast<size_t>(ulm) * 128 + j0);
-        d4[0] = make_float4(v[0], v[1], v[2], v[3]);
-        d4[1] = make_float4(v[4], v[5], v[6], v[7]);
-        lsm = (sg - seg_first) * MB + m;
-      }
-      // the 16 lanes of a half-warp share one (unit, batch row)
-#pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      if ((lane & 15) == 0 && lsm >= 0) atomicMax(S.xmax + lsm, __float_as_uint(mx));
-    }
-  }
   // ---- salient activations (gathered and scaled) ----
   for (int idx = threadIdx.x; idx < MB * p.n_sal; idx += kIT) {
     const int m = idx / p.n_sal, t = idx - m * p.n_sal;
@@ -351,280 +321,361 @@ __global__ void __launch_bounds__(kIT, 2)
     }
     S.xs[m * nsp + t] = v;
   }
-  __syncthreads();  // activations and their maxima complete
 
-  // ---- B fragments: task (unit, batch row, lane-in-group t, mask b, half r) writes the
-  //      words of slots 3m, 3m+1, 3m+2 for the 4 columns 32t + b + 4r + 8i (i = 0..3)
-  //      that MMA b pairs with lane t (register b0 for r = 0, b1 for r = 1) ----
-  {
-    const int total = nu * MB * 32;
-    for (int base = 0; base < total; base += kIT) {
-      const int ch = base + threadIdx.x;
-      int vs = 0;  // 4 values of |V| <= 2^22 per lane, 32 lanes: |sum| <= 2^29
-      int lsm = -1;
-      if (ch < total) {
-        const int ulm = ch >> 5, tbr = ch & 31;
-        const int ul = ulm / MB, m = ulm - ul * MB;
-        const int t = tbr >> 3, b = (tbr >> 1) & 3, r = tbr & 1;
-        lsm = S.useg[ul] * MB + m;
-        const int s = fixed_shift(__uint_as_float(S.xmax[lsm]));
-        float f1, f2;
-        pow2_pair(s, f1, f2);
-        const float* xc = S.xt + static_cast<size_t>(ulm) * 128 + 32 * t + b + 4 * r;
-        int d[3][4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int V = __float2int_rn((xc[8 * i] * f1) * f2);
-          vs += V;
-          const int d2 = sext8(V);
-          const int r1 = (V - d2) >> 8;
-          const int d1 = sext8(r1);
-          d[0][i] = (r1 - d1) >> 8;
-          d[1][i] = d1;
-          d[2][i] = d2;
-        }
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-          const int n = 3 * m + k;
-          const int g = n >> 3, L = (n & 7) * 4 + t;
-          unsigned* dst = reinterpret_cast<unsigned*>(S.bfr + (static_cast<size_t>(ul) * NG + g) * 64 + L * 2) + 2 * b + r;
-          *dst = __byte_perm(__byte_perm(d[k][0], d[k][1], 0x0040), __byte_perm(d[k][2], d[k][3], 0x0040), 0x5410);
-        }
-      }
-      // the 32 lanes of a warp share one (unit, batch row)
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) vs += __shfl_xor_sync(0xffffffffu, vs, o);
-      if (lane == 0 && lsm >= 0) atomicAdd(S.vsum + lsm, static_cast<unsigned long long>(static_cast<long long>(vs)));
-    }
-  }
-  __syncthreads();  // B fragments and sums complete
-  asm volatile("griddepcontrol.launch_dependents;");
-
-  const int nb = nt * BPT;
-  const int items = nb * nu;
-  const int i0 = warp * items / kIW, i1 = (warp + 1) * items / kIW;
-  // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v, read
-  // by the drains below
-  if (threadIdx.x < nls * kMaxSlots) {
-    const int ls = threadIdx.x / kMaxSlots, n = threadIdx.x - ls * kMaxSlots;
-    const int m = n / 3, dg = n - 3 * m;
-    float f1 = 0.f, f2 = 0.f;
-    if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
-    S.wsl[threadIdx.x] = f1 * f2;  // powers of two: the product is exact
-  } else if (threadIdx.x - nls * kMaxSlots < nls * MB) {
-    const int i = threadIdx.x - nls * kMaxSlots;
-    float f1, f2;
-    pow2_pair(-fixed_shift(__uint_as_float(S.xmax[i])), f1, f2);
-    S.ssf[i] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[i]))) * f1) * f2;
-  }
-  __syncthreads();
-
-  // ---- MMA loop over this warp's contiguous range of (row block, unit) items: per row
-  //      block, runs of units of one segment; inside a run the operands of the next unit
-  //      are loaded while the current unit's MMAs issue (two register sets, ping-pong).
-  //      When a warp has finished a row block it pushes the block's row partial sums
-  //      to the CTA that owns the rows (distributed shared memory) ----
+  // ---- phases: the units that do not read z, then (fused launches) the U^T units ----
+  int uT = nu;  // first local unit of a z-reading segment
+  if (fused && !role_z)
+    for (int ls = 0; ls < nls; ++ls)
+      if (p.seg[seg_first + ls].xsrc == 1) { uT = min(uT, S.lsstart[ls]); }
+  const int nph = (fused && !role_z && uT < nu && uT > 0) ? 2 : 1;
+  const int kcp = kc / (fused ? 2 : 1);  // contributor slots per phase
   bool ok = true;
   bool waited = false;  // this thread has completed the cluster barrier started above
-  {
-    int acc[RH][NG][4][4];
-#pragma unroll
-    for (int h = 0; h < RH; ++h)
-#pragma unroll
-      for (int g = 0; g < NG; ++g)
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
-    int cur_tile = -1;
-    bool tile_ok = true;
-    int it = i0;
-    while (it < i1) {
-      const int bl = it / nu;
-      const int tl = bl / BPT;
-      const int ua = it - bl * nu;
-      const int ub = min(nu, i1 - bl * nu);  // this warp's units of block bl: [ua, ub)
-      if (tl != cur_tile) {
-        cur_tile = tl;
-        tile_ok = dev::mbar_wait(S.bar + tl, 0u, wait_ns);
-        if (!tile_ok) ok = false;
+  for (int ph = 0; ph < nph; ++ph) {
+    const int pa = nph == 1 ? 0 : (ph == 0 ? 0 : uT);
+    const int pb = nph == 1 ? nu : (ph == 0 ? uT : nu);
+    const int nun = pb - pa;
+    const bool reads_z = fused && !role_z && (ph == 1 || (nph == 1 && uT == 0));
+    if (reads_z) {
+      // z is read from here on: wait (bounded) until every z-producing CTA has counted
+      // its stores
+      if (threadIdx.x == 0) {
+        const int target = ncl_z * p.C;
+        const unsigned long long end = dev::global_ns() + wait_ns;
+        bool ready = false;
+        while (!ready) {
+          int v;
+          asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(z_ready) : "memory");
+          ready = v >= target;
+          if (!ready && dev::global_ns() > end) break;
+        }
+        if (!ready) {
+          atomicExch(p.status, static_cast<int>(BISCO_ERR_TIMEOUT));
+          S.flags[1] = 1;
+        } else {
+          S.flags[1] = 0;
+        }
       }
-      const unsigned* wbase = reinterpret_cast<const unsigned*>(S.ring + static_cast<size_t>(tl) * nu * 512) +
-                              ((bl % BPT) * RB + g8) * 4 + tq;
-      const uint4* bbase = S.bfr + lane * 2;
-      float pacc[RH][2][MB];
+      __syncthreads();
+    }
+
+    // ---- activations: v = xin * c per (unit, batch row) in column order, 16-byte loads of
+    //      8 consecutive columns, and the maximum |v| per (segment, batch row) ----
+    {
+      const int total = nun * MB * 16;
+      for (int base = 0; base < total; base += kIT) {
+        const int ch = base + threadIdx.x;
+        float mx = 0.f;
+        int lsm = -1;
+        if (ch < total) {
+          const int ulm = pa * MB + (ch >> 4), j0 = (ch & 15) * 8;
+          const int ul = ulm / MB, m = ulm - ul * MB;
+          const int u = u0 + ul;
+          const int sg = seg_of_unit(p, u);
+          const SegParam& G = p.seg[sg];
+          const int cc = (u - G.unit0) * 128 + j0;
+          const int valid = max(0, min(8, G.ncols - cc));
+          float xv[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) xv[j] = 0.f;
+          if (m < p.Mc && valid > 0 && G.xsrc != 2) {
+            if (G.xsrc == 0)
+              dev::load8_act(p.X, static_cast<long long>(m) * p.ldx + cc, p.xdt, valid, p.x_vec != 0, xv);
+            else
+              dev::load8_act(p.Z, static_cast<long long>(m) * p.ldz + cc, BISCO_F32, valid, p.z_vec != 0, xv);
+          }
+          const float* cv = S.cs + ul * 128 + j0;
+          float v[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            v[j] = xv[j] * cv[j];
+            mx = fmaxf(mx, fabsf(v[j]));
+          }
+          float4* d4 = reinterpret_cast<float4*>(S.xt + static_cast<size_t>(ulm) * 128 + j0);
+          d4[0] = make_float4(v[0], v[1], v[2], v[3]);
+          d4[1] = make_float4(v[4], v[5], v[6], v[7]);
+          lsm = (sg - seg_first) * MB + m;
+        }
+        // the 16 lanes of a half-warp share one (unit, batch row)
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        if ((lane & 15) == 0 && lsm >= 0) atomicMax(S.xmax + lsm, __float_as_uint(mx));
+      }
+    }
+    __syncthreads();  // activations and their maxima complete
+
+    // ---- B fragments: task (unit, batch row, lane-in-group t, mask b, half r) writes the
+    //      words of slots 3m, 3m+1, 3m+2 for the 4 columns 32t + b + 4r + 8i (i = 0..3)
+    //      that MMA b pairs with lane t (register b0 for r = 0, b1 for r = 1) ----
+    {
+      const int total = nun * MB * 32;
+      for (int base = 0; base < total; base += kIT) {
+        const int ch = base + threadIdx.x;
+        int vs = 0;  // 4 values of |V| <= 2^22 per lane, 32 lanes: |sum| <= 2^29
+        int lsm = -1;
+        if (ch < total) {
+          const int ulm = pa * MB + (ch >> 5), tbr = ch & 31;
+          const int ul = ulm / MB, m = ulm - ul * MB;
+          const int t = tbr >> 3, b = (tbr >> 1) & 3, r = tbr & 1;
+          lsm = S.useg[ul] * MB + m;
+          const int s = fixed_shift(__uint_as_float(S.xmax[lsm]));
+          float f1, f2;
+          pow2_pair(s, f1, f2);
+          const float* xc = S.xt + static_cast<size_t>(ulm) * 128 + 32 * t + b + 4 * r;
+          int d[3][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int V = __float2int_rn((xc[8 * i] * f1) * f2);
+            vs += V;
+            const int d2 = sext8(V);
+            const int r1 = (V - d2) >> 8;
+            const int d1 = sext8(r1);
+            d[0][i] = (r1 - d1) >> 8;
+            d[1][i] = d1;
+            d[2][i] = d2;
+          }
+#pragma unroll
+          for (int k = 0; k < 3; ++k) {
+            const int n = 3 * m + k;
+            const int g = n >> 3, L = (n & 7) * 4 + t;
+            unsigned* dst = reinterpret_cast<unsigned*>(S.bfr + (static_cast<size_t>(ul) * NG + g) * 64 + L * 2) + 2 * b + r;
+            *dst = __byte_perm(__byte_perm(d[k][0], d[k][1], 0x0040), __byte_perm(d[k][2], d[k][3], 0x0040), 0x5410);
+          }
+        }
+        // the 32 lanes of a warp share one (unit, batch row)
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) vs += __shfl_xor_sync(0xffffffffu, vs, o);
+        if (lane == 0 && lsm >= 0) atomicAdd(S.vsum + lsm, static_cast<unsigned long long>(static_cast<long long>(vs)));
+      }
+    }
+    __syncthreads();  // B fragments and sums complete
+    if (ph == 0) asm volatile("griddepcontrol.launch_dependents;");
+
+    // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v, read
+    // by the drains below
+    if (threadIdx.x < nls * kMaxSlots) {
+      const int ls = threadIdx.x / kMaxSlots, n = threadIdx.x - ls * kMaxSlots;
+      const int m = n / 3, dg = n - 3 * m;
+      float f1 = 0.f, f2 = 0.f;
+      if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
+      S.wsl[threadIdx.x] = f1 * f2;  // powers of two: the product is exact
+    } else if (threadIdx.x - nls * kMaxSlots < nls * MB) {
+      const int i = threadIdx.x - nls * kMaxSlots;
+      float f1, f2;
+      pow2_pair(-fixed_shift(__uint_as_float(S.xmax[i])), f1, f2);
+      S.ssf[i] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[i]))) * f1) * f2;
+    }
+    __syncthreads();
+
+    // ---- MMA loop over this warp's contiguous range of (row block, unit) items: per row
+    //      block, runs of units of one segment; inside a run the operands of the next unit
+    //      are loaded while the current unit's MMAs issue (two register sets, ping-pong).
+    //      When a warp has finished a row block it pushes the block's row partial sums
+    //      to the CTA that owns the rows (distributed shared memory) ----
+    const int nb = nt * BPT;
+    const int items = nb * nun;
+    const int i0 = warp * items / kIW, i1 = (warp + 1) * items / kIW;
+    const bool skip_phase = reads_z && S.flags[1] != 0;  // z never became ready
+    if (!skip_phase) {
+      int acc[RH][NG][4][4];
 #pragma unroll
       for (int h = 0; h < RH; ++h)
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+        for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int m = 0; m < MB; ++m) pacc[h][r][m] = 0.f;
-      int ur = ua;
-      while (ur < ub) {
-        const int ls = S.useg[ur];
-        const int ue = min(ub, S.lsend[ls]);
-        if (S.lsbits[ls] && tile_ok) {
-          auto load_b = [&](int ul, unsigned (&B)[NG][8]) {
+          for (int b = 0; b < 4; ++b)
 #pragma unroll
-            for (int g = 0; g < NG; ++g) {
-              if (8 * g + g8 < 3 * MB) {
-                const uint4* src = bbase + (static_cast<size_t>(ul) * NG + g) * 64;
-                const uint4 q0 = src[0], q1 = src[1];
-                B[g][0] = q0.x; B[g][1] = q0.y; B[g][2] = q0.z; B[g][3] = q0.w;
-                B[g][4] = q1.x; B[g][5] = q1.y; B[g][6] = q1.z; B[g][7] = q1.w;
-              } else {
+            for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
+      int cur_tile = -1;
+      bool tile_ok = true;
+      int it = i0;
+      while (it < i1) {
+        const int bl = it / nun;
+        const int tl = bl / BPT;
+        const int ua = pa + (it - bl * nun);
+        const int ub = pa + min(nun, i1 - bl * nun);  // this warp's units of block bl: [ua, ub)
+        if (tl != cur_tile) {
+          cur_tile = tl;
+          tile_ok = dev::mbar_wait(S.bar + tl, 0u, wait_ns);
+          if (!tile_ok) ok = false;
+        }
+        const unsigned* wbase = reinterpret_cast<const unsigned*>(S.ring + static_cast<size_t>(tl) * nu * 512) +
+                                ((bl % BPT) * RB + g8) * 4 + tq;
+        const uint4* bbase = S.bfr + lane * 2;
+        float pacc[RH][2][MB];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) B[g][k] = 0u;
+        for (int h = 0; h < RH; ++h)
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int m = 0; m < MB; ++m) pacc[h][r][m] = 0.f;
+        int ur = ua;
+        while (ur < ub) {
+          const int ls = S.useg[ur];
+          const int ue = min(ub, S.lsend[ls]);
+          if (S.lsbits[ls] && tile_ok) {
+            auto load_b = [&](int ul, unsigned (&B)[NG][8]) {
+#pragma unroll
+              for (int g = 0; g < NG; ++g) {
+                if (8 * g + g8 < 3 * MB) {
+                  const uint4* src = bbase + (static_cast<size_t>(ul) * NG + g) * 64;
+                  const uint4 q0 = src[0], q1 = src[1];
+                  B[g][0] = q0.x; B[g][1] = q0.y; B[g][2] = q0.z; B[g][3] = q0.w;
+                  B[g][4] = q1.x; B[g][5] = q1.y; B[g][6] = q1.z; B[g][7] = q1.w;
+                } else {
+#pragma unroll
+                  for (int k = 0; k < 8; ++k) B[g][k] = 0u;
+                }
+              }
+            };
+            auto load_w = [&](int ul, unsigned (&wv)[2 * RH]) {
+              const unsigned* ws = wbase + ul * 128;
+#pragma unroll
+              for (int k = 0; k < 2 * RH; ++k) wv[k] = ws[k * 32];
+            };
+            auto mma_unit = [&](const unsigned (&B)[NG][8], const unsigned (&wv)[2 * RH]) {
+#pragma unroll
+              for (int h = 0; h < RH; ++h) {
+                const unsigned w0 = wv[2 * h], w1 = wv[2 * h + 1];
+                const unsigned s0 = w0 >> 4, s1 = w1 >> 4;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                  const unsigned mk = kByteMask << b;
+                  const unsigned a0 = w0 & mk, a1 = w1 & mk, a2 = s0 & mk, a3 = s1 & mk;
+#pragma unroll
+                  for (int g = 0; g < NG; ++g) mma_s8s8(acc[h][g][b], a0, a1, a2, a3, B[g][2 * b], B[g][2 * b + 1]);
+                }
+              }
+            };
+            if constexpr (NG <= 2) {
+              unsigned B0[NG][8], B1[NG][8], W0[2 * RH], W1[2 * RH];
+              load_b(ur, B0);
+              load_w(ur, W0);
+              int ul = ur;
+              for (; ul + 1 < ue; ul += 2) {
+                load_b(ul + 1, B1);
+                load_w(ul + 1, W1);
+                mma_unit(B0, W0);
+                if (ul + 2 < ue) {
+                  load_b(ul + 2, B0);
+                  load_w(ul + 2, W0);
+                }
+                mma_unit(B1, W1);
+              }
+              if (ul < ue) mma_unit(B0, W0);
+            } else {  // three slot groups: registers allow only the sign words to run ahead
+              unsigned B0[NG][8], W0[2 * RH], W1[2 * RH];
+              load_w(ur, W0);
+              int ul = ur;
+              for (; ul + 1 < ue; ul += 2) {
+                load_w(ul + 1, W1);
+                load_b(ul, B0);
+                mma_unit(B0, W0);
+                if (ul + 2 < ue) load_w(ul + 2, W0);
+                load_b(ul + 1, B0);
+                mma_unit(B0, W1);
+              }
+              if (ul < ue) {
+                load_b(ul, B0);
+                mma_unit(B0, W0);
               }
             }
-          };
-          auto load_w = [&](int ul, unsigned (&wv)[2 * RH]) {
-            const unsigned* ws = wbase + ul * 128;
+            // drain: D = sum_b (acc_b >> b) per slot, times the slot weight, summed over the
+            // slots of each batch row (the four lanes of a quad), times the row scale; the run
+            // that starts the CTA's range of the segment also subtracts r * sum_i v_i
+            float wlo[NG][2];
 #pragma unroll
-            for (int k = 0; k < 2 * RH; ++k) wv[k] = ws[k * 32];
-          };
-          auto mma_unit = [&](const unsigned (&B)[NG][8], const unsigned (&wv)[2 * RH]) {
+            for (int g = 0; g < NG; ++g) {
+              const float2 wf = reinterpret_cast<const float2*>(S.wsl)[(ls * kMaxSlots + 8 * g + 2 * tq) >> 1];
+              wlo[g][0] = wf.x;
+              wlo[g][1] = wf.y;
+            }
+            const bool first_run = ur == S.lsstart[ls];
 #pragma unroll
             for (int h = 0; h < RH; ++h) {
-              const unsigned w0 = wv[2 * h], w1 = wv[2 * h + 1];
-              const unsigned s0 = w0 >> 4, s1 = w1 >> 4;
+              float cv[2][MB];
 #pragma unroll
-              for (int b = 0; b < 4; ++b) {
-                const unsigned mk = kByteMask << b;
-                const unsigned a0 = w0 & mk, a1 = w1 & mk, a2 = s0 & mk, a3 = s1 & mk;
+              for (int r = 0; r < 2; ++r)
 #pragma unroll
-                for (int g = 0; g < NG; ++g) mma_s8s8(acc[h][g][b], a0, a1, a2, a3, B[g][2 * b], B[g][2 * b + 1]);
+                for (int m = 0; m < MB; ++m) cv[r][m] = 0.f;
+#pragma unroll
+              for (int g = 0; g < NG; ++g) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int n = 8 * g + 2 * tq + (j & 1);
+                  const int D = acc[h][g][0][j] + (acc[h][g][1][j] >> 1) + (acc[h][g][2][j] >> 2) + (acc[h][g][3][j] >> 3);
+                  const float val = static_cast<float>(D) * wlo[g][j & 1];
+                  const int m = n / 3;
+#pragma unroll
+                  for (int mm = 0; mm < MB; ++mm) cv[j >> 1][mm] += (m == mm) ? val : 0.f;
+                }
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
               }
-            }
-          };
-          if constexpr (NG <= 2) {
-            unsigned B0[NG][8], B1[NG][8], W0[2 * RH], W1[2 * RH];
-            load_b(ur, B0);
-            load_w(ur, W0);
-            int ul = ur;
-            for (; ul + 1 < ue; ul += 2) {
-              load_b(ul + 1, B1);
-              load_w(ul + 1, W1);
-              mma_unit(B0, W0);
-              if (ul + 2 < ue) {
-                load_b(ul + 2, B0);
-                load_w(ul + 2, W0);
+#pragma unroll
+              for (int r = 0; r < 2; ++r) {
+                const int row = (bl % BPT) * RB + 16 * h + g8 + 8 * r;  // row within the tile
+                const float rs = S.rsc[ls * p.max_tiles * 32 + tl * 32 + row];
+#pragma unroll
+                for (int mm = 0; mm < MB; ++mm) {
+                  float v = cv[r][mm];
+                  v += __shfl_xor_sync(0xffffffffu, v, 1);
+                  v += __shfl_xor_sync(0xffffffffu, v, 2);
+                  if (first_run) v -= S.ssf[ls * MB + mm];
+                  pacc[h][r][mm] = fmaf(v, rs, pacc[h][r][mm]);
+                }
               }
-              mma_unit(B1, W1);
-            }
-            if (ul < ue) mma_unit(B0, W0);
-          } else {  // three slot groups: registers allow only the sign words to run ahead
-            unsigned B0[NG][8], W0[2 * RH], W1[2 * RH];
-            load_w(ur, W0);
-            int ul = ur;
-            for (; ul + 1 < ue; ul += 2) {
-              load_w(ul + 1, W1);
-              load_b(ul, B0);
-              mma_unit(B0, W0);
-              if (ul + 2 < ue) load_w(ul + 2, W0);
-              load_b(ul + 1, B0);
-              mma_unit(B0, W1);
-            }
-            if (ul < ue) {
-              load_b(ul, B0);
-              mma_unit(B0, W0);
             }
           }
-          // drain: D = sum_b (acc_b >> b) per slot, times the slot weight, summed over the
-          // slots of each batch row (the four lanes of a quad), times the row scale; the run
-          // that starts the CTA's range of the segment also subtracts r * sum_i v_i
-          float wlo[NG][2];
+          ur = ue;
+        }
+        // push the block's row partial sums to the CTA that owns the rows, one store per
+        // lane: after the quad reduction every lane of a quad holds the same sums, so lane
+        // tq takes one (half, row) pair (32-row blocks) or one row and half the batch rows
+        // (16-row blocks). Slot c = this warp's index among the consecutive warps whose
+        // item ranges touch block bl, in this phase's set of slots.
+        if (!waited) {  // peers must be running and have zeroed their buffers
+          cluster.barrier_wait(std::move(started));
+          waited = true;
+        }
+        int wfirst = warp;
+        while (wfirst > 0 && ((wfirst) * items / kIW) > bl * nun) --wfirst;
+        const int c = ph * kcp + (warp - wfirst);
+        {
+          constexpr int VPL = RH == 2 ? MB : MB / 2;  // values per lane
+          const int hh = RH == 2 ? (tq >> 1) : 0;
+          const int rr = tq & 1;
+          const int m0 = RH == 2 ? 0 : (tq >> 1) * (MB / 2);
+          float v[VPL];
 #pragma unroll
-          for (int g = 0; g < NG; ++g) {
-            const float2 wf = reinterpret_cast<const float2*>(S.wsl)[(ls * kMaxSlots + 8 * g + 2 * tq) >> 1];
-            wlo[g][0] = wf.x;
-            wlo[g][1] = wf.y;
+          for (int e = 0; e < VPL; ++e) {
+            if constexpr (RH == 2) {  // (hh, rr) from tq; all MB values
+              const float lo = rr ? pacc[0][1][e] : pacc[0][0][e];
+              const float hi = rr ? pacc[RH - 1][1][e] : pacc[RH - 1][0][e];
+              v[e] = hh ? hi : lo;
+            } else {  // rr from tq, batch rows e or MB/2 + e
+              const float a = rr ? pacc[0][1][e] : pacc[0][0][e];
+              const float b = rr ? pacc[0][1][(MB / 2 + e) % MB] : pacc[0][0][(MB / 2 + e) % MB];
+              v[e] = (tq >> 1) ? b : a;
+            }
           }
-          const bool first_run = ur == S.lsstart[ls];
+          const int lr = bl * RB + 16 * hh + g8 + 8 * rr;  // row within the cluster's rows
+          const int dst = share_owner_i(lr, rows_c, p.C);
+          float* rp = cluster.map_shared_rank(S.recv, dst) +
+                      ((static_cast<size_t>(rank) * kc + c) * msh + (lr - share_begin_i(dst, rows_c, p.C))) * MB + m0;
+          if constexpr (VPL == 1) {
+            rp[0] = v[0];
+          } else if constexpr (VPL == 2) {
+            *reinterpret_cast<float2*>(rp) = make_float2(v[0], v[1]);
+          } else {
 #pragma unroll
-          for (int h = 0; h < RH; ++h) {
-            float cv[2][MB];
-#pragma unroll
-            for (int r = 0; r < 2; ++r)
-#pragma unroll
-              for (int m = 0; m < MB; ++m) cv[r][m] = 0.f;
-#pragma unroll
-            for (int g = 0; g < NG; ++g) {
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int n = 8 * g + 2 * tq + (j & 1);
-                const int D = acc[h][g][0][j] + (acc[h][g][1][j] >> 1) + (acc[h][g][2][j] >> 2) + (acc[h][g][3][j] >> 3);
-                const float val = static_cast<float>(D) * wlo[g][j & 1];
-                const int m = n / 3;
-#pragma unroll
-                for (int mm = 0; mm < MB; ++mm) cv[j >> 1][mm] += (m == mm) ? val : 0.f;
-              }
-#pragma unroll
-              for (int b = 0; b < 4; ++b)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[h][g][b][j] = 0;
-            }
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int row = (bl % BPT) * RB + 16 * h + g8 + 8 * r;  // row within the tile
-              const float rs = S.rsc[ls * p.max_tiles * 32 + tl * 32 + row];
-#pragma unroll
-              for (int mm = 0; mm < MB; ++mm) {
-                float v = cv[r][mm];
-                v += __shfl_xor_sync(0xffffffffu, v, 1);
-                v += __shfl_xor_sync(0xffffffffu, v, 2);
-                if (first_run) v -= S.ssf[ls * MB + mm];
-                pacc[h][r][mm] = fmaf(v, rs, pacc[h][r][mm]);
-              }
-            }
+            for (int e = 0; e < VPL; e += 4) *reinterpret_cast<float4*>(rp + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
           }
         }
-        ur = ue;
+        it = bl * nun + (ub - pa);
       }
-      // push the block's row partial sums to the CTA that owns the rows, one store per
-      // lane: after the quad reduction every lane of a quad holds the same sums, so lane tq
-      // takes one (half, row) pair (32-row blocks) or one row and half the batch rows
-      // (16-row blocks). Slot c = this warp's index among the consecutive warps whose item
-      // ranges touch block bl.
-      if (!waited) {  // peers must be running and have zeroed their buffers
-        cluster.barrier_wait(std::move(started));
-        waited = true;
-      }
-      int wfirst = warp;
-      while (wfirst > 0 && ((wfirst) * items / kIW) > bl * nu) --wfirst;
-      const int c = warp - wfirst;
-      {
-        constexpr int VPL = RH == 2 ? MB : MB / 2;  // values per lane
-        const int hh = RH == 2 ? (tq >> 1) : 0;
-        const int rr = tq & 1;
-        const int m0 = RH == 2 ? 0 : (tq >> 1) * (MB / 2);
-        float v[VPL];
-#pragma unroll
-        for (int e = 0; e < VPL; ++e) {
-          if constexpr (RH == 2) {  // (hh, rr) from tq; all MB values
-            const float lo = rr ? pacc[0][1][e] : pacc[0][0][e];
-            const float hi = rr ? pacc[RH - 1][1][e] : pacc[RH - 1][0][e];
-            v[e] = hh ? hi : lo;
-          } else {  // rr from tq, batch rows e or MB/2 + e
-            const float a = rr ? pacc[0][1][e] : pacc[0][0][e];
-            const float b = rr ? pacc[0][1][(MB / 2 + e) % MB] : pacc[0][0][(MB / 2 + e) % MB];
-            v[e] = (tq >> 1) ? b : a;
-          }
-        }
-        const int lr = bl * RB + 16 * hh + g8 + 8 * rr;  // row within the cluster's rows
-        const int dst = share_owner_i(lr, rows_c, p.C);
-        float* rp = cluster.map_shared_rank(S.recv, dst) +
-                    ((static_cast<size_t>(rank) * nbw + c) * msh + (lr - share_begin_i(dst, rows_c, p.C))) * MB + m0;
-        if constexpr (VPL == 1) {
-          rp[0] = v[0];
-        } else if constexpr (VPL == 2) {
-          *reinterpret_cast<float2*>(rp) = make_float2(v[0], v[1]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < VPL; e += 4) *reinterpret_cast<float4*>(rp + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-        }
-      }
-      it = bl * nu + ub;
     }
   }
   if (!ok) {
@@ -648,7 +699,7 @@ __global__ void __launch_bounds__(kIT, 2)
     float sum[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) sum[m] = 0.f;
-    for (int src = 0; src < p.C * nbw; ++src) {  // (rank, contributor slot), fixed order
+    for (int src = 0; src < p.C * kc; ++src) {  // (rank, contributor slot), fixed order
 #pragma unroll
       for (int m = 0; m < MB; ++m) sum[m] += S.recv[(static_cast<size_t>(src) * msh + sr) * MB + m];
     }
@@ -678,6 +729,22 @@ __global__ void __launch_bounds__(kIT, 2)
       }
     }
   }
+  if (fused) {
+    __syncthreads();  // this CTA's stores (z for the producers) are issued
+    if (threadIdx.x == 0) {
+      if (role_z) {
+        __threadfence();  // z visible device-wide before it is counted
+        atomicAdd(z_ready, 1);
+      }
+      // the last CTA of the grid to get here resets both counters for the next launch:
+      // every consumer counted itself after its wait, so nobody reads them any more
+      const int total = gridDim.x;
+      if (atomicAdd(z_done, 1) == total - 1) {
+        atomicExch(z_ready, 0);
+        atomicExch(z_done, 0);
+      }
+    }
+  }
 }
 
 template <int MB>
@@ -694,7 +761,8 @@ int imma_clusters(int C, size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, imma_gemv_kernel<MB>, &cfg) != cudaSuccess) {
+  // both variants are compiled for two CTAs of kIT threads per SM: same residency
+  if (cudaOccupancyMaxActiveClusters(&n, imma_gemv_kernel<MB, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -728,8 +796,11 @@ int max_segments_per_cta_i(int units, int C, const int* seg_unit0, int nseg) {
 
 template <int MB>
 cudaError_t imma_set_attrs(size_t lim) {
-  cudaError_t e = cudaFuncSetAttribute(imma_gemv_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(imma_gemv_kernel<MB, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(lim));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(imma_gemv_kernel<MB, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(lim));
   return e;
 }
 
@@ -757,15 +828,17 @@ cudaError_t imma_ensure_attrs() {
 // slots; a legacy m16n8k32 MMA holds its sub-partition's issue for about 10 cycles and
 // the masks add about half as much again: measured 237 cycles per 32 x 128 block and
 // warp with 8 warps per SM), the B-fragment writes (about 60 lane operations per task of
-// 4 columns and one batch row, 64 lanes per clock for one CTA), and a fixed cost for the
-// cluster reduction, plus a fixed cost when the CTA takes more than half of the SM's
-// shared memory (the next kernel's CTA then cannot be resident beside it) -- among the
-// plans whose shared memory fits. The grid holds as many CTAs as fit one per SM; with
-// half an SM or less per CTA the block scheduler still places two CTAs of one launch on
-// some SMs (measured: 120 CTAs on 98 SMs), which those SMs pay for, but exposing the next
-// kernel's prologue costs more.
+// 4 columns and one batch row, 64 lanes per clock for one CTA), a fixed cost for the
+// cluster reduction (and for the second phase of a fused launch), plus a fixed cost when
+// the CTA takes more than half of the SM's shared memory (the next kernel's CTA then
+// cannot be resident beside it) -- among the plans whose shared memory fits. The grid
+// holds as many clusters as fit with one CTA per SM; with half an SM or less per CTA the
+// block scheduler still places two CTAs of one launch on some SMs (measured: 120 CTAs on
+// 98 SMs), which those SMs pay for, but exposing the next kernel's prologue costs more.
+// With z given (the correction fused into one launch) the clusters are split between
+// the z pass and pass y in proportion to their work.
 // C = 0 in the result means no plan fits.
-ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, size_t smem_limit) {
+ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sal, size_t smem_limit) {
   ImmaPlan best{};
   if (imma_ensure_attrs() != cudaSuccess) return best;
   int dev = 0, per_sm = 0;
@@ -774,57 +847,78 @@ ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int
   // two CTAs per SM: each gets half of the SM's shared memory less the 1 KB the
   // hardware reserves per CTA
   const size_t half = per_sm > 0 ? static_cast<size_t>(per_sm) / 2 - 1024 : smem_limit / 2;
-  const int tiles = (rows + 31) / 32;
   const int NG = groups_of(MB), RB = block_rows(MB);
+  const int tiles_y = (y.rows + 31) / 32;
+  const int tiles_z = z ? (z->rows + 31) / 32 : 0;
   double best_cost = -1;
   for (int C = 1; C <= kMaxCluster; C *= 2) {
-    if (C > 1 && C > units) break;
-    const int max_units = (units + C - 1) / C;
-    const int max_lseg = max_segments_per_cta_i(units, C, seg_unit0, nseg);
+    if (C > 1 && (C > y.units || (z && C > z->units))) break;
     // clusters that fit with one CTA of the launch per SM (the query asks for more
     // than half of the SM's shared memory)
     const size_t force = smem_limit / 2 + 1024;
-    int fit = imma_clusters_mb(MB, C, force);
-    if (fit <= 0) continue;
-    const int ncl = std::max(1, std::min(tiles, fit));
-    const int max_tiles = (tiles + ncl - 1) / ncl;
-    // contributor slots per row: warps own equal contiguous ranges of (row block, unit)
-    // items, so with at least kIW row blocks in every CTA a block is touched by at most
-    // two warps; otherwise by at most kIW
-    const int nb_min = (tiles / ncl) * (32 / RB);
-    const int nbw = nb_min >= kIW ? 2 : kIW;
-    const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, nbw, n_sal);
-    if (need > smem_limit) continue;
-    // kIW warps of a CTA work on kIW blocks at once: 237 / kIW cycles per block and SM
-    const double mma = static_cast<double>(max_tiles) * max_units * NG * 237.0 / kIW;
-    const double bfr = static_cast<double>(max_units) * MB * 32.0 * 60.0 / 64.0;
-    const double red = C > 1 ? 1500.0 : 300.0;
-    // a CTA of at most half an SM lets the next kernel's CTA (launched early) be resident
-    // beside it and run its prologue during this kernel; a larger one exposes that
-    // prologue (measured on the 4096 x 4096 layer: 6.85 us vs 8.08 us per GEMV)
-    const bool coresident = need <= half;
-    const double cost = mma + bfr + red + (coresident ? 0.0 : 2500.0);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best.C = C;
-      best.ncl = ncl;
-      best.max_tiles = max_tiles;
-      best.max_units = max_units;
-      best.max_lseg = max_lseg;
-      best.nbw = nbw;
-      best.MB = MB;
-      best.smem = coresident ? need : std::max(need, force);
+    const int fit = imma_clusters_mb(MB, C, force);
+    if (fit <= 0 || (z && fit < 2)) continue;
+    // z clusters: from the share proportional to the work upwards (a few more z
+    // clusters shrink the largest tile count, and with it shared memory)
+    int nz0 = 0, nz1 = 0;
+    if (z) {
+      const double wz = static_cast<double>(tiles_z) * z->units, wy = static_cast<double>(tiles_y) * y.units;
+      nz0 = std::max(1, std::min({static_cast<int>(fit * wz / (wz + wy) + 0.5), tiles_z, fit - 1}));
+      nz1 = std::min({nz0 + 8, tiles_z, fit - 1});
+    }
+    for (int ncl_z = nz0; ncl_z <= nz1; ++ncl_z) {
+      const int ncl_y = std::max(1, std::min(tiles_y, fit - ncl_z));
+      const int mt_y = (tiles_y + ncl_y - 1) / ncl_y;
+      const int mu_y = (y.units + C - 1) / C;
+      const int mt_z = z ? (tiles_z + ncl_z - 1) / ncl_z : 0;
+      const int mu_z = z ? (z->units + C - 1) / C : 0;
+      const int max_tiles = std::max(mt_y, mt_z);
+      const int max_units = std::max(mu_y, mu_z);
+      const int max_lseg = std::max(max_segments_per_cta_i(y.units, C, y.seg_unit0, y.nseg),
+                                    z ? max_segments_per_cta_i(z->units, C, z->seg_unit0, z->nseg) : 1);
+      // contributor slots per row and phase: warps own equal contiguous ranges of (row
+      // block, unit) items, so with at least kIW row blocks in every CTA a block is
+      // touched by at most two warps; otherwise by at most kIW. A fused launch has two
+      // phases.
+      int nb_min = (tiles_y / ncl_y) * (32 / RB);
+      if (z) nb_min = std::min(nb_min, (tiles_z / ncl_z) * (32 / RB));
+      const int kc = (nb_min >= kIW ? 2 : kIW) * (z ? 2 : 1);
+      const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, kc, n_sal);
+      if (need > smem_limit) continue;
+      // kIW warps of a CTA work on kIW blocks at once: 237 / kIW cycles per block and SM
+      const double mma =
+          std::max(static_cast<double>(mt_y) * mu_y, static_cast<double>(mt_z) * mu_z) * NG * 237.0 / kIW;
+      const double bfr = static_cast<double>(max_units) * MB * 32.0 * 60.0 / 64.0;
+      const double red = (C > 1 ? 1500.0 : 300.0) + (z ? 1500.0 : 0.0);
+      // a CTA of at most half an SM lets the next kernel's CTA (launched early) be
+      // resident beside it and run its prologue during this kernel; a larger one exposes
+      // that prologue (measured on the 4096 x 4096 layer: 6.85 us vs 8.08 us per GEMV)
+      const bool coresident = need <= half;
+      const double cost = mma + bfr + red + (coresident ? 0.0 : 2500.0);
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best.C = C;
+        best.ncl = ncl_y;
+        best.ncl_z = ncl_z;
+        best.max_tiles = max_tiles;
+        best.max_units = max_units;
+        best.max_lseg = max_lseg;
+        best.nbw = kc;
+        best.MB = MB;
+        best.smem = coresident ? need : std::max(need, force);
+      }
     }
   }
   return best;
 }
 
-cudaError_t launch_imma(const PassParam& p, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
+cudaError_t launch_imma(const PassParam* pz, const PassParam& py, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
                         const ImmaDebug* dbg) {
   const cudaError_t e = imma_ensure_attrs();
   if (e != cudaSuccess) return e;
+  const int ncl_z = pz ? plan.ncl_z : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(plan.ncl * plan.C);
+  cfg.gridDim = dim3((plan.ncl + ncl_z) * plan.C);
   cfg.blockDim = dim3(kIT);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = stream;
@@ -839,11 +933,20 @@ cudaError_t launch_imma(const PassParam& p, const ImmaPlan& plan, cudaStream_t s
   cfg.numAttrs = pdl ? 2 : 1;
   const int skip = dbg ? dbg->skip_tile : -1;
   const unsigned long long wait_ns = dbg && dbg->wait_ns ? dbg->wait_ns : kDefaultWaitNs;
+  const PassParam& z = pz ? *pz : py;
   switch (plan.MB) {
-    case 1: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1>, p, plan.nbw, skip, wait_ns);
-    case 2: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2>, p, plan.nbw, skip, wait_ns);
-    case 4: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4>, p, plan.nbw, skip, wait_ns);
-    case 8: return cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8>, p, plan.nbw, skip, wait_ns);
+    case 1:
+      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
+                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, false>, z, py, 0, plan.nbw, skip, wait_ns);
+    case 2:
+      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
+                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, false>, z, py, 0, plan.nbw, skip, wait_ns);
+    case 4:
+      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
+                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, false>, z, py, 0, plan.nbw, skip, wait_ns);
+    case 8:
+      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
+                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, false>, z, py, 0, plan.nbw, skip, wait_ns);
     default: return cudaErrorInvalidValue;
   }
 }

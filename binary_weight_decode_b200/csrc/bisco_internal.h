@@ -87,7 +87,8 @@ size_t query_smem_limit();
 
 // Integer tensor-core GEMV (mma.sync u8 x s8) for batch chunks of up to 8 rows.
 struct ImmaPlan {
-  int C, ncl;            // cluster size (K split) and clusters; C == 0: no plan fits
+  int C, ncl;            // cluster size (K split) and clusters of the output pass; C == 0: no plan fits
+  int ncl_z;             // clusters of the z pass in a fused launch (0: not fused)
   int max_tiles;         // 32-row tiles of the largest cluster share
   int max_units;         // 128-column units of the largest CTA share
   int max_lseg;          // segments a CTA's unit range touches, at most
@@ -104,8 +105,19 @@ struct ImmaDebug {
   unsigned long long wait_ns;
 };
 constexpr unsigned long long kDefaultWaitNs = 200000000ull;  // bound on every mbarrier wait (200 ms)
-ImmaPlan make_imma_plan(int rows, int units, const int* seg_unit0, int nseg, int MB, int n_sal, size_t smem_limit);
-cudaError_t launch_imma(const PassParam& p, const ImmaPlan& plan, cudaStream_t stream, bool pdl, const ImmaDebug* dbg);
+// Rows and the 128-column units of a pass, with the first unit of each segment.
+struct ImmaShape {
+  int rows, units;
+  const int* seg_unit0;
+  int nseg;
+};
+// z == nullptr: a plan for one pass; otherwise for the z pass and pass y fused into one
+// launch (pass y's z-reading units run after a bounded wait for the z pass).
+ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sal, size_t smem_limit);
+// pz == nullptr: one pass (py); otherwise the fused launch of plan.ncl_z z clusters and
+// plan.ncl output clusters.
+cudaError_t launch_imma(const PassParam* pz, const PassParam& py, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
+                        const ImmaDebug* dbg);
 cudaError_t imma_ensure_attrs();
 
 // Tensor-core path (32..128 batch rows per launch): one launch per pass.

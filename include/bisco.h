@@ -113,6 +113,8 @@ bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* b
 
 /*
  * Prepare a workspace for first use: zero-fills ws_bytes bytes on `stream`.
+ * The workspace holds the device status word, counters that a launch computing z and
+ * y together uses to hand z over (each such launch returns them to zero), and z.
  * Every bisco_gemv call leaves the workspace ready for the next call, so this is
  * needed once per buffer (and again after a call reported an error).
  */
@@ -145,8 +147,9 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  * Which kernel family runs a batch chunk (process-wide; for tests and diagnostics).
  *  BISCO_PATH_AUTO (default): chunks of 32..128 rows on the tcgen05 tensor-core kernel
  *    (bf16 scales), chunks of 2..8 rows on the integer tensor-core kernel (mma.sync)
- *    when its shared-memory plan fits, single rows and the rest on the lookup-table
- *    kernels.
+ *    when its shared-memory plan fits, single rows of a layer with a correction on the
+ *    integer kernel's one-launch form, other single rows and the rest on the
+ *    lookup-table kernels.
  *  BISCO_PATH_LOOKUP_TABLE: as AUTO, but chunks of up to 8 rows always take the
  *    lookup-table kernels (FluxBin Sec. 3.2, Stages 1-3, restated for B200).
  *  BISCO_PATH_SMALL_BATCH_ONLY: as AUTO, but every chunk has at most 8 rows (no
@@ -164,7 +167,8 @@ enum {
   BISCO_KERNEL_LUT_WARP = 1,      /* lookup tables, 16-warp CTAs, <= 2 batch rows        */
   BISCO_KERNEL_LUT_STREAM = 2,    /* lookup tables, bulk-copy sign stream, <= 2 rows     */
   BISCO_KERNEL_LUT_ROWS = 3,      /* lookup tables, warps own row tiles, 4 or 8 rows     */
-  BISCO_KERNEL_INTEGER_MMA = 4,   /* int8 tensor cores (mma.sync), <= 8 rows             */
+  BISCO_KERNEL_INTEGER_MMA = 4,   /* int8 tensor cores (mma.sync), <= 8 rows; with a
+                                     correction, z and y in one launch                   */
   BISCO_KERNEL_TENSOR_CORE = 5    /* tcgen05 tensor cores, 32..128 rows                  */
 };
 

@@ -46,8 +46,9 @@ def test_kernel_choice(policy):
     assert kinds(L, 2) == [bw.BISCO_KERNEL_INTEGER_MMA]
     assert kinds(L, 8) == [bw.BISCO_KERNEL_INTEGER_MMA]
     assert kinds(L, 128) == [bw.BISCO_KERNEL_TENSOR_CORE]
-    L4, _ = build(4, 0, 2)  # correction: pass Z then pass Y
-    assert kinds(L4, 2) == [bw.BISCO_KERNEL_INTEGER_MMA] * 2
+    L4, _ = build(4, 0, 2)  # correction: z and y in one integer launch, single rows too
+    for M in (1, 2, 4, 8):
+        assert kinds(L4, M) == [bw.BISCO_KERNEL_INTEGER_MMA]
     policy(bw.BISCO_PATH_LOOKUP_TABLE)
     assert kinds(L, 1) == [bw.BISCO_KERNEL_LUT_WARP]
     assert kinds(L, 8) == [bw.BISCO_KERNEL_LUT_ROWS]
@@ -156,7 +157,7 @@ def test_integer_kernel_keeps_relative_precision_at_any_magnitude(scale_exp):
     M, out, in_ = 3, 200, 700
     X = make_activations(0, (820,), M, in_, "f32") * np.float32(2.0 ** scale_exp)
     L = make_layer(0, (820,), out, in_, 2, "f32", rank=24)
-    assert kinds(L, M, "f32") == [bw.BISCO_KERNEL_INTEGER_MMA] * 2
+    assert kinds(L, M, "f32") == [bw.BISCO_KERNEL_INTEGER_MMA]
     check(run(L, X, "f32", "f32"), oracle.gemv(L, X, "f32"), X, "f32", "f32")
 
 
@@ -208,6 +209,69 @@ def test_integer_kernel_wait_gives_up_and_reports_timeout():
     assert bw.bisco_sync_status(ws) == bw.BISCO_OK
     Y = Yd.cpu().numpy().astype(np.float64)
     check(Y, oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
+
+
+# ---- the correction in one launch: z handed over inside the grid ------------------
+
+@pytest.mark.parametrize("out,in_,K,rank", [(200, 128, 1, 512), (64, 4096, 2, 64), (4100, 300, 2, 1000),
+                                            (96, 256, 0, 40), (1000, 1000, 3, 7)],
+                         ids=["rank_heavy", "wide", "ragged", "correction_only", "rank7"])
+@pytest.mark.parametrize("M", [1, 2, 8])
+def test_fused_correction_launch(policy, out, in_, K, rank, M):
+    # z = alpha (.) (V x) computed by the first clusters of the grid and read by the U^T
+    # units of the others; shapes where a CTA holds only U^T units, only base units, or
+    # both, and ragged row and column counts
+    policy(bw.BISCO_PATH_INTEGER_MMA)
+    X = make_activations(0, (824, out, M), M, in_, "bf16")
+    L = make_layer(0, (824, out, in_, K), out, in_, K, "bf16", rank=rank, sal_frac=0.01, x_for_salience=X,
+                   x_dtype="bf16")
+    assert kinds(L, M) == [bw.BISCO_KERNEL_INTEGER_MMA]
+    check(run(L, X, "bf16", "f32"), oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
+
+
+def test_fused_correction_repeated_calls_are_identical():
+    # the hand-over counters return to zero at the end of every launch: back-to-back
+    # calls on one workspace, without re-initialising it, give bit-identical results
+    L, X = build(4, 0, 4)
+    dl = bw.DeviceLayer(L)
+    assert kinds(L, 4) == [bw.BISCO_KERNEL_INTEGER_MMA]
+    ws = bw.alloc_workspace([dl], 4)
+    Xd = to_dev_x(X, "bf16")
+    outs = []
+    for _ in range(4):
+        Yd = torch.empty((4, L.out), dtype=torch.float32, device="cuda")
+        bw.bisco_gemv(dl, Xd, Yd, ws)
+        outs.append(Yd)
+    assert bw.bisco_sync_status(ws) == bw.BISCO_OK
+    # the two hand-over counters: 32-bit words 32 and 33 of the status region
+    assert int(ws[128:136].to(torch.int32).sum()) == 0
+    for Yd in outs[1:]:
+        assert torch.equal(Yd, outs[0])
+    rows = sample_rows(L.out, 128, 5)
+    check(outs[0].cpu().numpy().astype(np.float64)[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
+
+
+def test_fused_correction_wait_gives_up_and_reports_timeout():
+    # with one tile's copies unissued in every CTA, the z producers give up on their
+    # tile and the output CTAs on z; both record BISCO_ERR_TIMEOUT, the counters are
+    # still returned to zero, and the next call after bisco_workspace_init is correct
+    L, X = build(4, 0, 2)
+    dl = bw.DeviceLayer(L)
+    assert kinds(L, 2) == [bw.BISCO_KERNEL_INTEGER_MMA]
+    ws = bw.alloc_workspace([dl], 2)
+    Xd = to_dev_x(X, "bf16")
+    Yd = torch.empty((2, L.out), dtype=torch.float32, device="cuda")
+    try:
+        bw.bisco_debug_set_wait_test(0, 1_000_000)
+        bw.bisco_gemv(dl, Xd, Yd, ws)
+        assert bw.bisco_sync_status(ws) == bw.BISCO_ERR_TIMEOUT
+    finally:
+        bw.bisco_debug_set_wait_test(-1, 0)
+    bw.bisco_workspace_init(ws)
+    bw.bisco_gemv(dl, Xd, Yd, ws)
+    assert bw.bisco_sync_status(ws) == bw.BISCO_OK
+    rows = sample_rows(L.out, 128, 6)
+    check(Yd.cpu().numpy().astype(np.float64)[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
 
 
 def test_tensor_core_kernel_wait_gives_up_and_reports_timeout():
