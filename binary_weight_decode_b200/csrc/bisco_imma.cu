@@ -152,9 +152,12 @@ __device__ __forceinline__ int share_owner_i(int r, int R, int C) { return ((r +
 // Fixed-point exponent of a segment: V = round(v * 2^s) keeps |V| <= 2^22 for every
 // |v| <= vmax. vmax == 0 gives s = 0 (every V is 0).
 __device__ __forceinline__ int fixed_shift(float vmax) {
+  // vmax = f * 2^e with f in [0.5, 1): for a normal float e is the biased exponent - 126
+  const int eb = static_cast<int>((__float_as_uint(vmax) >> 23) & 0xFFu);
+  if (eb != 0) return 22 - (eb - 126);
   if (!(vmax > 0.f)) return 0;
   int e;
-  frexpf(vmax, &e);  // vmax = f * 2^e, f in [0.5, 1)
+  frexpf(vmax, &e);  // subnormal
   return 22 - e;
 }
 // 2^k for any integer k in [-252, 252], as the product of two representable factors.
@@ -699,6 +702,7 @@ __global__ void __launch_bounds__(kIT, 2)
     float sum[MB];
 #pragma unroll
     for (int m = 0; m < MB; ++m) sum[m] = 0.f;
+#pragma unroll 4
     for (int src = 0; src < p.C * kc; ++src) {  // (rank, contributor slot), fixed order
 #pragma unroll
       for (int m = 0; m < MB; ++m) sum[m] += S.recv[(static_cast<size_t>(src) * msh + sr) * MB + m];
@@ -777,6 +781,51 @@ int imma_clusters_mb(int MB, int C, size_t smem) {
     case 8: return imma_clusters<8>(C, smem);
     default: return 0;
   }
+}
+
+// Contributor slots a phase needs: nb row blocks x nun units split into kIW equal
+// contiguous item ranges; a warp writes slot (warp - first warp whose range starts at or
+// before the block's first item), exactly as the kernel numbers them.
+int phase_slots(int nb, int nun) {
+  if (nb <= 0 || nun <= 0) return 1;
+  const long long items = static_cast<long long>(nb) * nun;
+  int need = 1;
+  for (int w = 0; w < kIW; ++w) {
+    const long long a = w * items / kIW, b = (w + 1) * items / kIW;
+    if (b <= a) continue;
+    for (long long bl = a / nun; bl <= (b - 1) / nun; ++bl) {
+      int wf = w;
+      while (wf > 0 && wf * items / kIW > bl * nun) --wf;
+      need = std::max(need, w - wf + 1);
+    }
+  }
+  return need;
+}
+
+// Slots over every CTA shape of a pass: tile counts floor/ceil(tiles / ncl), the unit
+// range of each cluster rank, and (u_split >= 0) the two phases of the output pass of a
+// fused launch, split at unit u_split.
+int pass_slots(int tiles, int ncl, int units, int C, int BPT, int u_split) {
+  int need = 1;
+  for (int nt : {tiles / ncl, (tiles + ncl - 1) / ncl}) {
+    if (nt <= 0) continue;
+    const int nb = nt * BPT;
+    for (int r = 0; r < C; ++r) {
+      const int u0 = r * units / C, u1 = (r + 1) * units / C, nu = u1 - u0;
+      if (u_split < 0) {
+        need = std::max(need, phase_slots(nb, nu));
+      } else {
+        const int n0 = std::max(0, std::min(nu, u_split - u0)), n1 = nu - n0;
+        if (n0 > 0 && n1 > 0) {
+          need = std::max(need, phase_slots(nb, n0));
+          need = std::max(need, phase_slots(nb, n1));
+        } else {
+          need = std::max(need, phase_slots(nb, nu));
+        }
+      }
+    }
+  }
+  return need;
 }
 
 int max_segments_per_cta_i(int units, int C, const int* seg_unit0, int nseg) {
@@ -876,13 +925,10 @@ ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sa
       const int max_units = std::max(mu_y, mu_z);
       const int max_lseg = std::max(max_segments_per_cta_i(y.units, C, y.seg_unit0, y.nseg),
                                     z ? max_segments_per_cta_i(z->units, C, z->seg_unit0, z->nseg) : 1);
-      // contributor slots per row and phase: warps own equal contiguous ranges of (row
-      // block, unit) items, so with at least kIW row blocks in every CTA a block is
-      // touched by at most two warps; otherwise by at most kIW. A fused launch has two
-      // phases.
-      int nb_min = (tiles_y / ncl_y) * (32 / RB);
-      if (z) nb_min = std::min(nb_min, (tiles_z / ncl_z) * (32 / RB));
-      const int kc = (nb_min >= kIW ? 2 : kIW) * (z ? 2 : 1);
+      // contributor slots per row and phase (a fused launch has two phases)
+      int kcp = pass_slots(tiles_y, ncl_y, y.units, C, 32 / RB, z ? y.seg_unit0[y.nseg - 1] : -1);
+      if (z) kcp = std::max(kcp, pass_slots(tiles_z, ncl_z, z->units, C, 32 / RB, -1));
+      const int kc = kcp * (z ? 2 : 1);
       const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, kc, n_sal);
       if (need > smem_limit) continue;
       // kIW warps of a CTA work on kIW blocks at once: 237 / kIW cycles per block and SM
