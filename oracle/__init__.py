@@ -13,6 +13,7 @@ from .bisco_oracle import (  # noqa: F401
     decode_values,
     dense_correction_storage_bits,
     fluxbin_average_bit_width,
+    fluxbin_sign_search,
     fp4_weight_bits,
     gemv,
     gemv_rows,

@@ -234,6 +234,40 @@ def biloco_decompose(W, v0, rounds=5):
     return U, V, greedy, refit
 
 
+def fluxbin_sign_search(W, row_scale, col_scale, group=0):
+    """Joint binary signs of Kb bases for fixed magnitudes ("FluxBin", Sec. 3.1,
+    Decoupled Row-Column Binary Bases: with M^(k) = alpha_r^(k) alpha_c^(k)T the signs
+    minimise the reconstruction error, found by evaluating all 2^Kb sign combinations).
+
+    W [rows][cols]; row_scale [Kb][rows] (group == 0) or [Kb][rows][ceil(cols/group)] (one
+    row scale per weight group); col_scale [Kb][cols]. Element (o, i) takes the combination
+    c in 0 .. 2^Kb - 1 (bit k of c set: base k gets +1, clear: -1) with the smallest
+    (W[o][i] - sum_k s_k M^(k)[o][i])^2, the first such c on ties; fp64 throughout.
+    Returns the signs [Kb][rows][cols] as +1/-1 int8.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    rows, cols = W.shape
+    C = np.asarray(col_scale, dtype=np.float64)
+    Kb = C.shape[0]
+    R = np.asarray(row_scale, dtype=np.float64)
+    if group:
+        R = R.reshape(Kb, rows, -1)[:, :, np.arange(cols) // group]   # [Kb][rows][cols]
+    else:
+        R = np.broadcast_to(R.reshape(Kb, rows, 1), (Kb, rows, cols))
+    Mk = R * C[:, None, :]                                             # magnitudes M^(k)
+    best_err = np.full((rows, cols), np.inf)
+    best = np.zeros((rows, cols), dtype=np.int64)
+    for c in range(1 << Kb):
+        rec = np.zeros((rows, cols))
+        for k in range(Kb):
+            rec += (1.0 if (c >> k) & 1 else -1.0) * Mk[k]
+        err = (W - rec) ** 2
+        take = err < best_err  # strict: the first combination wins a tie
+        best[take] = c
+        best_err[take] = err[take]
+    return np.stack([np.where((best >> k) & 1, 1, -1).astype(np.int8) for k in range(Kb)])
+
+
 # ----------------------------------------------------------------------------
 # storage and byte accounting
 # ----------------------------------------------------------------------------

@@ -471,3 +471,88 @@ def test_row_decoder_matches_independent_packer(rows, cols):
     w = py_pack(S.tolist())
     sel = sorted({0, rows - 1, rows // 2, min(31, rows - 1), min(32, rows - 1)})
     assert np.array_equal(oracle.unpack_bit_rows(w, rows, cols, sel), S[sel])
+
+
+# ---- FluxBin joint sign search ("FluxBin", Sec. 3.1) --------------------------
+
+def _mags(rng, Kb, rows, cols, ng=None):
+    r = np.abs(rng.standard_normal((Kb, rows) if ng is None else (Kb, rows, ng))) + 0.05
+    c = np.abs(rng.standard_normal((Kb, cols))) + 0.05
+    return r, c
+
+
+def test_fluxbin_one_base_is_the_sign_of_w():
+    # Kb = 1: (w - m)^2 < (w + m)^2 exactly when w > 0 (m > 0); w = 0 ties and the first
+    # combination (-1) is kept
+    rng = np.random.default_rng(41)
+    W = rng.standard_normal((7, 9))
+    W[2, 3] = 0.0
+    r, c = _mags(rng, 1, 7, 9)
+    S = oracle.fluxbin_sign_search(W, r, c)
+    assert np.array_equal(S[0], np.where(W > 0, 1, -1))
+
+
+def test_fluxbin_two_bases_pick_the_nearest_of_four_levels():
+    # Kb = 2 with m1 > m2 > 0 per element: the levels -m1-m2 < -m1+m2 < m1-m2 < m1+m2 have
+    # midpoints -m1, 0, m1, so the optimum is (sign(w), sign(|w| - m1) * sign(w))
+    rng = np.random.default_rng(42)
+    rows, cols = 11, 13
+    W = rng.standard_normal((rows, cols)) * 2.0
+    r = np.stack([np.full(rows, 1.0), np.full(rows, 0.5)])
+    c = np.stack([np.abs(rng.standard_normal(cols)) + 1.0, np.abs(rng.standard_normal(cols)) * 0.5 + 0.1])
+    m1 = r[0][:, None] * c[0][None, :]
+    m2 = r[1][:, None] * c[1][None, :]
+    assert np.all(m1 > m2)
+    S = oracle.fluxbin_sign_search(W, r, c)
+    s1 = np.where(W >= 0, 1, -1)
+    s2 = np.where(np.abs(W) >= m1, 1, -1) * s1
+    assert np.array_equal(S[0], s1) and np.array_equal(S[1], s2)
+
+
+def test_fluxbin_brute_force_on_a_tiny_layer():
+    # every element against an explicit enumeration of sign vectors
+    import itertools
+    rng = np.random.default_rng(43)
+    rows, cols, Kb = 2, 3, 3
+    W = rng.standard_normal((rows, cols))
+    r, c = _mags(rng, Kb, rows, cols)
+    S = oracle.fluxbin_sign_search(W, r, c)
+    for o in range(rows):
+        for i in range(cols):
+            errs = {}
+            for sv in itertools.product((-1, 1), repeat=Kb):
+                errs[sv] = (W[o, i] - sum(sv[k] * r[k, o] * c[k, i] for k in range(Kb))) ** 2
+            chosen = tuple(int(S[k, o, i]) for k in range(Kb))
+            assert errs[chosen] == min(errs.values())
+
+
+def test_fluxbin_is_odd_and_beats_greedy_residual_signs():
+    rng = np.random.default_rng(44)
+    rows, cols, Kb = 16, 40, 3
+    W = rng.standard_normal((rows, cols))
+    r, c = _mags(rng, Kb, rows, cols)
+    S = oracle.fluxbin_sign_search(W, r, c)
+    assert np.array_equal(oracle.fluxbin_sign_search(-W, r, c), -S)  # symmetric levels, no ties
+    M = r[:, :, None] * c[:, None, :]
+    err = ((W - (S * M).sum(0)) ** 2).sum()
+    R = W.copy()
+    G = np.zeros_like(S)
+    for k in range(Kb):  # greedy: each base takes the sign of the current residual
+        G[k] = np.where(R >= 0, 1, -1)
+        R = R - G[k] * M[k]
+    assert err <= ((W - (G * M).sum(0)) ** 2).sum() + 1e-12
+
+
+def test_fluxbin_grouped_row_scales_use_the_group_of_each_column():
+    # one row scale per (row, group of g columns): equal to the ungrouped search run on each
+    # column block with that block's row scale
+    rng = np.random.default_rng(45)
+    rows, cols, Kb, g = 5, 300, 2, 128
+    ng = -(-cols // g)
+    W = rng.standard_normal((rows, cols))
+    r, c = _mags(rng, Kb, rows, cols, ng)
+    S = oracle.fluxbin_sign_search(W, r, c, group=g)
+    for j in range(ng):
+        blk = slice(j * g, min(cols, (j + 1) * g))
+        Sj = oracle.fluxbin_sign_search(W[:, blk], r[:, :, j], c[:, blk])
+        assert np.array_equal(S[:, :, blk], Sj)
