@@ -6,7 +6,12 @@ graph holding S back-to-back GEMVs over S distinct weight copies whose total
 size exceeds 3x the L2 cache, so every GEMV streams its weights from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bisco|reference]
-                    [--workload attn4096|mlp_gate_up|mlp_down|lowrank5120|cfg1] [--M m]
+                    [--workload attn4096|mlp_gate_up|mlp_down|lowrank5120|cfg1|decoder7b] [--M m]
+
+Workload decoder7b is the 32-layer Llama-7B-shaped decoder weight stream (per layer
+q, k, v, o 4096x4096, gate and up 4096->11008, down 11008->4096; 2 bases and a
+rank-256 binary correction each): one step replays a graph of all 224 GEMVs, in
+layer order, over 1.71 GB of distinct weights.
 
 Metric: effective HBM GB/s of the M=1 binary GEMV (algorithmic bytes: packed
 sign bits, scales, correction signs and coefficients, salient payload, X read
@@ -40,7 +45,21 @@ WORKLOADS = {
     "mlp_down": (3, 1, 1, "Llama-7B MLP down 11008->4096, 2 bases, 1% salient int8 columns"),
     "lowrank5120": (4, 0, 1, "5120x5120, 2 bases + rank-512 binary correction, 0.1% outliers x20"),
     "cfg1": (1, 0, 1, "256x512, 1 base, fp32 scales, rank-8 correction"),
+    "decoder7b": (5, None, 1, "32-layer Llama-7B decoder weight stream: q/k/v/o 4096^2, gate/up 4096->11008, "
+                              "down 11008->4096, 2 bases + rank-256 binary correction each (224 GEMVs)"),
 }
+DECODER_LAYERS = 32
+DECODER_MATRICES = 7  # q, k, v, o, gate, up, down
+
+
+def base_matrices(workload, M):
+    """(layer, X) pairs of the distinct matrices of a workload: one for the single-layer
+    workloads, the seven matrix shapes of a decoder layer for decoder7b (every decoder
+    layer streams its own device copy of them)."""
+    cfg, spec, _, _ = WORKLOADS[workload]
+    if spec is None:
+        return [build(cfg, i, M) for i in range(DECODER_MATRICES)]
+    return [build(cfg, spec, M)]
 
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
@@ -107,21 +126,6 @@ def max_over_ranks(value, dist, device):
     return float(t.item())
 
 
-def launches_per_gemv(M, rank, scale_bf16, tc_min=32, tc_max=128, lut_max=8):
-    """Kernel launches of one bisco_gemv call: the library's batch-chunk schedule
-    (tensor-core chunks of up to 128 rows from 32 rows up when the scales are bf16,
-    lookup-table chunks of up to 8 rows otherwise), one launch per pass per chunk.
-    The tensor-core plan also needs its accumulators to leave room in tensor memory
-    (at most three blocks at 128 rows); every bench workload has at most two bases
-    plus one correction/salient block, so the schedule above is the one that runs."""
-    chunks, rem = 0, M
-    while rem > 0:
-        take = min(rem, tc_max) if (scale_bf16 and rem >= tc_min) else min(rem, lut_max)
-        rem -= take
-        chunks += 1
-    return chunks * (2 if rank else 1)
-
-
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -179,7 +183,7 @@ def cpu_baseline(workload, M, budget_s=12.0):
     import oracle
     from threadpoolctl import threadpool_info
     cfg, spec, _, _ = WORKLOADS[workload]
-    L, X = build(cfg, spec, M)
+    L, X = build(cfg, spec if spec is not None else 0, M)  # decoder7b: its q projection
     xdt = "f32" if cfg == 1 else "bf16"
     nbytes = oracle.algorithmic_bytes(L, M, xdt, "bf16")
     n, t0 = 0, time.perf_counter()
@@ -192,7 +196,8 @@ def cpu_baseline(workload, M, budget_s=12.0):
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     return {"value": round(n * nbytes / el / 1e9, 4), "unit": "GB/s", "cores": int(threads),
             "kind": "oracle", "us_per_gemv": el / n * 1e6,
-            "sample": f"{n} full fp64 oracle GEMVs of the {workload} layer (M={M}) in {el:.1f} s on {os.cpu_count()} host cores"}
+            "sample": f"{n} full fp64 oracle GEMVs of the {workload} layer{' q projection' if spec is None else ''} "
+                      f"(M={M}) in {el:.1f} s on {os.cpu_count()} host cores"}
 
 
 def run_reference(args):
@@ -256,12 +261,17 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
 
     M = args.M
-    L, X = build(cfg, spec, M)
+    mats = base_matrices(args.workload, M)
     xdt = "f32" if cfg == 1 else "bf16"
+
+    def dev_x(X):
+        Xh = torch.from_numpy(X.view(np.int16) if xdt == "bf16" else X)
+        return Xh, (Xh.to("cuda").view(torch.bfloat16) if xdt == "bf16" else Xh.to("cuda"))
+
     if args.calls:  # small case for ncu captures: no graph, no timing
+        L, X = mats[0]
         dl = bw.DeviceLayer(L)
-        Xd = torch.from_numpy(X.view(np.int16) if xdt == "bf16" else X).cuda()
-        Xd = Xd.view(torch.bfloat16) if xdt == "bf16" else Xd
+        Xd = dev_x(X)[1]
         Yd = torch.empty((M, L.out), dtype=torch.bfloat16, device="cuda")
         ws = bw.alloc_workspace([dl], M)
         for _ in range(args.calls):
@@ -273,31 +283,41 @@ def main():
         return
     x_bytes = 4 if xdt == "f32" else 2
     y_dtype = torch.bfloat16
-    nbytes = algorithmic_bytes(L, M, x_bytes, 2)
+    nbytes_b = [algorithmic_bytes(L, M, x_bytes, 2) for (L, _) in mats]
     props = torch.cuda.get_device_properties(local)
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
-    S = max(4, math.ceil(3 * l2 / nbytes))
+    if WORKLOADS[args.workload][1] is None:
+        S = DECODER_LAYERS  # the decoder stream: one copy per layer (1.7 GB, far above L2)
+    else:
+        S = max(4, math.ceil(3 * l2 / nbytes_b[0]))
+    nbytes = sum(nbytes_b)  # one pass over the distinct matrices
 
-    # S distinct weight copies: same values, separate HBM buffers
-    dls = [bw.DeviceLayer(L) for _ in range(S)]
-    Xh = torch.from_numpy(X.view(np.int16) if xdt == "bf16" else X)
-    Xd = Xh.to("cuda")
-    if xdt == "bf16":
-        Xd = Xd.view(torch.bfloat16)
-    Yd = torch.empty((S, M, L.out), dtype=y_dtype, device="cuda")
-    ws = bw.alloc_workspace(dls[:1], M)
+    # S distinct device copies of every base matrix: same values, separate HBM buffers
+    first = [bw.DeviceLayer(L) for (L, _) in mats]
+    dls = [[d] + [d.clone() for _ in range(S - 1)] for d in first]
+    xs = [dev_x(X) for (_, X) in mats]
+    Yd = [torch.empty((S, M, L.out), dtype=y_dtype, device="cuda") for (L, _) in mats]
+    ws = bw.alloc_workspace(first, M)
+    ws_bytes = ws.numel() * ws.element_size()
+    xcode = bw.BISCO_BF16 if xdt == "bf16" else bw.BISCO_F32
+    kinds = [bw.bisco_plan_kernels(d, M, xcode, ws_bytes) for d in first]
+
+    def stream_once(stream):
+        for i in range(S):
+            for b in range(len(mats)):
+                bw.bisco_gemv(dls[b][i], xs[b][1], Yd[b][i], ws, stream=stream)
 
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
-        for i in range(S):  # eager warm-up run (also sets kernel attributes before capture)
-            bw.bisco_gemv(dls[i], Xd, Yd[i], ws, stream=stream)
+        stream_once(stream)  # eager warm-up run (also sets kernel attributes before capture)
     stream.synchronize()
+    st = bw.bisco_sync_status(ws)
+    if st != bw.BISCO_OK:
+        raise SystemExit(f"device status {bw.bisco_status_string(st)}")
     with torch.cuda.graph(graph, stream=stream):
-        for i in range(S):
-            bw.bisco_gemv(dls[i], Xd, Yd[i], ws, stream=stream)
-    kernels_per_gemv = launches_per_gemv(M, L.rank, L.K == 0 or L.scale_dtype == "bf16")
+        stream_once(stream)
 
     def barrier():
         if dist is not None:
@@ -323,15 +343,14 @@ def main():
     ms = e0.elapsed_time(e1)
     clocks = sampler.stop()
     ms = max_over_ranks(ms, dist, "cuda")
-    gemvs = args.steps * S
+    gemvs = args.steps * S * len(mats)
     us_per_gemv = ms * 1000.0 / gemvs
-    value = world * gemvs * nbytes / (ms / 1000.0) / 1e9
+    value = world * args.steps * S * nbytes / (ms / 1000.0) / 1e9
 
     # end to end through the public API: pinned host X in, host Y out, every step
-    Xpin = Xh.pin_memory()
-    Ypin = torch.empty((S, M, L.out), dtype=torch.int16).pin_memory()
-    Yd16 = Yd.view(torch.int16)
-    Xd_raw = Xd.view(torch.int16) if xdt == "bf16" else Xd
+    Xpins = [xh.pin_memory() for (xh, _) in xs]
+    Xraws = [xd.view(torch.int16) if xdt == "bf16" else xd for (_, xd) in xs]
+    Ypins = [torch.empty(y.shape, dtype=torch.int16).pin_memory() for y in Yd]
     e2 = torch.cuda.Event(enable_timing=True)
     e3 = torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, args.steps // 2)
@@ -339,25 +358,29 @@ def main():
     e2.record(stream)
     with torch.cuda.stream(stream):
         for _ in range(e2e_steps):
-            Xd_raw.copy_(Xpin, non_blocking=True)
+            for xr, xp in zip(Xraws, Xpins):
+                xr.copy_(xp, non_blocking=True)
             graph.replay()
-            Ypin.copy_(Yd16, non_blocking=True)
+            for yp, y in zip(Ypins, Yd):
+                yp.copy_(y.view(torch.int16), non_blocking=True)
     e3.record(stream)
     barrier()
     ms_e2e = e2.elapsed_time(e3)
     ms_e2e = max_over_ranks(ms_e2e, dist, "cuda")
     e2e_value = world * e2e_steps * S * nbytes / (ms_e2e / 1000.0) / 1e9
-
+    L = mats[0][0]
     peak, peak_kind = hbm_peak()
-    achieved = nbytes / (us_per_gemv * 1e-6) / 1e9
+    us_per_pass = ms * 1000.0 / (args.steps * S)  # one GEMV of every distinct matrix
+    achieved = nbytes / (us_per_pass * 1e-6) / 1e9
     # batch chunks of 32+ rows run on the tensor cores (bf16 scales): a dense contraction
     on_tensor = M >= 32 and (L.K == 0 or L.scale_dtype == "bf16")
     if on_tensor:
         tpeak, tpeak_kind = tensor_peak()
-        tflops = algorithmic_flops(L, M) / (us_per_gemv * 1e-6) / 1e12
+        flops = sum(algorithmic_flops(Lb, M) for (Lb, _) in mats)
+        tflops = flops / (us_per_pass * 1e-6) / 1e12
         roofline = {"bound": "tensor", "achieved": round(tflops, 2), "peak": tpeak, "unit": "TFLOP/s",
                     "frac": round(tflops / tpeak, 4), "peak_kind": f"{tpeak_kind} dense bf16 (burst)",
-                    "flops_per_gemv": algorithmic_flops(L, M), "traffic": traffic_for(args.workload, M)}
+                    "flops_per_gemv": flops / len(mats), "traffic": traffic_for(args.workload, M)}
     else:
         roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
@@ -368,17 +391,21 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if on_tensor else "f32",
         "data": "synthetic",
         "impl": "bisco",
-        "config": {"workload": f"{args.workload}: {desc}", "M": M, "gemvs_per_step": S,
-                   "algorithmic_bytes_per_gemv": nbytes, "y_dtype": "bf16",
-                   "l2": f"inputs larger than L2: each step streams {S} distinct weight copies "
+        "config": {"workload": f"{args.workload}: {desc}", "M": M, "gemvs_per_step": S * len(mats),
+                   "algorithmic_bytes_per_gemv": nbytes if len(mats) == 1 else round(nbytes / len(mats)),
+                   "algorithmic_bytes_per_step": S * nbytes, "y_dtype": "bf16",
+                   "l2": f"inputs larger than L2: each step streams {S * len(mats)} distinct weight copies "
                          f"({S * nbytes / 2 ** 20:.0f} MiB > 3x L2)",
+                   "kernels_per_gemv": kinds if len(mats) > 1 else kinds[0],
                    "parallelism": f"replicas x{world} (no collective)"},
         "us_per_gemv": round(us_per_gemv, 4),
+        "us_per_step": round(ms * 1000.0 / args.steps, 2),
         "roofline": roofline,
         "clocks": clocks,
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(Xh.numel() * Xh.element_size()),
-                "d2h_bytes_per_step": int(Ypin.numel() * 2)},
-        "gpu_launches": int(args.steps * S * kernels_per_gemv),
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": int(sum(x.numel() * x.element_size() for x in Xpins)),
+                "d2h_bytes_per_step": int(sum(y.numel() * 2 for y in Ypins))},
+        "gpu_launches": int(args.steps * S * sum(len(k) for k in kinds)),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, M)

@@ -32,6 +32,7 @@ EXPORTED = [
     "bisco_packed_words", "bisco_pack", "bisco_unpack", "bisco_workspace_size", "bisco_workspace_init",
     "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string", "bisco_gemv_noalloc",
     "bisco_set_path_policy", "bisco_plan_kernels", "bisco_debug_set_wait_test",
+    "bisco_fluxbin_signs", "bisco_biloco_workspace_size", "bisco_biloco_decompose",
 ]
 
 
@@ -43,6 +44,7 @@ class bisco_layer(ctypes.Structure):
         ("v_bits", ctypes.c_void_p), ("ut_bits", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
         ("n_sal", ctypes.c_int32), ("sal_stride", ctypes.c_int32),
         ("sal_idx", ctypes.c_void_p), ("sal_q", ctypes.c_void_p), ("sal_scale", ctypes.c_void_p),
+        ("row_group", ctypes.c_int32),
     ]
 
 
@@ -91,6 +93,14 @@ _lib.bisco_plan_kernels.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32,
 _lib.bisco_plan_kernels.restype = ctypes.c_int32
 _lib.bisco_debug_set_wait_test.argtypes = [ctypes.c_int32, ctypes.c_uint64]
 _lib.bisco_debug_set_wait_test.restype = ctypes.c_int
+_lib.bisco_fluxbin_signs.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, ctypes.c_int32, _P, _P]
+_lib.bisco_fluxbin_signs.restype = ctypes.c_int
+_lib.bisco_biloco_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+                                             ctypes.POINTER(ctypes.c_size_t)]
+_lib.bisco_biloco_workspace_size.restype = ctypes.c_int
+_lib.bisco_biloco_decompose.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                        _P, _P, _P, _P, ctypes.c_size_t, _P]
+_lib.bisco_biloco_decompose.restype = ctypes.c_int
 
 
 class BiscoError(RuntimeError):
@@ -173,15 +183,15 @@ class DeviceLayer:
                 return torch.from_numpy(a.view(np.int32)).to(device)
             return torch.from_numpy(a).to(device)
 
-        if getattr(host, "group", 0):
-            # bisco_layer carries one row scale per (base, row); grouped row scales are not
-            # part of the C ABI yet
-            raise NotImplementedError("grouped row scales are not supported by libbisco")
         self.host = host
+        self.row_group = int(getattr(host, "group", 0) or 0)
         self.out, self.in_, self.K = host.out, host.in_, host.K
         self.rank, self.n_sal = host.rank, host.n_sal
         self.bits = up(host.bits) if host.K else None
-        self.row_scale = up(host.row_scale) if host.K else None
+        rs = host.row_scale
+        if host.K and self.row_group:  # host [K][out][groups] -> device [K][groups][out]
+            rs = np.ascontiguousarray(np.asarray(rs).reshape(host.K, host.out, -1).transpose(0, 2, 1))
+        self.row_scale = up(rs) if host.K else None
         self.col_scale = up(host.col_scale) if host.K else None
         self.v_bits = up(host.v_bits)
         self.ut_bits = up(host.ut_bits)
@@ -196,7 +206,26 @@ class DeviceLayer:
             scale_dtype=BISCO_BF16 if host.scale_dtype == "bf16" else BISCO_F32,
             rank=host.rank, v_bits=ptr(self.v_bits), ut_bits=ptr(self.ut_bits), alpha=ptr(self.alpha),
             n_sal=host.n_sal, sal_stride=host.sal_stride if host.n_sal else 0,
-            sal_idx=ptr(self.sal_idx), sal_q=ptr(self.sal_q), sal_scale=ptr(self.sal_scale))
+            sal_idx=ptr(self.sal_idx), sal_q=ptr(self.sal_q), sal_scale=ptr(self.sal_scale),
+            row_group=self.row_group)
+
+    def clone(self):
+        """Another device copy of the same layer (same values, separate device buffers)."""
+        c = DeviceLayer.__new__(DeviceLayer)
+        c.host = self.host
+        c.out, c.in_, c.K, c.rank, c.n_sal = self.out, self.in_, self.K, self.rank, self.n_sal
+        c.row_group = self.row_group
+        for n in ("bits", "row_scale", "col_scale", "v_bits", "ut_bits", "alpha", "sal_idx", "sal_q", "sal_scale"):
+            t = getattr(self, n)
+            setattr(c, n, t.clone() if t is not None else None)
+        ptr = lambda t: (t.data_ptr() if t is not None else None)  # noqa: E731
+        d = self.desc
+        c.desc = bisco_layer(
+            out=d.out, in_=d.in_, num_bases=d.num_bases, bits=ptr(c.bits), row_scale=ptr(c.row_scale),
+            col_scale=ptr(c.col_scale), scale_dtype=d.scale_dtype, rank=d.rank, v_bits=ptr(c.v_bits),
+            ut_bits=ptr(c.ut_bits), alpha=ptr(c.alpha), n_sal=d.n_sal, sal_stride=d.sal_stride,
+            sal_idx=ptr(c.sal_idx), sal_q=ptr(c.sal_q), sal_scale=ptr(c.sal_scale), row_group=d.row_group)
+        return c
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
@@ -285,3 +314,43 @@ def bisco_plan_kernels(layer, M: int, x_dtype: int, ws_bytes: int) -> list:
 def bisco_debug_set_wait_test(skip_tile: int, wait_ns: int = 0):
     """Test hook for the integer kernel's bounded waits (skip_tile = -1 turns it off)."""
     _check(_lib.bisco_debug_set_wait_test(int(skip_tile), int(wait_ns)), "bisco_debug_set_wait_test")
+
+
+def bisco_fluxbin_signs(W, row_scale, col_scale, group=0, stream=None):
+    """Packed joint signs of Kb bases ([Kb, packed_words] int32 on W's device) for fp64
+    device tensors W [rows, cols], row_scale [Kb, rows] (or [Kb, groups, rows] with
+    group > 0) and col_scale [Kb, cols]; see include/bisco.h."""
+    torch = _torch()
+    rows, cols = W.shape
+    Kb = col_scale.shape[0]
+    for t in (W, row_scale, col_scale):
+        if t.dtype != torch.float64 or not t.is_contiguous():
+            raise BiscoError(BISCO_ERR_INVALID_ARG, "bisco_fluxbin_signs")
+    bits = torch.empty((Kb, bisco_packed_words(rows, cols)), dtype=torch.int32, device=W.device)
+    _check(_lib.bisco_fluxbin_signs(ctypes.c_void_p(W.data_ptr()), rows, cols, Kb,
+                                    ctypes.c_void_p(row_scale.data_ptr()), ctypes.c_void_p(col_scale.data_ptr()),
+                                    int(group), ctypes.c_void_p(bits.data_ptr()), _stream_ptr(stream)),
+           "bisco_fluxbin_signs")
+    return bits
+
+
+def bisco_biloco_decompose(W, v0, rounds=5, stream=None):
+    """Binary low-rank decomposition of an fp64 device matrix W [rows, cols] from starting
+    signs v0 [rank, cols] (int8, +-1): returns U [rows, rank], V [rank, cols] (int8) and the
+    greedy and refit coefficients [rank] (fp64); see include/bisco.h."""
+    torch = _torch()
+    rows, cols = W.shape
+    rank = v0.shape[0]
+    if W.dtype != torch.float64 or v0.dtype != torch.int8 or not W.is_contiguous() or not v0.is_contiguous():
+        raise BiscoError(BISCO_ERR_INVALID_ARG, "bisco_biloco_decompose")
+    n = ctypes.c_size_t(0)
+    _check(_lib.bisco_biloco_workspace_size(rows, cols, rank, ctypes.byref(n)), "bisco_biloco_workspace_size")
+    ws = torch.empty(int(n.value), dtype=torch.uint8, device=W.device)
+    U = torch.empty((rows, rank), dtype=torch.int8, device=W.device)
+    V = torch.empty((rank, cols), dtype=torch.int8, device=W.device)
+    ag = torch.empty(rank, dtype=torch.float64, device=W.device)
+    ar = torch.empty(rank, dtype=torch.float64, device=W.device)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    _check(_lib.bisco_biloco_decompose(p(W), rows, cols, rank, int(rounds), p(v0), p(U), p(V), p(ag), p(ar), p(ws),
+                                       int(n.value), _stream_ptr(stream)), "bisco_biloco_decompose")
+    return U, V, ag, ar

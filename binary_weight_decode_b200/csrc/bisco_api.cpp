@@ -59,6 +59,7 @@ bisco_status validate_layer(const bisco_layer* L) {
   if (!L) return BISCO_ERR_INVALID_ARG;
   if (L->out < 1 || L->in < 1 || L->num_bases < 0 || L->num_bases > kMaxBases) return BISCO_ERR_INVALID_ARG;
   if (L->rank < 0 || L->rank > (1 << 20) || L->n_sal < 0 || L->n_sal > L->in) return BISCO_ERR_INVALID_ARG;
+  if (L->row_group < 0) return BISCO_ERR_INVALID_ARG;
   if (L->num_bases > 0) {
     if (!L->bits || !L->row_scale || !L->col_scale || !aligned16(L->bits)) return BISCO_ERR_INVALID_ARG;
     if (!dtype_ok(L->scale_dtype)) return BISCO_ERR_INVALID_ARG;
@@ -80,14 +81,22 @@ int batch_block(int Mc) { return Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8; }
 // a layer with neither gets one empty unit so the salient term still has a home.
 struct SegList {
   int unit0[kMaxSeg];
+  int rgu[kMaxSeg];  // quads per row-scale group (0: one row scale per row)
   int nseg, units;
 };
 
+// Quads per row-scale group of the bases (0 without grouped row scales).
+int row_group_quads(const bisco_layer* L) { return L->row_group > 0 ? L->row_group / 128 : 0; }
+
 SegList segs_y(const bisco_layer* L) {
   SegList s{};
-  for (int k = 0; k < L->num_bases; ++k) { s.unit0[s.nseg++] = s.units; s.units += quads(L->in); }
-  if (L->rank > 0) { s.unit0[s.nseg++] = s.units; s.units += quads(L->rank); }
-  if (s.nseg == 0) { s.unit0[s.nseg++] = 0; s.units = 1; }
+  for (int k = 0; k < L->num_bases; ++k) {
+    s.rgu[s.nseg] = row_group_quads(L);
+    s.unit0[s.nseg++] = s.units;
+    s.units += quads(L->in);
+  }
+  if (L->rank > 0) { s.rgu[s.nseg] = 0; s.unit0[s.nseg++] = s.units; s.units += quads(L->rank); }
+  if (s.nseg == 0) { s.rgu[s.nseg] = 0; s.unit0[s.nseg++] = 0; s.units = 1; }
   return s;
 }
 
@@ -106,12 +115,12 @@ Layout layout_for(const bisco_layer* L, int MB, int dev) {
   lo.has_z = L->rank > 0;
   const SegList sy = segs_y(L);
   lo.py = make_plan(L->out, sy.units, sy.unit0, sy.nseg, MB, L->n_sal, sms, lim);
-  const ImmaShape ys{L->out, sy.units, sy.unit0, sy.nseg};
+  const ImmaShape ys{L->out, sy.units, sy.unit0, sy.nseg, sy.rgu};
   lo.iy = make_imma_plan(ys, nullptr, MB, L->n_sal, lim);
   if (lo.has_z) {
     const int z0 = 0;
     lo.pz = make_plan(L->rank, quads(L->in), &z0, 1, MB, 0, sms, lim);
-    const ImmaShape zs{L->rank, quads(L->in), &z0, 1};
+    const ImmaShape zs{L->rank, quads(L->in), &z0, 1, nullptr};
     lo.iz = make_imma_plan(zs, nullptr, MB, 0, lim);
     lo.ifz = make_imma_plan(ys, &zs, MB, L->n_sal, lim);
   }
@@ -124,15 +133,16 @@ Layout layout_for(const bisco_layer* L, int MB, int dev) {
 // re-run the occupancy queries.
 Layout cached_layout(const bisco_layer* L, int MB, int dev) {
   struct Key {
-    int dev, out, in, K, rank, n_sal, MB;
+    int dev, out, in, K, rank, n_sal, MB, rg;
     bool operator==(const Key& o) const {
-      return dev == o.dev && out == o.out && in == o.in && K == o.K && rank == o.rank && n_sal == o.n_sal && MB == o.MB;
+      return dev == o.dev && out == o.out && in == o.in && K == o.K && rank == o.rank && n_sal == o.n_sal &&
+             MB == o.MB && rg == o.rg;
     }
   };
   struct Entry { Key k; Layout lo; };
   static std::mutex mu;
   static std::vector<Entry>* cache = new std::vector<Entry>();
-  const Key k{dev, L->out, L->in, L->num_bases, L->rank, L->n_sal, MB};
+  const Key k{dev, L->out, L->in, L->num_bases, L->rank, L->n_sal, MB, L->row_group};
   std::lock_guard<std::mutex> g(mu);
   for (const Entry& e : *cache)
     if (e.k == k) return e.lo;
@@ -187,6 +197,9 @@ void pass_z(const bisco_layer* L, PassParam& pz, const void* Xc, int32_t x_dtype
   V.rdt = BISCO_F32;
   V.cvec = 0;
   V.rvec = aligned16(L->alpha);
+  V.rgu = 0;
+  V.rgstride = 0;
+  V.part0 = 0;
   pz.rows = L->rank;
   pz.tiles = (L->rank + 31) / 32;
   pz.units = V.nq;
@@ -205,7 +218,7 @@ void pass_z(const bisco_layer* L, PassParam& pz, const void* Xc, int32_t x_dtype
 void pass_y(const bisco_layer* L, PassParam& py, const void* Xc, int32_t x_dtype, int Mc, void* Yc, int32_t y_dtype,
             float* zbuf, int* status) {
   const size_t xb = dtype_bytes(x_dtype);
-  int nseg = 0, unit = 0;
+  int nseg = 0, unit = 0, parts = 0;
   for (int k = 0; k < L->num_bases; ++k) {
     SegParam& B = py.seg[nseg++];
     B.bits = reinterpret_cast<const uint4*>(L->bits + static_cast<size_t>(k) * bisco_packed_words(L->out, L->in));
@@ -216,10 +229,17 @@ void pass_y(const bisco_layer* L, PassParam& py, const void* Xc, int32_t x_dtype
     B.xsrc = 0;
     B.cscale = static_cast<const unsigned char*>(L->col_scale) + static_cast<size_t>(k) * L->in * dtype_bytes(L->scale_dtype);
     B.cdt = L->scale_dtype;
-    B.rscale = static_cast<const unsigned char*>(L->row_scale) + static_cast<size_t>(k) * L->out * dtype_bytes(L->scale_dtype);
+    const size_t ngroups = L->row_group > 0 ? (static_cast<size_t>(L->in) + L->row_group - 1) / L->row_group : 1;
+    B.rscale = static_cast<const unsigned char*>(L->row_scale) +
+               static_cast<size_t>(k) * ngroups * L->out * dtype_bytes(L->scale_dtype);
     B.rdt = L->scale_dtype;
+    B.rgu = row_group_quads(L);
+    B.rgstride = L->out;
+    B.part0 = parts;
+    parts += B.rgu > 0 ? (B.nq + B.rgu - 1) / B.rgu : 1;
     B.cvec = aligned16(B.cscale);
-    B.rvec = aligned16(B.rscale);
+    // vector loads of a group's scale vector need every group offset 16-byte aligned too
+    B.rvec = aligned16(B.rscale) && (B.rgu == 0 || (static_cast<size_t>(L->out) * dtype_bytes(L->scale_dtype)) % 16 == 0);
   }
   if (L->rank > 0) {
     SegParam& U = py.seg[nseg++];
@@ -234,12 +254,18 @@ void pass_y(const bisco_layer* L, PassParam& py, const void* Xc, int32_t x_dtype
     U.rscale = nullptr;
     U.rdt = BISCO_F32;
     U.cvec = U.rvec = 0;
+    U.rgu = 0;
+    U.rgstride = 0;
+    U.part0 = parts++;
   }
   if (nseg == 0) {  // salient-only (or empty) layer: one empty unit
     SegParam& E = py.seg[nseg++];
     E.bits = nullptr; E.nq = 1; E.ncols = 0; E.unit0 = 0; E.xsrc = 2;
     E.cscale = nullptr; E.rscale = nullptr; E.cdt = E.rdt = BISCO_F32;
     E.cvec = E.rvec = 0;
+    E.rgu = 0;
+    E.rgstride = 0;
+    E.part0 = 0;
     unit = 1;
   }
   py.nseg = nseg;
@@ -317,8 +343,11 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
     tc_rows = static_cast<int>(std::min<size_t>(kTcMaxBatch, fit / 16 * 16));
   }
   const int policy = g_policy.load();
+  // grouped row scales: only the integer tensor-core kernel applies them, per 128-column unit
+  const bool grouped = L->num_bases > 0 && L->row_group > 0;
+  if (grouped && L->row_group % 128 != 0) return BISCO_ERR_UNSUPPORTED;
   const bool tc_ok = (L->num_bases == 0 || L->scale_dtype == BISCO_BF16) && tc_rows >= kTcMinBatch &&
-                     policy != BISCO_PATH_SMALL_BATCH_ONLY;
+                     policy != BISCO_PATH_SMALL_BATCH_ONLY && !grouped;
   for (int m0 = 0; m0 < M;) {
     Chunk ch{};
     ch.m0 = m0;
@@ -334,9 +363,10 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
       // which are faster there; with a correction the one-launch integer kernel wins
       // (5120 x 5120, rank 512: 13.5 us against 16.4 us for the two lookup-table launches)
       const bool fusable = ch.lo.has_z && ch.lo.ifz.C > 0;
-      ch.imma = policy != BISCO_PATH_LOOKUP_TABLE && imma_fits(ch.lo) &&
-                (batch_block(ch.Mc) >= 2 || policy == BISCO_PATH_INTEGER_MMA || fusable);
+      ch.imma = imma_fits(ch.lo) && (grouped || (policy != BISCO_PATH_LOOKUP_TABLE &&
+                (batch_block(ch.Mc) >= 2 || policy == BISCO_PATH_INTEGER_MMA || fusable)));
       ch.fused = ch.imma && fusable;
+      if (grouped && !ch.imma) return BISCO_ERR_UNSUPPORTED;
       if (!ch.imma && !plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
     }
     out->push_back(ch);

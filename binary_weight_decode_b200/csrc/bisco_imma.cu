@@ -71,6 +71,7 @@ struct ISmem {
   int* lsstart;            // [max_lseg]                  start (local unit index) of a local segment
   int* lsend;              // [max_lseg]                  end (local unit index) of a local segment
   int* lsbits;             // [max_lseg]                  1 if the segment has sign bits
+  int2* lsinfo;            // [max_lseg]                  (segment, row-scale group) of a local part
   unsigned* xmax;          // [max_lseg][MB]              max |v| (float bits) over the CTA's columns
   unsigned long long* vsum;  // [max_lseg][MB]            sum of the fixed-point values V (two's complement)
   int* flags;              // [4]                         [0]: a wait timed out
@@ -97,6 +98,7 @@ __host__ __device__ __forceinline__ size_t ismem_bytes(int MB, int C, int max_ti
   n += a16(static_cast<size_t>(max_tiles) * 8);
   n += a16(static_cast<size_t>(max_units) * 4);
   n += 3 * a16(static_cast<size_t>(max_lseg) * 4);
+  n += a16(static_cast<size_t>(max_lseg) * 8);
   n += a16(static_cast<size_t>(max_lseg) * MB * 4);
   n += a16(static_cast<size_t>(max_lseg) * MB * 8);
   n += 16;
@@ -122,6 +124,7 @@ __device__ __forceinline__ ISmem icarve(unsigned char* smem, const PassParam& p,
   s.lsstart = reinterpret_cast<int*>(q);             q += a16(static_cast<size_t>(p.max_lseg) * 4);
   s.lsend = reinterpret_cast<int*>(q);               q += a16(static_cast<size_t>(p.max_lseg) * 4);
   s.lsbits = reinterpret_cast<int*>(q);              q += a16(static_cast<size_t>(p.max_lseg) * 4);
+  s.lsinfo = reinterpret_cast<int2*>(q);             q += a16(static_cast<size_t>(p.max_lseg) * 8);
   s.xmax = reinterpret_cast<unsigned*>(q);           q += a16(static_cast<size_t>(p.max_lseg) * MB * 4);
   s.vsum = reinterpret_cast<unsigned long long*>(q); q += a16(static_cast<size_t>(p.max_lseg) * MB * 8);
   s.flags = reinterpret_cast<int*>(q);               q += 16;
@@ -144,6 +147,13 @@ __device__ __forceinline__ int seg_of_unit(const PassParam& p, int u) {
   for (int k = 1; k < kMaxSeg; ++k)
     if (k < p.nseg && u >= p.seg[k].unit0) s = k;
   return s;
+}
+
+// Pass-wide index of the (segment, row-scale group) part holding unit u: a segment
+// without grouped row scales is one part.
+__device__ __forceinline__ int part_of_unit(const PassParam& p, int u) {
+  const SegParam& G = p.seg[seg_of_unit(p, u)];
+  return G.part0 + (G.rgu > 0 ? (u - G.unit0) / G.rgu : 0);
 }
 
 __device__ __forceinline__ int share_begin_i(int d, int R, int C) { return d * R / C; }
@@ -208,8 +218,9 @@ __global__ void __launch_bounds__(kIT, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, tq = lane & 3;
   const int nsp = (p.n_sal + 3) & ~3;
-  const int seg_first = nu > 0 ? seg_of_unit(p, u0) : 0;
-  const int nls = nu > 0 ? seg_of_unit(p, u1 - 1) - seg_first + 1 : 0;
+  // local parts: the (segment, row-scale group) pairs this CTA's units touch, in order
+  const int part_first = nu > 0 ? part_of_unit(p, u0) : 0;
+  const int nls = nu > 0 ? part_of_unit(p, u1 - 1) - part_first + 1 : 0;
   const ISmem S = icarve(smem, p, MB, kc);
   const int rows_c = nt * 32;
   const int msh = msh_of(p.max_tiles, p.C);
@@ -219,14 +230,18 @@ __global__ void __launch_bounds__(kIT, 2)
   // ---- set-up: barriers, unit table, counters ----
   for (int i = threadIdx.x; i < nt; i += kIT) dev::mbar_init(S.bar + i, 1);
   for (int ul = threadIdx.x; ul < nu; ul += kIT) {
-    const int sg = seg_of_unit(p, u0 + ul);
-    S.useg[ul] = sg - seg_first;
-  }
-  for (int ls = threadIdx.x; ls < nls; ls += kIT) {
-    const SegParam& G = p.seg[seg_first + ls];
-    S.lsstart[ls] = max(u0, G.unit0) - u0;
-    S.lsend[ls] = min(u1, G.unit0 + G.nq) - u0;
-    S.lsbits[ls] = G.bits != nullptr ? 1 : 0;
+    const int u = u0 + ul;
+    const int sg = seg_of_unit(p, u);
+    const SegParam& G = p.seg[sg];
+    const int grp = G.rgu > 0 ? (u - G.unit0) / G.rgu : 0;
+    const int lp = G.part0 + grp - part_first;
+    S.useg[ul] = lp;
+    if (ul == 0 || part_of_unit(p, u - 1) != G.part0 + grp) {  // first unit of its part
+      S.lsstart[lp] = ul;
+      S.lsbits[lp] = G.bits != nullptr ? 1 : 0;
+      S.lsinfo[lp] = make_int2(sg, grp);
+    }
+    if (ul == nu - 1 || part_of_unit(p, u + 1) != G.part0 + grp) S.lsend[lp] = ul + 1;
   }
   for (int i = threadIdx.x; i < nls * MB; i += kIT) { S.xmax[i] = 0u; S.vsum[i] = 0ull; }
   if (threadIdx.x == 0) { S.flags[0] = 0; S.flags[1] = 0; }
@@ -262,14 +277,17 @@ __global__ void __launch_bounds__(kIT, 2)
       } else {
         const int rc = ch - n_cs;
         const int ls = rc / (nt * 4), r8 = (rc - ls * nt * 4) * 8;
-        const SegParam& G = p.seg[seg_first + ls];
+        const int2 li = S.lsinfo[ls];
+        const SegParam& G = p.seg[li.x];
         const int o = t0 * 32 + r8;
         const int valid = max(0, min(8, p.rows - o));
         if (G.rscale == nullptr) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) v[j] = j < valid ? 1.f : 0.f;
         } else if (valid > 0) {
-          dev::load8_ro(G.rscale, o, G.rdt, valid, G.rvec != 0, v);
+          // group li.y's scale vector (the host clears rvec when a group offset would break
+          // the 16-byte alignment)
+          dev::load8_ro(G.rscale, static_cast<long long>(li.y) * G.rgstride + o, G.rdt, valid, G.rvec != 0, v);
         }
         d = S.rsc + ls * p.max_tiles * 32 + r8;
       }
@@ -329,7 +347,7 @@ __global__ void __launch_bounds__(kIT, 2)
   int uT = nu;  // first local unit of a z-reading segment
   if (fused && !role_z)
     for (int ls = 0; ls < nls; ++ls)
-      if (p.seg[seg_first + ls].xsrc == 1) { uT = min(uT, S.lsstart[ls]); }
+      if (p.seg[S.lsinfo[ls].x].xsrc == 1) { uT = min(uT, S.lsstart[ls]); }
   const int nph = (fused && !role_z && uT < nu && uT > 0) ? 2 : 1;
   const int kcp = kc / (fused ? 2 : 1);  // contributor slots per phase
   bool ok = true;
@@ -397,7 +415,7 @@ __global__ void __launch_bounds__(kIT, 2)
           float4* d4 = reinterpret_cast<float4*>(S.xt + static_cast<size_t>(ulm) * 128 + j0);
           d4[0] = make_float4(v[0], v[1], v[2], v[3]);
           d4[1] = make_float4(v[4], v[5], v[6], v[7]);
-          lsm = (sg - seg_first) * MB + m;
+          lsm = S.useg[ul] * MB + m;
         }
         // the 16 lanes of a half-warp share one (unit, batch row)
 #pragma unroll
@@ -456,17 +474,19 @@ __global__ void __launch_bounds__(kIT, 2)
 
     // per-slot weights 2^(17 - 8 digit - s) and per-segment sums of the quantised v, read
     // by the drains below
-    if (threadIdx.x < nls * kMaxSlots) {
-      const int ls = threadIdx.x / kMaxSlots, n = threadIdx.x - ls * kMaxSlots;
-      const int m = n / 3, dg = n - 3 * m;
-      float f1 = 0.f, f2 = 0.f;
-      if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
-      S.wsl[threadIdx.x] = f1 * f2;  // powers of two: the product is exact
-    } else if (threadIdx.x - nls * kMaxSlots < nls * MB) {
-      const int i = threadIdx.x - nls * kMaxSlots;
-      float f1, f2;
-      pow2_pair(-fixed_shift(__uint_as_float(S.xmax[i])), f1, f2);
-      S.ssf[i] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[i]))) * f1) * f2;
+    for (int i = threadIdx.x; i < nls * (kMaxSlots + MB); i += kIT) {
+      if (i < nls * kMaxSlots) {
+        const int ls = i / kMaxSlots, n = i - ls * kMaxSlots;
+        const int m = n / 3, dg = n - 3 * m;
+        float f1 = 0.f, f2 = 0.f;
+        if (m < MB) pow2_pair(17 - 8 * dg - fixed_shift(__uint_as_float(S.xmax[ls * MB + m])), f1, f2);
+        S.wsl[i] = f1 * f2;  // powers of two: the product is exact
+      } else {
+        const int j = i - nls * kMaxSlots;
+        float f1, f2;
+        pow2_pair(-fixed_shift(__uint_as_float(S.xmax[j])), f1, f2);
+        S.ssf[j] = (static_cast<float>(static_cast<double>(static_cast<long long>(S.vsum[j]))) * f1) * f2;
+      }
     }
     __syncthreads();
 
@@ -828,17 +848,25 @@ int pass_slots(int tiles, int ncl, int units, int C, int BPT, int u_split) {
   return need;
 }
 
-int max_segments_per_cta_i(int units, int C, const int* seg_unit0, int nseg) {
-  auto seg_of = [&](int u) {
-    int s = 0;
-    for (int k = 1; k < nseg; ++k)
-      if (u >= seg_unit0[k]) s = k;
-    return s;
+// Largest number of (segment, row-scale group) parts one CTA's unit range touches.
+int max_parts_per_cta(const ImmaShape& sh, int C) {
+  auto part_of = [&](int u) {
+    int part = 0, s = 0;
+    for (int k = 0; k < sh.nseg; ++k) {
+      if (u >= sh.seg_unit0[k]) s = k;
+    }
+    for (int k = 0; k < s; ++k) {
+      const int nq = (k + 1 < sh.nseg ? sh.seg_unit0[k + 1] : sh.units) - sh.seg_unit0[k];
+      const int g = sh.seg_rgu ? sh.seg_rgu[k] : 0;
+      part += g > 0 ? (nq + g - 1) / g : 1;
+    }
+    const int g = sh.seg_rgu ? sh.seg_rgu[s] : 0;
+    return part + (g > 0 ? (u - sh.seg_unit0[s]) / g : 0);
   };
   int m = 1;
   for (int r = 0; r < C; ++r) {
-    const int a = r * units / C, b = (r + 1) * units / C;
-    if (b > a) m = std::max(m, seg_of(b - 1) - seg_of(a) + 1);
+    const int a = r * sh.units / C, b = (r + 1) * sh.units / C;
+    if (b > a) m = std::max(m, part_of(b - 1) - part_of(a) + 1);
   }
   return m;
 }
@@ -923,8 +951,7 @@ ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sa
       const int mu_z = z ? (z->units + C - 1) / C : 0;
       const int max_tiles = std::max(mt_y, mt_z);
       const int max_units = std::max(mu_y, mu_z);
-      const int max_lseg = std::max(max_segments_per_cta_i(y.units, C, y.seg_unit0, y.nseg),
-                                    z ? max_segments_per_cta_i(z->units, C, z->seg_unit0, z->nseg) : 1);
+      const int max_lseg = std::max(max_parts_per_cta(y, C), z ? max_parts_per_cta(*z, C) : 1);
       // contributor slots per row and phase (a fused launch has two phases)
       int kcp = pass_slots(tiles_y, ncl_y, y.units, C, 32 / RB, z ? y.seg_unit0[y.nseg - 1] : -1);
       if (z) kcp = std::max(kcp, pass_slots(tiles_z, ncl_z, z->units, C, 32 / RB, -1));

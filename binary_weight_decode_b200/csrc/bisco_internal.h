@@ -32,6 +32,9 @@ struct SegParam {
   int cdt;               // dtype of cscale
   int rdt;               // dtype of rscale
   int cvec, rvec;        // 1 if cscale / rscale are 16-byte aligned (vector loads allowed)
+  int rgu;               // grouped row scales: quads per group (0: one scale per row)
+  int rgstride;          // elements between the row-scale vectors of consecutive groups
+  int part0;             // pass-wide index of the segment's first (segment, group) part
 };
 
 // One launch of the cluster LUT GEMV kernel.
@@ -110,6 +113,7 @@ struct ImmaShape {
   int rows, units;
   const int* seg_unit0;
   int nseg;
+  const int* seg_rgu;  // per segment: quads per row-scale group (0: none); may be null
 };
 // z == nullptr: a plan for one pass; otherwise for the z pass and pass y fused into one
 // launch (pass y's z-reading units run after a bounded wait for the z pass).

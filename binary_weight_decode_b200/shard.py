@@ -42,8 +42,6 @@ def _tile_slice(words, rows, cols, t0, t1):
 
 def shard_rows(layer, rank, world):
     """The host layer of `rank`'s rows (same dataclass as `layer`, out = r1 - r0)."""
-    if getattr(layer, "group", 0):
-        raise NotImplementedError("grouped row scales are not sharded yet")
     r0, r1 = shard_bounds(layer.out, world)[rank]
     t0, t1 = r0 // TILE, (r1 + TILE - 1) // TILE
     rows = r1 - r0
@@ -51,7 +49,10 @@ def shard_rows(layer, rank, world):
     if layer.K:
         bits = np.asarray(layer.bits).reshape(layer.K, -1)
         kw["bits"] = np.stack([_tile_slice(bits[k], layer.out, layer.in_, t0, t1) for k in range(layer.K)])
-        kw["row_scale"] = np.ascontiguousarray(np.asarray(layer.row_scale).reshape(layer.K, layer.out)[:, r0:r1])
+        # [K][out] or, with grouped row scales, [K][out][groups]: the rows are axis 1
+        rs = np.asarray(layer.row_scale)
+        rs = rs.reshape(layer.K, layer.out, -1)[:, r0:r1]
+        kw["row_scale"] = np.ascontiguousarray(rs if getattr(layer, "group", 0) else rs[:, :, 0])
     if layer.rank:
         kw["ut_bits"] = _tile_slice(layer.ut_bits, layer.out, layer.rank, t0, t1)
     if layer.n_sal:

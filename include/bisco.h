@@ -91,7 +91,8 @@ typedef struct {
   int32_t in;               /* input features (columns of W), >= 1                    */
   int32_t num_bases;        /* K >= 0 binary bases                                    */
   const uint32_t* bits;     /* [K][bisco_packed_words(out, in)] sign matrices B_k     */
-  const void* row_scale;    /* [K][out] r_k, dtype scale_dtype                        */
+  const void* row_scale;    /* [K][out] r_k, dtype scale_dtype (row_group == 0);
+                               [K][ceil(in/row_group)][out] with grouped row scales   */
   const void* col_scale;    /* [K][in]  c_k, dtype scale_dtype                        */
   int32_t scale_dtype;      /* BISCO_F32 or BISCO_BF16                                */
   int32_t rank;             /* R >= 0; 0 = no low-rank correction                     */
@@ -103,6 +104,12 @@ typedef struct {
   const int32_t* sal_idx;   /* [n_s] strictly ascending column indices in [0, in)     */
   const int8_t* sal_q;      /* [out][sal_stride] int8 values q[o][t]                  */
   const float* sal_scale;   /* [n_s] per-column scales s_t                            */
+  int32_t row_group;        /* g >= 0: 0 = one row scale per (base, row); g > 0 = one
+                               per (base, row, group of g input columns), "FluxBin"
+                               Sec. 3.1: W_k[o][i] = r_k[i/g][o] c_k[i] (2b - 1).
+                               The kernels take g a multiple of 128 (else
+                               BISCO_ERR_UNSUPPORTED); grouped layers run on the
+                               integer tensor-core kernel in chunks of up to 8 rows */
 } bisco_layer;
 
 /*
@@ -256,6 +263,49 @@ typedef struct {
  * CUDA failure; the graph is released before returning.
  */
 bisco_status bisco_bench(const bisco_bench_args* args, bisco_bench_result* result);
+
+/*
+ * Offline quantisers (device, fp64). They produce the weight format above from dense
+ * weights; nothing in bisco_gemv depends on them.
+ *
+ * bisco_fluxbin_signs: joint binary signs of Kb bases for fixed magnitudes ("FluxBin",
+ * Sec. 3.1, Decoupled Row-Column Binary Bases: M^(k) = alpha_r^(k) alpha_c^(k)T, all 2^Kb
+ * sign combinations evaluated). Element (o, i) takes the combination c (bit k of c set:
+ * base k is +1) with the smallest (W[o][i] - sum_k s_k r_k c_k)^2, the first c on ties.
+ *  W:         device, [rows][cols] row-major fp64.
+ *  row_scale: device fp64, [Kb][rows] (group == 0) or [Kb][ceil(cols/group)][rows]
+ *             (one row scale per group of `group` columns, the layout bisco_layer uses).
+ *  col_scale: device fp64, [Kb][cols].
+ *  bits:      device, Kb * bisco_packed_words(rows, cols) words, written in full in the
+ *             packed layout (base k at word offset k * bisco_packed_words(rows, cols)).
+ * Asynchronous on `stream`. BISCO_ERR_INVALID_ARG for null pointers, sizes < 1,
+ * Kb outside 1..8 or group < 0; BISCO_ERR_CUDA if the launch fails.
+ */
+bisco_status bisco_fluxbin_signs(const double* W, int64_t rows, int64_t cols, int32_t Kb, const double* row_scale,
+                                 const double* col_scale, int32_t group, uint32_t* bits, void* stream);
+
+/*
+ * bisco_biloco_decompose: binary low-rank decomposition W ~ sum_j alpha_j u_j v_j^T
+ * ("BiLoCo: Binary Low-Rank Corrections for Post-Training Quantization", "Finding the
+ * sign vectors"). For j = 0 .. rank-1 on the residual R (initially W): v = v0[j], then
+ * `rounds` times u = sign(R v), v = sign(R^T u) (a zero sum takes +1); the greedy
+ * coefficient alpha_j = u^T R v / (rows cols); R -= alpha_j u v^T. Then the joint refit:
+ * the least-squares coefficients of the chosen sign pairs, G alpha = b with
+ * G_ij = (u_i . u_j)(v_i . v_j) and b_j = u_j^T W v_j, solved by Gaussian elimination
+ * with partial pivoting (G must be nonsingular: distinct sign pairs).
+ *  W:      device [rows][cols] fp64 (not modified).
+ *  v0:     device [rank][cols] int8, starting signs, each +1 or -1.
+ *  U:      device [rows][rank] int8 (+-1), column j = u_j.   V: device [rank][cols] int8.
+ *  alpha_greedy, alpha_refit: device [rank] fp64.
+ *  ws:     device workspace of bisco_biloco_workspace_size bytes (the residual and the
+ *          normal equations).
+ * Asynchronous on `stream` (launches from the host thread, in order). Errors as above,
+ * BISCO_ERR_WORKSPACE for a short workspace; rank <= 4096.
+ */
+bisco_status bisco_biloco_workspace_size(int64_t rows, int64_t cols, int32_t rank, size_t* bytes);
+bisco_status bisco_biloco_decompose(const double* W, int64_t rows, int64_t cols, int32_t rank, int32_t rounds,
+                                    const int8_t* v0, int8_t* U, int8_t* V, double* alpha_greedy,
+                                    double* alpha_refit, void* ws, size_t ws_bytes, void* stream);
 
 /* Static string naming a status code. */
 const char* bisco_status_string(bisco_status status);

@@ -86,7 +86,7 @@ class Layer:
     name: str = ""
     extra: dict = field(default_factory=dict)
     # 0: one row scale per (base, row); g > 0: one per (base, row, group of g input
-    # columns), row_scale [K, out, ceil(in/g)] (grouped row scales: oracle only so far)
+    # columns), row_scale [K, out, ceil(in/g)] ("FluxBin" Sec. 3.1 grouped row scales)
     group: int = 0
 
     @property

@@ -63,13 +63,16 @@ def test_max_without_process_group_is_identity():
     assert _bench().max_over_ranks(3.25, None, "cpu") == 3.25
 
 
-@pytest.mark.parametrize("M,rank,bf16,expected", [
-    (1, 0, True, 1), (1, 256, True, 2), (8, 0, True, 1), (9, 0, True, 2), (16, 0, True, 2),
-    (32, 0, True, 1), (33, 0, True, 1), (128, 256, True, 2), (130, 0, True, 2), (160, 0, True, 2),
-    (190, 0, True, 2), (64, 0, False, 8), (31, 0, True, 4),
-])
-def test_launch_schedule(M, rank, bf16, expected):
-    assert _bench().launches_per_gemv(M, rank, bf16) == expected
+def test_decoder_stream_matrices():
+    # the decoder7b workload streams, per layer, the seven Llama-7B matrix shapes in layer
+    # order with two bases and a rank-256 correction each (1,714,176,000 algorithmic bytes
+    # per 32-layer stream at M=1, the figure the workload table gives)
+    b = _bench()
+    mats = b.base_matrices("decoder7b", 1)
+    assert [(L.out, L.in_) for (L, _) in mats] == [(4096, 4096)] * 4 + [(11008, 4096)] * 2 + [(4096, 11008)]
+    assert all(L.K == 2 and L.rank == 256 and L.n_sal == 0 for (L, _) in mats)
+    total = sum(b.algorithmic_bytes(L, 1, 2, 2) for (L, _) in mats) * b.DECODER_LAYERS
+    assert total == 1_714_176_000
 
 
 def test_reference_arm_prints_one_contract_line():

@@ -80,9 +80,14 @@ def test_gemv_rejects_bad_arguments_before_touching_the_device():
     assert bw.bisco_status_string(bw.BISCO_ERR_WORKSPACE) == "BISCO_ERR_WORKSPACE"
 
 
-def test_grouped_row_scales_are_refused_by_the_binding():
-    # the C ABI carries one row scale per (base, row): a grouped layer must not be uploaded
-    from synth import make_layer
-    L = make_layer(0, (8,), 64, 256, 2, "bf16", group=128)
-    with pytest.raises(NotImplementedError):
-        bw.DeviceLayer(L)
+def test_row_group_field_and_negative_group():
+    # bisco_layer ends with row_group (0 = one row scale per row); a negative group is
+    # refused before anything touches the device
+    hdr = open(os.path.join(ROOT, "include", "bisco.h")).read()
+    body = hdr[hdr.index("typedef struct {", hdr.index("One layer.")):hdr.index("} bisco_layer;")]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)  # drop comments
+    declared = re.findall(r"(\w+)\s*;", body)  # field names in declaration order
+    assert [n.rstrip("_") for n, _ in bw.bisco_layer._fields_] == declared
+    assert declared[-1] == "row_group"
+    L = bw.bisco_layer(out=10, in_=10, num_bases=0, row_group=-1)
+    assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG

@@ -53,10 +53,14 @@ def test_shards_hold_the_row_slices_of_the_layer(world):
         assert np.allclose(oracle.gemv(S, X, "bf16"), Y[:, r0:r1], rtol=1e-12, atol=0)
 
 
-def test_grouped_layers_are_not_sharded_yet():
-    L = make_layer(0, (611,), 64, 256, 1, "bf16", group=128)
-    with pytest.raises(NotImplementedError):
-        shard.shard_rows(L, 0, 2)
+@pytest.mark.parametrize("world", [2, 3])
+def test_grouped_layers_shard_by_rows(world):
+    # grouped row scales [K][out][groups] are cut along the rows like everything else
+    L = make_layer(0, (611,), 100, 300, 2, "bf16", group=128)
+    W = oracle.reconstruct(L)
+    for rank, (r0, r1) in enumerate(shard.shard_bounds(L.out, world)):
+        S = shard.shard_rows(L, rank, world)
+        assert np.array_equal(oracle.reconstruct(S), W[r0:r1])
 
 
 def _free_port():
