@@ -238,6 +238,8 @@ def main():
     ap.add_argument("--workload", default="attn4096", choices=sorted(WORKLOADS))
     ap.add_argument("--M", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-group", action="store_true",
+                    help="decoder7b: one bisco_gemv per matrix instead of one bisco_gemv_group for q/k/v and gate/up")
     ap.add_argument("--calls", type=int, default=0,
                     help="profiling case: run this many plain bisco_gemv calls on one weight copy and exit")
     args = ap.parse_args()
@@ -295,17 +297,29 @@ def main():
     # S distinct device copies of every base matrix: same values, separate HBM buffers
     first = [bw.DeviceLayer(L) for (L, _) in mats]
     dls = [[d] + [d.clone() for _ in range(S - 1)] for d in first]
+    grouped = WORKLOADS[args.workload][1] is None and not args.no_group
+    if grouped:  # q/k/v read one x, gate/up another (as in a decoder layer)
+        mats = [(L, mats[0][1]) if b in (1, 2) else (L, mats[4][1]) if b == 5 else (L, X)
+                for b, (L, X) in enumerate(mats)]
     xs = [dev_x(X) for (_, X) in mats]
     Yd = [torch.empty((S, M, L.out), dtype=y_dtype, device="cuda") for (L, _) in mats]
-    ws = bw.alloc_workspace(first, M)
+    groups = [[0, 1, 2], [3], [4, 5], [6]] if grouped else [[b] for b in range(len(mats))]
+    need = [bw.bisco_workspace_size(d, M) for d in first]
+    need += [bw.bisco_group_workspace_size([first[b] for b in g], M) for g in groups if len(g) > 1]
+    ws = torch.empty(max(need), dtype=torch.uint8, device="cuda")
+    bw.bisco_workspace_init(ws)
     ws_bytes = ws.numel() * ws.element_size()
     xcode = bw.BISCO_BF16 if xdt == "bf16" else bw.BISCO_F32
-    kinds = [bw.bisco_plan_kernels(d, M, xcode, ws_bytes) for d in first]
+    kinds = [bw.bisco_plan_group_kernels([first[b] for b in g], M, xcode, ws_bytes) if len(g) > 1
+             else bw.bisco_plan_kernels(first[g[0]], M, xcode, ws_bytes) for g in groups]
 
     def stream_once(stream):
         for i in range(S):
-            for b in range(len(mats)):
-                bw.bisco_gemv(dls[b][i], xs[b][1], Yd[b][i], ws, stream=stream)
+            for g in groups:
+                if len(g) == 1:
+                    bw.bisco_gemv(dls[g[0]][i], xs[g[0]][1], Yd[g[0]][i], ws, stream=stream)
+                else:
+                    bw.bisco_gemv_group([dls[b][i] for b in g], xs[g[0]][1], [Yd[b][i] for b in g], ws, stream=stream)
 
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -397,6 +411,8 @@ def main():
                    "l2": f"inputs larger than L2: each step streams {S * len(mats)} distinct weight copies "
                          f"({S * nbytes / 2 ** 20:.0f} MiB > 3x L2)",
                    "kernels_per_gemv": kinds if len(mats) > 1 else kinds[0],
+                   "grouped_calls": [[["q", "k", "v", "o", "gate", "up", "down"][b] for b in g] for g in groups]
+                   if len(mats) > 1 else None,
                    "parallelism": f"replicas x{world} (no collective)"},
         "us_per_gemv": round(us_per_gemv, 4),
         "us_per_step": round(ms * 1000.0 / args.steps, 2),

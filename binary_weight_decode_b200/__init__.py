@@ -33,6 +33,7 @@ EXPORTED = [
     "bisco_gemv", "bisco_sync_status", "bisco_bench", "bisco_status_string", "bisco_gemv_noalloc",
     "bisco_set_path_policy", "bisco_plan_kernels", "bisco_debug_set_wait_test",
     "bisco_fluxbin_signs", "bisco_biloco_workspace_size", "bisco_biloco_decompose",
+    "bisco_group_workspace_size", "bisco_gemv_group", "bisco_plan_group_kernels",
 ]
 
 
@@ -93,6 +94,15 @@ _lib.bisco_plan_kernels.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32,
 _lib.bisco_plan_kernels.restype = ctypes.c_int32
 _lib.bisco_debug_set_wait_test.argtypes = [ctypes.c_int32, ctypes.c_uint64]
 _lib.bisco_debug_set_wait_test.restype = ctypes.c_int
+_lib.bisco_group_workspace_size.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.POINTER(ctypes.c_size_t)]
+_lib.bisco_group_workspace_size.restype = ctypes.c_int
+_lib.bisco_gemv_group.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32, _P, ctypes.c_int32, ctypes.c_int32,
+                                  ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32, _P, ctypes.c_size_t, _P]
+_lib.bisco_gemv_group.restype = ctypes.c_int
+_lib.bisco_plan_group_kernels.argtypes = [ctypes.POINTER(bisco_layer), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                          ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+_lib.bisco_plan_group_kernels.restype = ctypes.c_int32
 _lib.bisco_fluxbin_signs.argtypes = [_P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _P, _P, ctypes.c_int32, _P, _P]
 _lib.bisco_fluxbin_signs.restype = ctypes.c_int
 _lib.bisco_biloco_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
@@ -354,3 +364,47 @@ def bisco_biloco_decompose(W, v0, rounds=5, stream=None):
     _check(_lib.bisco_biloco_decompose(p(W), rows, cols, rank, int(rounds), p(v0), p(U), p(V), p(ag), p(ar), p(ws),
                                        int(n.value), _stream_ptr(stream)), "bisco_biloco_decompose")
     return U, V, ag, ar
+
+
+def _layer_array(layers):
+    arr = (bisco_layer * len(layers))()
+    for i, L in enumerate(layers):
+        arr[i] = _desc(L)
+    return arr
+
+
+def bisco_group_workspace_size(layers, M: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_lib.bisco_group_workspace_size(_layer_array(layers), len(layers), M, ctypes.byref(n)),
+           "bisco_group_workspace_size")
+    return int(n.value)
+
+
+def alloc_group_workspace(layers, M: int, device="cuda"):
+    """Zero-initialised workspace for bisco_gemv_group over `layers` at batch M."""
+    torch = _torch()
+    ws = torch.empty(bisco_group_workspace_size(layers, M), dtype=torch.uint8, device=device)
+    bisco_workspace_init(ws)
+    return ws
+
+
+def bisco_gemv_group(layers, X, Ys, ws, stream=None):
+    """Ys[j][M, out_j] = X[M, in] @ W_j^T for layers sharing X, in one call."""
+    M = X.shape[0] if X.dim() == 2 else 1
+    ptrs = (ctypes.c_void_p * len(Ys))(*[y.data_ptr() for y in Ys])
+    ydt = _dtype_code(Ys[0])
+    if any(_dtype_code(y) != ydt for y in Ys):
+        raise BiscoError(BISCO_ERR_INVALID_ARG, "bisco_gemv_group")
+    _check(_lib.bisco_gemv_group(_layer_array(layers), len(layers), ctypes.c_void_p(X.data_ptr()), _dtype_code(X), M,
+                                 ptrs, ydt, ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+                                 _stream_ptr(stream)), "bisco_gemv_group")
+    return Ys
+
+
+def bisco_plan_group_kernels(layers, M: int, x_dtype: int, ws_bytes: int) -> list:
+    cap = 256
+    buf = (ctypes.c_int32 * cap)()
+    n = int(_lib.bisco_plan_group_kernels(_layer_array(layers), len(layers), M, x_dtype, ws_bytes, buf, cap))
+    if n < 0:
+        raise BiscoError(BISCO_ERR_INVALID_ARG, "bisco_plan_group_kernels")
+    return [int(buf[i]) for i in range(min(n, cap))]

@@ -116,13 +116,16 @@ Layout layout_for(const bisco_layer* L, int MB, int dev) {
   const SegList sy = segs_y(L);
   lo.py = make_plan(L->out, sy.units, sy.unit0, sy.nseg, MB, L->n_sal, sms, lim);
   const ImmaShape ys{L->out, sy.units, sy.unit0, sy.nseg, sy.rgu};
-  lo.iy = make_imma_plan(ys, nullptr, MB, L->n_sal, lim);
+  const ImmaRole ry{ys, L->n_sal, -1};
+  lo.iy = make_imma_plan(&ry, 1, MB, lim);
   if (lo.has_z) {
     const int z0 = 0;
     lo.pz = make_plan(L->rank, quads(L->in), &z0, 1, MB, 0, sms, lim);
     const ImmaShape zs{L->rank, quads(L->in), &z0, 1, nullptr};
-    lo.iz = make_imma_plan(zs, nullptr, MB, 0, lim);
-    lo.ifz = make_imma_plan(ys, &zs, MB, L->n_sal, lim);
+    const ImmaRole rz{zs, 0, -1};
+    lo.iz = make_imma_plan(&rz, 1, MB, lim);
+    const ImmaRole rf[2] = {rz, ImmaRole{ys, L->n_sal, sy.unit0[sy.nseg - 1]}};
+    lo.ifz = make_imma_plan(rf, 2, MB, lim);
   }
   lo.off_z = kStatusBytes;
   lo.total = lo.off_z + align256(lo.has_z ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
@@ -173,11 +176,30 @@ void fill_plan(PassParam& P, const Plan& pl) {
   P.max_lseg = pl.max_lseg; P.col_stride_bytes = pl.col_stride_bytes;
 }
 
-// ncl: the clusters of this pass (a fused launch splits its grid between two passes,
-// which share the plan's shared-memory maxima)
+// ncl: the clusters of this pass (a launch with several roles splits its grid between
+// them; they share the plan's shared-memory maxima)
 void fill_imma(PassParam& P, const ImmaPlan& pl, int ncl) {
   P.C = pl.C; P.ncl = ncl; P.max_tiles = pl.max_tiles; P.max_units = pl.max_units;
   P.max_lseg = pl.max_lseg; P.col_stride_bytes = 0;
+}
+
+// One integer launch of n passes in plan order: zsrc[r] is the role whose z role r reads
+// (-1: none), is_z[r] marks the roles that compute a z.
+cudaError_t run_imma(PassParam* passes, const int* zsrc, const int* is_z, int n, const ImmaPlan& pl, cudaStream_t s,
+                     const ImmaDebug* dbg) {
+  ImmaLaunch L{};
+  L.rt.nroles = n;
+  int c = 0;
+  for (int r = 0; r < n; ++r) {
+    fill_imma(passes[r], pl, pl.ncl[r]);
+    L.pass[r] = passes[r];
+    L.rt.cl0[r] = c;
+    c += pl.ncl[r];
+    L.rt.zsrc[r] = zsrc ? zsrc[r] : -1;
+    L.rt.is_z[r] = is_z ? is_z[r] : 0;
+  }
+  L.rt.cl0[n] = c;
+  return launch_imma(L, pl, s, true, dbg);
 }
 
 
@@ -466,9 +488,9 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       PassParam pz{}, py{};
       pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);
       pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
-      fill_imma(pz, ch.lo.ifz, ch.lo.ifz.ncl_z);
-      fill_imma(py, ch.lo.ifz, ch.lo.ifz.ncl);
-      if (launch_imma(&pz, py, ch.lo.ifz, s, true, &dbg) != cudaSuccess) return BISCO_ERR_CUDA;
+      PassParam both[2] = {pz, py};
+      const int zsrc[2] = {-1, 0}, is_z[2] = {1, 0};
+      if (run_imma(both, zsrc, is_z, 2, ch.lo.ifz, s, &dbg) != cudaSuccess) return BISCO_ERR_CUDA;
       continue;
     }
     if (L->rank > 0) {
@@ -478,8 +500,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
       if (ch.tc) {
         e = launch_tc(pz, ch.tz, s, &dbg);
       } else if (ch.imma) {
-        fill_imma(pz, ch.lo.iz, ch.lo.iz.ncl);
-        e = launch_imma(nullptr, pz, ch.lo.iz, s, true, &dbg);
+        e = run_imma(&pz, nullptr, nullptr, 1, ch.lo.iz, s, &dbg);
       } else {
         fill_plan(pz, ch.lo.pz);
         e = launch_pass(pz, ch.lo.pz, s, true);
@@ -492,8 +513,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
     if (ch.tc) {
       e = launch_tc(py, ch.ty, s, &dbg);
     } else if (ch.imma) {
-      fill_imma(py, ch.lo.iy, ch.lo.iy.ncl);
-      e = launch_imma(nullptr, py, ch.lo.iy, s, true, &dbg);
+      e = run_imma(&py, nullptr, nullptr, 1, ch.lo.iy, s, &dbg);
     } else {
       fill_plan(py, ch.lo.py);
       e = launch_pass(py, ch.lo.py, s, true);
@@ -501,6 +521,201 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
     if (e != cudaSuccess) return BISCO_ERR_CUDA;
   }
   return BISCO_OK;
+}
+
+// ---- layers that share x in one launch ------------------------------------------
+
+namespace {
+
+constexpr int kMaxGroup = 3;
+
+// Workspace of a group call: the status region and z of one 8-row chunk for every layer.
+size_t group_ws_need(const bisco_layer* Ls, int n) {
+  size_t b = kStatusBytes;
+  for (int j = 0; j < n; ++j) b += align256(Ls[j].rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * Ls[j].rank * 4 : 0);
+  return b;
+}
+
+bisco_status validate_group(const bisco_layer* Ls, int32_t n) {
+  if (!Ls || n < 1 || n > kMaxGroup) return BISCO_ERR_INVALID_ARG;
+  for (int j = 0; j < n; ++j) {
+    const bisco_status st = validate_layer(&Ls[j]);
+    if (st != BISCO_OK) return st;
+    if (Ls[j].in != Ls[0].in) return BISCO_ERR_INVALID_ARG;
+  }
+  return BISCO_OK;
+}
+
+// The integer plan of a group at batch block MB: z roles of the layers with a correction
+// first, then the output roles (cached by shapes).
+struct GroupPlan {
+  ImmaPlan plan;
+  int n_roles;
+  int layer_of[kMaxRoles];  // layer of each role
+  int zrole[kMaxRoles];     // output role: role of its z, or -1
+  int is_z[kMaxRoles];
+};
+
+GroupPlan group_plan(const bisco_layer* Ls, int n, int MB, int dev) {
+  struct Key {
+    int dev, MB, n, v[kMaxGroup][6];
+    bool operator==(const Key& o) const {
+      if (dev != o.dev || MB != o.MB || n != o.n) return false;
+      for (int j = 0; j < n; ++j)
+        for (int k = 0; k < 6; ++k)
+          if (v[j][k] != o.v[j][k]) return false;
+      return true;
+    }
+  };
+  struct Entry { Key k; GroupPlan g; };
+  static std::mutex mu;
+  static std::vector<Entry>* cache = new std::vector<Entry>();
+  Key k{};
+  k.dev = dev; k.MB = MB; k.n = n;
+  for (int j = 0; j < n; ++j) {
+    const int vals[6] = {Ls[j].out, Ls[j].in, Ls[j].num_bases, Ls[j].rank, Ls[j].n_sal, Ls[j].row_group};
+    for (int q = 0; q < 6; ++q) k.v[j][q] = vals[q];
+  }
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (const Entry& e : *cache)
+      if (e.k == k) return e.g;
+  }
+  GroupPlan gp{};
+  SegList sy[kMaxGroup];
+  const int z0 = 0;
+  ImmaRole roles[kMaxRoles];
+  int nr = 0;
+  for (int j = 0; j < n; ++j) {
+    sy[j] = segs_y(&Ls[j]);
+    if (Ls[j].rank > 0) {
+      roles[nr] = ImmaRole{ImmaShape{Ls[j].rank, quads(Ls[j].in), &z0, 1, nullptr}, 0, -1};
+      gp.layer_of[nr] = j;
+      gp.is_z[nr] = 1;
+      gp.zrole[nr] = -1;
+      ++nr;
+    }
+  }
+  for (int j = 0; j < n; ++j) {
+    const SegList& q = sy[j];
+    int zr = -1;
+    for (int r = 0; r < nr; ++r)
+      if (gp.is_z[r] && gp.layer_of[r] == j) zr = r;
+    roles[nr] = ImmaRole{ImmaShape{Ls[j].out, q.units, q.unit0, q.nseg, q.rgu}, Ls[j].n_sal,
+                         zr >= 0 ? q.unit0[q.nseg - 1] : -1};
+    gp.layer_of[nr] = j;
+    gp.is_z[nr] = 0;
+    gp.zrole[nr] = zr;
+    ++nr;
+  }
+  gp.n_roles = nr;
+  gp.plan = make_imma_plan(roles, nr, MB, cached_smem_limit(dev));
+  std::lock_guard<std::mutex> g(mu);
+  if (cache->size() > 4096) cache->clear();
+  cache->push_back(Entry{k, gp});
+  return gp;
+}
+
+// Whether a group call runs chunk by chunk as one integer launch (else layer by layer
+// through bisco_gemv): batches below the tensor-core chunk size, a plan that fits, and a
+// policy that allows the integer kernel.
+bool group_launch_ok(const bisco_layer* Ls, int n, int M, int dev) {
+  if (n < 2 || M >= kTcMinBatch || g_policy.load() == BISCO_PATH_LOOKUP_TABLE) return false;
+  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
+    const int Mc = std::min(kMaxBatchChunk, M - m0);
+    if (group_plan(Ls, n, batch_block(Mc), dev).plan.C == 0) return false;
+  }
+  for (int j = 0; j < n; ++j)
+    if (Ls[j].num_bases > 0 && Ls[j].row_group > 0 && Ls[j].row_group % 128 != 0) return false;
+  return true;
+}
+
+}  // namespace
+
+bisco_status bisco_group_workspace_size(const bisco_layer* layers, int32_t n, int32_t M, size_t* bytes) {
+  if (!bytes || M < 1) return BISCO_ERR_INVALID_ARG;
+  const bisco_status st = validate_group(layers, n);
+  if (st != BISCO_OK) return st;
+  size_t b = group_ws_need(layers, n);
+  for (int j = 0; j < n; ++j) b = std::max(b, ws_pref(&layers[j], M));
+  *bytes = b;
+  return BISCO_OK;
+}
+
+bisco_status bisco_gemv_group(const bisco_layer* layers, int32_t n, const void* X, int32_t x_dtype, int32_t M,
+                              void* const* Y, int32_t y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  bisco_status st = validate_group(layers, n);
+  if (st != BISCO_OK) return st;
+  if (M < 0 || !dtype_ok(x_dtype) || !dtype_ok(y_dtype) || !Y) return BISCO_ERR_INVALID_ARG;
+  if (M == 0) return BISCO_OK;
+  if (!X || !aligned16(X)) return BISCO_ERR_INVALID_ARG;
+  for (int j = 0; j < n; ++j)
+    if (!Y[j] || !aligned16(Y[j])) return BISCO_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return BISCO_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
+  if (ws_bytes < group_ws_need(layers, n)) return BISCO_ERR_WORKSPACE;
+  if (!group_launch_ok(layers, n, M, dev)) {
+    // layer by layer, in order, on the same stream and workspace
+    for (int j = 0; j < n; ++j) {
+      st = bisco_gemv(&layers[j], X, x_dtype, M, Y[j], y_dtype, ws, ws_bytes, stream);
+      if (st != BISCO_OK) return st;
+    }
+    return BISCO_OK;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  int* status = reinterpret_cast<int*>(wsb);
+  float* zb[kMaxGroup] = {};
+  size_t off = kStatusBytes;
+  for (int j = 0; j < n; ++j) {
+    zb[j] = reinterpret_cast<float*>(wsb + off);
+    off += align256(layers[j].rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * layers[j].rank * 4 : 0);
+  }
+  const size_t xb = dtype_bytes(x_dtype), yb = dtype_bytes(y_dtype);
+  const ImmaDebug dbg{g_dbg_skip_tile.load(), g_dbg_wait_ns.load()};
+  for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
+    const int Mc = std::min(kMaxBatchChunk, M - m0);
+    const GroupPlan gp = group_plan(layers, n, batch_block(Mc), dev);
+    const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(m0) * layers[0].in * xb;
+    PassParam passes[kMaxRoles];
+    for (int r = 0; r < gp.n_roles; ++r) {
+      const bisco_layer* L = &layers[gp.layer_of[r]];
+      passes[r] = PassParam{};
+      if (gp.is_z[r]) {
+        pass_z(L, passes[r], Xc, x_dtype, Mc, zb[gp.layer_of[r]], status);
+      } else {
+        void* Yc = static_cast<unsigned char*>(Y[gp.layer_of[r]]) + static_cast<size_t>(m0) * L->out * yb;
+        pass_y(L, passes[r], Xc, x_dtype, Mc, Yc, y_dtype, zb[gp.layer_of[r]], status);
+      }
+    }
+    if (run_imma(passes, gp.zrole, gp.is_z, gp.n_roles, gp.plan, s, &dbg) != cudaSuccess) return BISCO_ERR_CUDA;
+  }
+  return BISCO_OK;
+}
+
+int32_t bisco_plan_group_kernels(const bisco_layer* layers, int32_t n, int32_t M, int32_t x_dtype, size_t ws_bytes,
+                                 int32_t* kinds, int32_t max_kinds) {
+  if (validate_group(layers, n) != BISCO_OK || M < 0 || !dtype_ok(x_dtype) || max_kinds < 0 ||
+      (max_kinds > 0 && !kinds))
+    return -1;
+  if (M == 0) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (ws_bytes < group_ws_need(layers, n)) return -1;
+  if (group_launch_ok(layers, n, M, dev)) {
+    const int chunks = (M + kMaxBatchChunk - 1) / kMaxBatchChunk;
+    for (int c = 0; c < chunks && c < max_kinds; ++c) kinds[c] = BISCO_KERNEL_INTEGER_MMA;
+    return chunks;
+  }
+  int total = 0;
+  for (int j = 0; j < n; ++j) {
+    const int got = bisco_plan_kernels(&layers[j], M, x_dtype, ws_bytes, kinds ? kinds + std::min(total, max_kinds) : nullptr,
+                                       std::max(0, max_kinds - total));
+    if (got < 0) return -1;
+    total += got;
+  }
+  return total;
 }
 
 bisco_status bisco_set_path_policy(int32_t policy) {

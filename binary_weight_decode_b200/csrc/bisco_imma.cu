@@ -190,17 +190,17 @@ __device__ __forceinline__ void mma_s8s8(int (&c)[4], unsigned a0, unsigned a1, 
 // The low byte of x, sign-extended.
 __device__ __forceinline__ int sext8(int x) { return static_cast<int>(static_cast<signed char>(x & 0xFF)); }
 
-// One launch computes one pass (pz unused, ncl_z = 0), or -- the correction fused into
-// one launch -- both: the first ncl_z clusters compute z = alpha (.) (V x) (pass pz) into
-// the workspace and count their CTAs done on a ready counter; the other clusters compute
-// pass py, first the units that do not read z (the bases), then, after a bounded wait
-// for the counter, the U^T units. Every CTA of the grid is resident before the next
-// kernel on the stream can start, and the z producers wait for nothing but the
-// previous kernel, so the wait always ends; it is bounded anyway (BISCO_ERR_TIMEOUT).
-template <int MB, bool FUSED>
+// One launch computes one pass (MULTI = false: role 0), or several side by side on
+// disjoint clusters (MULTI = true): roles that compute a z = alpha (.) (V x) into the
+// workspace come first and count their CTAs done on a ready counter; an output role that
+// reads a z runs its base units first, then, after a bounded wait for that counter, its
+// U^T units. Every CTA of the grid is resident before the next kernel on the stream can
+// start, and the z roles wait for nothing but the previous kernel, so the wait always
+// ends; it is bounded anyway (BISCO_ERR_TIMEOUT).
+template <int MB, bool MULTI>
 __global__ void __launch_bounds__(kIT, 2)
-    imma_gemv_kernel(const __grid_constant__ PassParam pz, const __grid_constant__ PassParam py, const int ncl_z,
-                     const int kc, const int dbg_skip_tile, const unsigned long long wait_ns) {
+    imma_gemv_kernel(const __grid_constant__ ImmaLaunch L, const int kc, const int dbg_skip_tile,
+                     const unsigned long long wait_ns) {
   constexpr int NG = groups_of(MB);
   constexpr int RB = block_rows(MB);   // rows per work item
   constexpr int RH = RB / 16;          // 16-row MMA blocks per item
@@ -208,11 +208,16 @@ __global__ void __launch_bounds__(kIT, 2)
   extern __shared__ __align__(128) unsigned char smem[];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
-  const int ci_all = blockIdx.x / py.C;
-  constexpr bool fused = FUSED;
-  const bool role_z = FUSED && ci_all < ncl_z;
-  const PassParam& p = role_z ? pz : py;
-  const int ci = role_z ? ci_all : ci_all - ncl_z;
+  const int ci_all = blockIdx.x / L.pass[0].C;
+  int role = 0;
+  if (MULTI)
+    for (int r = 1; r < L.rt.nroles; ++r)
+      if (ci_all >= L.rt.cl0[r]) role = r;
+  constexpr bool fused = MULTI;
+  const bool role_z = MULTI && L.rt.is_z[role] != 0;
+  const int zsrc = MULTI ? L.rt.zsrc[role] : -1;  // the role whose z this output role reads
+  const PassParam& p = L.pass[role];
+  const int ci = ci_all - (MULTI ? L.rt.cl0[role] : 0);
   const int t0 = ci * p.tiles / p.ncl, t1 = (ci + 1) * p.tiles / p.ncl, nt = t1 - t0;
   const int u0 = rank * p.units / p.C, u1 = (rank + 1) * p.units / p.C, nu = u1 - u0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -224,8 +229,10 @@ __global__ void __launch_bounds__(kIT, 2)
   const ISmem S = icarve(smem, p, MB, kc);
   const int rows_c = nt * 32;
   const int msh = msh_of(p.max_tiles, p.C);
-  int* const z_ready = p.status + 32;  // counters in the workspace's status region
-  int* const z_done = p.status + 33;
+  // counters in the workspace's status region: words 32 + r are the ready counters of
+  // the z roles, word 48 counts the grid's CTAs done
+  int* const z_ready = p.status + 32 + (role_z ? role : max(zsrc, 0));
+  int* const z_done = p.status + 48;
 
   // ---- set-up: barriers, unit table, counters ----
   for (int i = threadIdx.x; i < nt; i += kIT) dev::mbar_init(S.bar + i, 1);
@@ -345,10 +352,11 @@ __global__ void __launch_bounds__(kIT, 2)
 
   // ---- phases: the units that do not read z, then (fused launches) the U^T units ----
   int uT = nu;  // first local unit of a z-reading segment
-  if (fused && !role_z)
+  const bool waits = fused && zsrc >= 0;  // an output role that reads a z
+  if (waits)
     for (int ls = 0; ls < nls; ++ls)
       if (p.seg[S.lsinfo[ls].x].xsrc == 1) { uT = min(uT, S.lsstart[ls]); }
-  const int nph = (fused && !role_z && uT < nu && uT > 0) ? 2 : 1;
+  const int nph = (waits && uT < nu && uT > 0) ? 2 : 1;
   const int kcp = kc / (fused ? 2 : 1);  // contributor slots per phase
   bool ok = true;
   bool waited = false;  // this thread has completed the cluster barrier started above
@@ -356,12 +364,12 @@ __global__ void __launch_bounds__(kIT, 2)
     const int pa = nph == 1 ? 0 : (ph == 0 ? 0 : uT);
     const int pb = nph == 1 ? nu : (ph == 0 ? uT : nu);
     const int nun = pb - pa;
-    const bool reads_z = fused && !role_z && (ph == 1 || (nph == 1 && uT == 0));
+    const bool reads_z = waits && (ph == 1 || (nph == 1 && uT == 0));
     if (reads_z) {
       // z is read from here on: wait (bounded) until every z-producing CTA has counted
       // its stores
       if (threadIdx.x == 0) {
-        const int target = ncl_z * p.C;
+        const int target = (L.rt.cl0[zsrc + 1] - L.rt.cl0[zsrc]) * p.C;
         const unsigned long long end = dev::global_ns() + wait_ns;
         bool ready = false;
         while (!ready) {
@@ -760,11 +768,10 @@ __global__ void __launch_bounds__(kIT, 2)
         __threadfence();  // z visible device-wide before it is counted
         atomicAdd(z_ready, 1);
       }
-      // the last CTA of the grid to get here resets both counters for the next launch:
-      // every consumer counted itself after its wait, so nobody reads them any more
-      const int total = gridDim.x;
-      if (atomicAdd(z_done, 1) == total - 1) {
-        atomicExch(z_ready, 0);
+      // the last CTA of the grid to get here returns the counters to zero for the next
+      // launch: every consumer counted itself after its wait, so nobody reads them any more
+      if (atomicAdd(z_done, 1) == static_cast<int>(gridDim.x) - 1) {
+        for (int r = 0; r < L.rt.nroles; ++r) atomicExch(p.status + 32 + r, 0);
         atomicExch(z_done, 0);
       }
     }
@@ -906,18 +913,16 @@ cudaError_t imma_ensure_attrs() {
 // the masks add about half as much again: measured 237 cycles per 32 x 128 block and
 // warp with 8 warps per SM), the B-fragment writes (about 60 lane operations per task of
 // 4 columns and one batch row, 64 lanes per clock for one CTA), a fixed cost for the
-// cluster reduction (and for the second phase of a fused launch), plus a fixed cost when
-// the CTA takes more than half of the SM's shared memory (the next kernel's CTA then
-// cannot be resident beside it) -- among the plans whose shared memory fits. The grid
-// holds as many clusters as fit with one CTA per SM; with half an SM or less per CTA the
-// block scheduler still places two CTAs of one launch on some SMs (measured: 120 CTAs on
-// 98 SMs), which those SMs pay for, but exposing the next kernel's prologue costs more.
-// With z given (the correction fused into one launch) the clusters are split between
-// the z pass and pass y in proportion to their work.
+// cluster reduction (and for the z hand-over of a launch with several roles), plus a fixed
+// cost when the CTA takes more than half of the SM's shared memory (the next kernel's CTA
+// then cannot be resident beside it) -- among the plans whose shared memory fits. The
+// grid holds as many clusters as fit with one CTA per SM; with half an SM or less per CTA
+// the block scheduler still places two CTAs of one launch on some SMs (measured: 120 CTAs
+// on 98 SMs), which those SMs pay for, but exposing the next kernel's prologue costs more.
 // C = 0 in the result means no plan fits.
-ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sal, size_t smem_limit) {
+ImmaPlan make_imma_plan(const ImmaRole* roles, int nroles, int MB, size_t smem_limit) {
   ImmaPlan best{};
-  if (imma_ensure_attrs() != cudaSuccess) return best;
+  if (nroles < 1 || nroles > kMaxRoles || imma_ensure_attrs() != cudaSuccess) return best;
   int dev = 0, per_sm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
@@ -925,54 +930,74 @@ ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sa
   // hardware reserves per CTA
   const size_t half = per_sm > 0 ? static_cast<size_t>(per_sm) / 2 - 1024 : smem_limit / 2;
   const int NG = groups_of(MB), RB = block_rows(MB);
-  const int tiles_y = (y.rows + 31) / 32;
-  const int tiles_z = z ? (z->rows + 31) / 32 : 0;
+  int tiles[kMaxRoles], min_units = 1 << 30, n_sal = 0;
+  bool waits = false;
+  for (int r = 0; r < nroles; ++r) {
+    tiles[r] = (roles[r].sh.rows + 31) / 32;
+    min_units = std::min(min_units, roles[r].sh.units);
+    n_sal = std::max(n_sal, roles[r].n_sal);
+    waits = waits || roles[r].u_split >= 0;
+  }
   double best_cost = -1;
   for (int C = 1; C <= kMaxCluster; C *= 2) {
-    if (C > 1 && (C > y.units || (z && C > z->units))) break;
+    if (C > 1 && C > min_units) break;
     // clusters that fit with one CTA of the launch per SM (the query asks for more
     // than half of the SM's shared memory)
     const size_t force = smem_limit / 2 + 1024;
     const int fit = imma_clusters_mb(MB, C, force);
-    if (fit <= 0 || (z && fit < 2)) continue;
-    // z clusters: from the share proportional to the work upwards (a few more z
-    // clusters shrink the largest tile count, and with it shared memory)
-    int nz0 = 0, nz1 = 0;
-    if (z) {
-      const double wz = static_cast<double>(tiles_z) * z->units, wy = static_cast<double>(tiles_y) * y.units;
-      nz0 = std::max(1, std::min({static_cast<int>(fit * wz / (wz + wy) + 0.5), tiles_z, fit - 1}));
-      nz1 = std::min({nz0 + 8, tiles_z, fit - 1});
-    }
-    for (int ncl_z = nz0; ncl_z <= nz1; ++ncl_z) {
-      const int ncl_y = std::max(1, std::min(tiles_y, fit - ncl_z));
-      const int mt_y = (tiles_y + ncl_y - 1) / ncl_y;
-      const int mu_y = (y.units + C - 1) / C;
-      const int mt_z = z ? (tiles_z + ncl_z - 1) / ncl_z : 0;
-      const int mu_z = z ? (z->units + C - 1) / C : 0;
-      const int max_tiles = std::max(mt_y, mt_z);
-      const int max_units = std::max(mu_y, mu_z);
-      const int max_lseg = std::max(max_parts_per_cta(y, C), z ? max_parts_per_cta(*z, C) : 1);
-      // contributor slots per row and phase (a fused launch has two phases)
-      int kcp = pass_slots(tiles_y, ncl_y, y.units, C, 32 / RB, z ? y.seg_unit0[y.nseg - 1] : -1);
-      if (z) kcp = std::max(kcp, pass_slots(tiles_z, ncl_z, z->units, C, 32 / RB, -1));
-      const int kc = kcp * (z ? 2 : 1);
+    if (fit < nroles) continue;
+    int mu[kMaxRoles];
+    for (int r = 0; r < nroles; ++r) mu[r] = (roles[r].sh.units + C - 1) / C;
+    auto load = [&](int r, int n) {  // blocks of the largest CTA share of role r with n clusters
+      return static_cast<double>((tiles[r] + n - 1) / n) * mu[r];
+    };
+    // The roles share the shared-memory maxima (tiles x units of the largest share), so
+    // the split is searched over a cap T on the row tiles of any cluster: every role first
+    // gets the clusters the cap needs, the rest go one at a time to the role with the
+    // heaviest share.
+    int t_hi = 1;
+    for (int r = 0; r < nroles; ++r) t_hi = std::max(t_hi, tiles[r]);
+    for (int T = 1; T <= t_hi; ++T) {
+      int ncl[kMaxRoles], used = 0;
+      for (int r = 0; r < nroles; ++r) {
+        ncl[r] = std::max(1, (tiles[r] + T - 1) / T);
+        used += ncl[r];
+      }
+      if (used > fit) continue;
+      for (int left = fit - used; left > 0; --left) {
+        int pick = -1;
+        for (int r = 0; r < nroles; ++r)
+          if (ncl[r] < tiles[r] && (pick < 0 || load(r, ncl[r]) > load(pick, ncl[pick]))) pick = r;
+        if (pick < 0) break;
+        ++ncl[pick];
+      }
+      int max_tiles = 0, max_units = 0, max_lseg = 1, kcp = 1;
+      double mma = 0;
+      for (int r = 0; r < nroles; ++r) {
+        max_tiles = std::max(max_tiles, (tiles[r] + ncl[r] - 1) / ncl[r]);
+        max_units = std::max(max_units, mu[r]);
+        max_lseg = std::max(max_lseg, max_parts_per_cta(roles[r].sh, C));
+        // contributor slots per row and phase
+        kcp = std::max(kcp, pass_slots(tiles[r], ncl[r], roles[r].sh.units, C, 32 / RB, roles[r].u_split));
+        mma = std::max(mma, load(r, ncl[r]));
+      }
+      const int kc = kcp * (nroles > 1 ? 2 : 1);  // a launch with several roles has two phases
       const size_t need = ismem_bytes(MB, C, max_tiles, max_units, max_lseg, kc, n_sal);
       if (need > smem_limit) continue;
       // kIW warps of a CTA work on kIW blocks at once: 237 / kIW cycles per block and SM
-      const double mma =
-          std::max(static_cast<double>(mt_y) * mu_y, static_cast<double>(mt_z) * mu_z) * NG * 237.0 / kIW;
+      const double cyc = mma * NG * 237.0 / kIW;
       const double bfr = static_cast<double>(max_units) * MB * 32.0 * 60.0 / 64.0;
-      const double red = (C > 1 ? 1500.0 : 300.0) + (z ? 1500.0 : 0.0);
+      const double red = (C > 1 ? 1500.0 : 300.0) + (waits ? 1500.0 : 0.0);
       // a CTA of at most half an SM lets the next kernel's CTA (launched early) be
       // resident beside it and run its prologue during this kernel; a larger one exposes
       // that prologue (measured on the 4096 x 4096 layer: 6.85 us vs 8.08 us per GEMV)
       const bool coresident = need <= half;
-      const double cost = mma + bfr + red + (coresident ? 0.0 : 2500.0);
+      const double cost = cyc + bfr + red + (coresident ? 0.0 : 2500.0);
       if (best_cost < 0 || cost < best_cost) {
         best_cost = cost;
         best.C = C;
-        best.ncl = ncl_y;
-        best.ncl_z = ncl_z;
+        best.nroles = nroles;
+        for (int r = 0; r < nroles; ++r) best.ncl[r] = ncl[r];
         best.max_tiles = max_tiles;
         best.max_units = max_units;
         best.max_lseg = max_lseg;
@@ -985,13 +1010,12 @@ ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sa
   return best;
 }
 
-cudaError_t launch_imma(const PassParam* pz, const PassParam& py, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
+cudaError_t launch_imma(const ImmaLaunch& L, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
                         const ImmaDebug* dbg) {
   const cudaError_t e = imma_ensure_attrs();
   if (e != cudaSuccess) return e;
-  const int ncl_z = pz ? plan.ncl_z : 0;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((plan.ncl + ncl_z) * plan.C);
+  cfg.gridDim = dim3(L.rt.cl0[L.rt.nroles] * plan.C);
   cfg.blockDim = dim3(kIT);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = stream;
@@ -1006,20 +1030,20 @@ cudaError_t launch_imma(const PassParam* pz, const PassParam& py, const ImmaPlan
   cfg.numAttrs = pdl ? 2 : 1;
   const int skip = dbg ? dbg->skip_tile : -1;
   const unsigned long long wait_ns = dbg && dbg->wait_ns ? dbg->wait_ns : kDefaultWaitNs;
-  const PassParam& z = pz ? *pz : py;
+  const bool multi = L.rt.nroles > 1;
   switch (plan.MB) {
     case 1:
-      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
-                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, false>, z, py, 0, plan.nbw, skip, wait_ns);
+      return multi ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, true>, L, plan.nbw, skip, wait_ns)
+                   : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<1, false>, L, plan.nbw, skip, wait_ns);
     case 2:
-      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
-                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, false>, z, py, 0, plan.nbw, skip, wait_ns);
+      return multi ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, true>, L, plan.nbw, skip, wait_ns)
+                   : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<2, false>, L, plan.nbw, skip, wait_ns);
     case 4:
-      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
-                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, false>, z, py, 0, plan.nbw, skip, wait_ns);
+      return multi ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, true>, L, plan.nbw, skip, wait_ns)
+                   : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<4, false>, L, plan.nbw, skip, wait_ns);
     case 8:
-      return ncl_z > 0 ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, true>, z, py, ncl_z, plan.nbw, skip, wait_ns)
-                       : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, false>, z, py, 0, plan.nbw, skip, wait_ns);
+      return multi ? cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, true>, L, plan.nbw, skip, wait_ns)
+                   : cudaLaunchKernelEx(&cfg, imma_gemv_kernel<8, false>, L, plan.nbw, skip, wait_ns);
     default: return cudaErrorInvalidValue;
   }
 }

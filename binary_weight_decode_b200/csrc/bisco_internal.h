@@ -89,12 +89,28 @@ int query_num_sms();
 size_t query_smem_limit();
 
 // Integer tensor-core GEMV (mma.sync u8 x s8) for batch chunks of up to 8 rows.
+// Roles of one integer-kernel launch: passes that run side by side on disjoint clusters.
+// A launch of one role is a plain pass; with several, z passes come first and the output
+// passes that read a z wait (bounded) for its CTAs to count themselves done.
+constexpr int kMaxRoles = 6;  // three layers sharing x, each with a correction
+struct RoleTable {
+  int nroles;
+  int cl0[kMaxRoles + 1];  // first cluster of role r; cl0[nroles] = clusters of the grid
+  int zsrc[kMaxRoles];     // output role: the role computing the z it reads, or -1
+  int is_z[kMaxRoles];     // 1 if the role computes a z (it counts itself ready)
+};
+struct ImmaLaunch {
+  PassParam pass[kMaxRoles];
+  RoleTable rt;
+};
+
 struct ImmaPlan {
-  int C, ncl;            // cluster size (K split) and clusters of the output pass; C == 0: no plan fits
-  int ncl_z;             // clusters of the z pass in a fused launch (0: not fused)
-  int max_tiles;         // 32-row tiles of the largest cluster share
+  int C;                 // cluster size (K split); C == 0: no plan fits
+  int nroles;
+  int ncl[kMaxRoles];    // clusters of each role
+  int max_tiles;         // 32-row tiles of the largest cluster share (over roles)
   int max_units;         // 128-column units of the largest CTA share
-  int max_lseg;          // segments a CTA's unit range touches, at most
+  int max_lseg;          // (segment, row-scale group) parts a CTA's unit range touches, at most
   int nbw;               // partial-sum slots per row and CTA (warps whose items touch one row block)
   int MB;                // batch rows per launch (1, 2, 4 or 8)
   size_t smem;
@@ -115,13 +131,18 @@ struct ImmaShape {
   int nseg;
   const int* seg_rgu;  // per segment: quads per row-scale group (0: none); may be null
 };
-// z == nullptr: a plan for one pass; otherwise for the z pass and pass y fused into one
-// launch (pass y's z-reading units run after a bounded wait for the z pass).
-ImmaPlan make_imma_plan(const ImmaShape& y, const ImmaShape* z, int MB, int n_sal, size_t smem_limit);
-// pz == nullptr: one pass (py); otherwise the fused launch of plan.ncl_z z clusters and
-// plan.ncl output clusters.
-cudaError_t launch_imma(const PassParam* pz, const PassParam& py, const ImmaPlan& plan, cudaStream_t stream, bool pdl,
-                        const ImmaDebug* dbg);
+// One role of a launch: its shape, salient columns, and (output passes reading a z) the
+// first unit of the U^T segment, else -1.
+struct ImmaRole {
+  ImmaShape sh;
+  int n_sal;
+  int u_split;
+};
+// Clusters per role (each at least one, then one at a time to the role with the largest
+// share per cluster), cluster size from a cycle estimate, shared-memory maxima over roles.
+ImmaPlan make_imma_plan(const ImmaRole* roles, int nroles, int MB, size_t smem_limit);
+// L.pass[r] holds role r's pass with the plan's maxima filled in; L.rt its role table.
+cudaError_t launch_imma(const ImmaLaunch& L, const ImmaPlan& plan, cudaStream_t stream, bool pdl, const ImmaDebug* dbg);
 cudaError_t imma_ensure_attrs();
 
 // Tensor-core path (32..128 batch rows per launch): one launch per pass.

@@ -144,6 +144,26 @@ bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype
                         void* Y, int32_t y_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Layers that read the same X (a decoder's q/k/v projections, gate and up) in one call:
+ * Y[j] = X * W_j^T for j < n (1 <= n <= 3, every layer with the same `in`). For batches
+ * below 32 rows each chunk of up to 8 rows runs as ONE integer tensor-core launch whose
+ * clusters are split between the layers (and, for a layer with a correction, between its
+ * z pass and its output pass, as in bisco_gemv), so the dependent chain of a launch is paid
+ * once for the group. Larger batches, or groups whose launch does not fit, run layer by
+ * layer exactly as bisco_gemv (same results within the documented tolerance either way).
+ *  layers: host array of n layers.   X: device [M][in].   Y: host array of n device
+ *  pointers, Y[j] [M][layers[j].out].   ws: at least bisco_group_workspace_size bytes,
+ *  prepared by bisco_workspace_init. Errors as bisco_gemv; BISCO_ERR_INVALID_ARG for n
+ *  outside 1..3 or layers of different `in`.
+ */
+bisco_status bisco_group_workspace_size(const bisco_layer* layers, int32_t n, int32_t M, size_t* bytes);
+bisco_status bisco_gemv_group(const bisco_layer* layers, int32_t n, const void* X, int32_t x_dtype, int32_t M,
+                              void* const* Y, int32_t y_dtype, void* ws, size_t ws_bytes, void* stream);
+/* Launches of bisco_gemv_group, as bisco_plan_kernels reports them for bisco_gemv. */
+int32_t bisco_plan_group_kernels(const bisco_layer* layers, int32_t n, int32_t M, int32_t x_dtype, size_t ws_bytes,
+                                 int32_t* kinds, int32_t max_kinds);
+
+/*
  * Synchronise `stream` and return the device-side status recorded in workspace
  * `ws` by earlier bisco_gemv calls (BISCO_OK if none). A recorded error stays
  * until bisco_workspace_init clears it.
