@@ -1,17 +1,19 @@
-// C ABI front end: argument validation, host packing, workspace sizing and the
-// two-pass launch sequence of bisco_gemv.
+// C ABI front end: argument validation, host packing, workspace sizing and the launch
+// sequence of bisco_gemv and bisco_gemv_group.
 //
 // A layer with a binary low-rank correction ("BiLoCo", "The core idea": the
-// correction is applied as alpha * u * (v . x)) runs as two launches: pass Z computes
+// correction is applied as alpha * u * (v . x)) has two passes: pass Z computes
 // z = alpha (.) (V x) into the workspace, pass Y computes
-// sum_k r_k (.) (B_k (c_k (.) x)) + U^T z + salient term into Y. Pass Y reads z only
-// after griddepcontrol.wait, i.e. after pass Z completed.
+// sum_k r_k (.) (B_k (c_k (.) x)) + U^T z + salient term into Y. On the integer kernel
+// both run in one launch (z clusters first, output clusters wait for them, bounded);
+// on the other kernels as two launches, pass Y reading z after griddepcontrol.wait.
 //
 // The batch is cut into chunks: up to 128 rows per launch on the tensor-core path
-// (tcgen05) when a chunk has at least 32 rows (and the scales are bf16, so that folding
+// (tcgen05) when a chunk has at least 16 rows (and the scales are bf16, so that folding
 // a column scale into the expanded signs is exact), otherwise up to 8 rows per launch on
 // the integer tensor-core kernel (mma.sync, bisco_imma.cu) when its shared-memory plan
-// fits, else on the lookup-table kernels.
+// fits, else on the lookup-table kernels. Single rows of layers without a correction
+// take the lookup-table kernels.
 
 #include <cuda_runtime.h>
 
@@ -161,7 +163,9 @@ size_t ws_need(const bisco_layer* L, int32_t) {
   return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
 }
 size_t ws_pref(const bisco_layer* L, int32_t M) {
-  const int rows = std::max(kMaxBatchChunk, std::min<int>(M, kTcMaxBatch));
+  // z rows of a tensor-core chunk (padded to 16; from 8 batch rows up a chunk may go to
+  // the tensor cores when the integer plan does not fit)
+  const int rows = M < kMaxBatchChunk ? kMaxBatchChunk : std::min<int>((M + 15) / 16 * 16, kTcMaxBatch);
   return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(rows) * L->rank * 4 : 0);
 }
 
@@ -389,7 +393,21 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
                 (batch_block(ch.Mc) >= 2 || policy == BISCO_PATH_INTEGER_MMA || fusable)));
       ch.fused = ch.imma && fusable;
       if (grouped && !ch.imma) return BISCO_ERR_UNSUPPORTED;
-      if (!ch.imma && !plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
+      // a chunk of 8 rows whose integer plan does not fit (large K at 8 batch rows, e.g.
+      // 4096 x 11008 with a rank-256 correction) is faster on the tensor cores, padded to
+      // 16 columns, than on the lookup-table kernels (that layer: 97 us for a 16-row
+      // tensor-core chunk, 110 us per 8-row lookup-table chunk)
+      if (!ch.imma && tc_ok && policy != BISCO_PATH_LOOKUP_TABLE && rem >= kMaxBatchChunk) {
+        const int Mt = std::min(rem, tc_rows);
+        TcPlan tz{}, ty{};
+        if (tc_plans(L, Mt, x_dtype, dev, &tz, &ty)) {
+          ch.tc = true;
+          ch.Mc = Mt;
+          ch.tz = tz;
+          ch.ty = ty;
+        }
+      }
+      if (!ch.tc && !ch.imma && !plans_fit(ch.lo, lim)) return BISCO_ERR_UNSUPPORTED;
     }
     out->push_back(ch);
     m0 += ch.Mc;

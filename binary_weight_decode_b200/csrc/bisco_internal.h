@@ -145,8 +145,8 @@ ImmaPlan make_imma_plan(const ImmaRole* roles, int nroles, int MB, size_t smem_l
 cudaError_t launch_imma(const ImmaLaunch& L, const ImmaPlan& plan, cudaStream_t stream, bool pdl, const ImmaDebug* dbg);
 cudaError_t imma_ensure_attrs();
 
-// Tensor-core path (32..128 batch rows per launch): one launch per pass.
-constexpr int kTcMinBatch = 32;           // smallest batch chunk sent to the tensor cores
+// Tensor-core path (16..128 batch rows per launch): one launch per pass.
+constexpr int kTcMinBatch = 16;           // smallest batch chunk sent to the tensor cores
 constexpr int kTcMaxBatch = 128;          // batch rows per launch
 struct TcPlan {
   int Np;                // batch rows padded to a multiple of 16 (MMA N per part)

@@ -146,7 +146,7 @@ bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype
 /*
  * Layers that read the same X (a decoder's q/k/v projections, gate and up) in one call:
  * Y[j] = X * W_j^T for j < n (1 <= n <= 3, every layer with the same `in`). For batches
- * below 32 rows each chunk of up to 8 rows runs as ONE integer tensor-core launch whose
+ * below 16 rows each chunk of up to 8 rows runs as ONE integer tensor-core launch whose
  * clusters are split between the layers (and, for a layer with a correction, between its
  * z pass and its output pass, as in bisco_gemv), so the dependent chain of a launch is paid
  * once for the group. Larger batches, or groups whose launch does not fit, run layer by
@@ -172,7 +172,7 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
 
 /*
  * Which kernel family runs a batch chunk (process-wide; for tests and diagnostics).
- *  BISCO_PATH_AUTO (default): chunks of 32..128 rows on the tcgen05 tensor-core kernel
+ *  BISCO_PATH_AUTO (default): chunks of 16..128 rows on the tcgen05 tensor-core kernel
  *    (bf16 scales), chunks of 2..8 rows on the integer tensor-core kernel (mma.sync)
  *    when its shared-memory plan fits, single rows of a layer with a correction on the
  *    integer kernel's one-launch form, other single rows and the rest on the
@@ -196,7 +196,7 @@ enum {
   BISCO_KERNEL_LUT_ROWS = 3,      /* lookup tables, warps own row tiles, 4 or 8 rows     */
   BISCO_KERNEL_INTEGER_MMA = 4,   /* int8 tensor cores (mma.sync), <= 8 rows; with a
                                      correction, z and y in one launch                   */
-  BISCO_KERNEL_TENSOR_CORE = 5    /* tcgen05 tensor cores, 32..128 rows                  */
+  BISCO_KERNEL_TENSOR_CORE = 5    /* tcgen05 tensor cores, 16..128 rows                  */
 };
 
 /*
@@ -243,7 +243,7 @@ bisco_status bisco_debug_set_wait_test(int32_t skip_tile, uint64_t wait_ns);
  * make that first call before any stream capture starts. A failed lookup is not cached
  * (the next call retries); a device reset invalidates the cached address.
  * With the fixed array, z fits at most floor(8192 / rank) batch rows, so a batch chunk on
- * the tcgen05 tensor-core kernel (32..128 rows) is limited to floor(8192 / rank / 16) * 16
+ * the tcgen05 tensor-core kernel (16..128 rows) is limited to floor(8192 / rank / 16) * 16
  * rows; layers with rank > 256 run every chunk on the small-batch kernels (correct, slower
  * at large batch than bisco_gemv with its preferred workspace).
  * All calls share the one array: calls that may overlap on the GPU (different streams,

@@ -211,6 +211,16 @@ def test_integer_kernel_wait_gives_up_and_reports_timeout():
     check(Y, oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
 
 
+def test_eight_rows_without_an_integer_plan_take_the_tensor_cores():
+    # the decoder's down projection (4096 x 11008, rank 256) at 8 batch rows: the integer
+    # plan does not fit shared memory, so the chunk runs on the tcgen05 kernel (z, then y)
+    L, X = build(5, 6, 8)
+    assert kinds(L, 8) == [bw.BISCO_KERNEL_TENSOR_CORE] * 2
+    Y = run(L, X, "bf16", "f32")
+    rows = sample_rows(L.out, 128, 70)
+    check(Y[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
+
+
 # ---- the correction in one launch: z handed over inside the grid ------------------
 
 @pytest.mark.parametrize("out,in_,K,rank", [(200, 128, 1, 512), (64, 4096, 2, 64), (4100, 300, 2, 1000),

@@ -1,10 +1,10 @@
-"""GPU parity of the tensor-core path (batch chunks of 32..128 rows) against the oracle.
+"""GPU parity of the tensor-core path (batch chunks of 16..128 rows) against the oracle.
 
-bisco_gemv sends a batch chunk of at least 32 rows to the tensor cores when the layer's
+bisco_gemv sends a batch chunk of at least 16 rows to the tensor cores when the layer's
 scales are bf16: the signs are expanded to bf16 tiles (column scale folded in, exact),
 fp32-valued inputs (the correction's z, salient inputs, fp32 activations) are split into
 high and low bf16 parts, and the products accumulate in fp32. The bars are those of
-tests/test_gemv_gpu.py. Batch sizes straddle the chunk boundaries (32, 128) so that
+tests/test_gemv_gpu.py. Batch sizes straddle the chunk boundaries (16, 128) so that
 mixed schedules (tensor-core chunks followed by lookup-table chunks) are covered too.
 """
 
@@ -38,6 +38,10 @@ CASES = [
     (192, 512, 2, 17, 0.0, 48, "f32", "f32"),       # fp32 activations: split on the bases
     (128, 256, 0, 64, 0.05, 32, "bf16", "f32"),     # correction + salient, no base
     (96, 200, 0, 0, 0.1, 40, "bf16", "f32"),        # salient only
+    (256, 512, 2, 0, 0.0, 16, "bf16", "f32"),       # the smallest tensor-core chunk
+    (300, 700, 2, 24, 0.02, 17, "bf16", "f32"),     # 17 rows: one chunk padded to 32 columns
+    (333, 1000, 2, 40, 0.0, 24, "bf16", "bf16"),
+    (130, 4100, 1, 0, 0.01, 31, "bf16", "f32"),
 ]
 
 
