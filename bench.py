@@ -194,7 +194,18 @@ def cpu_baseline(workload, M, budget_s=12.0):
         if el >= budget_s or n >= 200:
             break
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    # the same oracle on one thread, over a shorter sample
+    from threadpoolctl import threadpool_limits
+    n1, t1 = 0, time.perf_counter()
+    with threadpool_limits(limits=1):
+        while True:
+            oracle.gemv(L, X, xdt)
+            n1 += 1
+            el1 = time.perf_counter() - t1
+            if el1 >= budget_s / 4 or n1 >= 50:
+                break
     return {"value": round(n * nbytes / el / 1e9, 4), "unit": "GB/s", "cores": int(threads),
+            "value_1thread": round(n1 * nbytes / el1 / 1e9, 4),
             "kind": "oracle", "us_per_gemv": el / n * 1e6,
             "sample": f"{n} full fp64 oracle GEMVs of the {workload} layer{' q projection' if spec is None else ''} "
                       f"(M={M}) in {el:.1f} s on {os.cpu_count()} host cores"}
