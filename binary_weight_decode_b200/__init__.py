@@ -194,6 +194,10 @@ class DeviceLayer:
             return torch.from_numpy(a).to(device)
 
         self.host = host
+        if getattr(host, "ref_K", 0):
+            # FluxBin's binary salient refinement bases have no kernel (row-scale groups of s
+            # gathered columns); refuse rather than drop them
+            raise NotImplementedError("the binary salient refinement is not supported by libbisco")
         self.row_group = int(getattr(host, "group", 0) or 0)
         self.out, self.in_, self.K = host.out, host.in_, host.K
         self.rank, self.n_sal = host.rank, host.n_sal

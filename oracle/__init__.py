@@ -14,6 +14,7 @@ from .bisco_oracle import (  # noqa: F401
     dense_correction_storage_bits,
     fluxbin_average_bit_width,
     fluxbin_sign_search,
+    fluxbin_storage_bits,
     fp4_weight_bits,
     gemv,
     gemv_rows,

@@ -162,9 +162,31 @@ def _salient_part_rows(layer, rows):
     return W
 
 
+def _refinement_part_rows(layer, rows):
+    """Binary salient refinement ("FluxBin", Sec. 4, Kb-sS-gG, and the Virtual Columnar
+    Mapping of Sec. 3.2: the sparse salient bases stored as one dense matrix over the
+    gathered columns), rows `rows`: entry (o, idx_t) gains
+    sum_k r^s_k[o][idx_t // g] c^s_k[t] (2b - 1), b = bit (o, t) of refinement base k."""
+    W = np.zeros((len(rows), layer.in_), dtype=np.float64)
+    Ks = getattr(layer, "ref_K", 0)
+    if not Ks:
+        return W
+    g = layer.group
+    idx = np.asarray(layer.ref_idx, dtype=np.int64)
+    n = len(idx)
+    R = decode_values(layer.ref_row_scale, layer.scale_dtype).reshape(Ks, layer.out, -1)
+    C = decode_values(layer.ref_col_scale, layer.scale_dtype).reshape(Ks, n)
+    bits = np.asarray(layer.ref_bits).reshape(Ks, -1)
+    for k in range(Ks):
+        S = unpack_bit_rows(bits[k], layer.out, n, rows)                  # [rows, n]
+        W[:, idx] += R[k][rows][:, idx // g] * S * C[k][None, :]
+    return W
+
+
 def reconstruct_rows(layer, rows):
     rows = np.asarray(rows, dtype=np.int64)
-    return _binary_part_rows(layer, rows) + _correction_part_rows(layer, rows) + _salient_part_rows(layer, rows)
+    return (_binary_part_rows(layer, rows) + _correction_part_rows(layer, rows) + _salient_part_rows(layer, rows) +
+            _refinement_part_rows(layer, rows))
 
 
 def reconstruct(layer):
@@ -301,6 +323,22 @@ def fluxbin_average_bit_width(rows, cols, Kb, Ks, g, s, scale_bits=16):
     bits += (Kb * cols + Ks * n_sal) * scale_bits               # column scales
     bits += n_sal * scale_bits                                  # salient column indices
     return bits / (rows * cols)
+
+
+def fluxbin_storage_bits(layer, scale_bits=16):
+    """Bits a FluxBin-style layer actually stores, counted from its arrays: the global and
+    refinement sign bits (no padding), one row scale per (base, row, group) and one column
+    scale per column of every base, one index per salient column, each scale and index in
+    `scale_bits` bits (the accounting of "FluxBin", Sec. C.2)."""
+    rows, cols, g = layer.out, layer.in_, layer.group
+    ng = -(-cols // g)
+    Ks = getattr(layer, "ref_K", 0)
+    n_ref = len(layer.ref_idx) if Ks else 0
+    bits = layer.K * rows * cols + Ks * rows * n_ref
+    bits += (layer.K + Ks) * rows * ng * scale_bits
+    bits += (layer.K * cols + Ks * n_ref) * scale_bits
+    bits += n_ref * scale_bits
+    return bits
 
 
 def _dtype_bytes(dtype):

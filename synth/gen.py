@@ -18,14 +18,14 @@ Distributions (the binary-weight GEMV workloads):
 """
 
 from dataclasses import dataclass, field
-from typing import Optional, Sequence
+from typing import Optional, Sequence, Tuple
 
 import numpy as np
 
 from .layout import packed_words, zero_padding_bits
 
 # tensor ids inside one layer's key space
-T_BITS, T_ROW, T_COL, T_V, T_UT, T_ALPHA, T_SALQ, T_X, T_OUTLIER = range(9)
+T_BITS, T_ROW, T_COL, T_V, T_UT, T_ALPHA, T_SALQ, T_X, T_OUTLIER, T_REF = range(10)
 
 
 def _rng(seed: int, key: Sequence[int], tensor: int) -> np.random.Generator:
@@ -88,6 +88,15 @@ class Layer:
     # 0: one row scale per (base, row); g > 0: one per (base, row, group of g input
     # columns), row_scale [K, out, ceil(in/g)] ("FluxBin" Sec. 3.1 grouped row scales)
     group: int = 0
+    # binary salient refinement ("FluxBin" Sec. 4, Kb-sS-gG): ref_K bases over the s salient
+    # columns of every group of `group` columns, stored as a dense sign matrix over the
+    # gathered columns (ref_idx ascending), with one row scale per (base, row, group) and
+    # one column scale per (base, salient column); additive on top of the global bases
+    ref_K: int = 0
+    ref_idx: Optional[np.ndarray] = None        # int32 [n_ref]
+    ref_bits: Optional[np.ndarray] = None       # uint32 [ref_K, packed_words(out, n_ref)]
+    ref_row_scale: Optional[np.ndarray] = None  # [ref_K, out, ceil(in/group)] in scale_dtype
+    ref_col_scale: Optional[np.ndarray] = None  # [ref_K, n_ref] in scale_dtype
 
     @property
     def sal_stride(self) -> int:
@@ -111,7 +120,8 @@ def make_activations(seed: int, key: Sequence[int], M: int, n: int, dtype: str,
 
 def make_layer(seed: int, key: Sequence[int], out: int, in_: int, K: int, scale_dtype: str,
                rank: int = 0, sal_frac: float = 0.0, x_for_salience: Optional[np.ndarray] = None,
-               x_dtype: str = "bf16", name: str = "", group: int = 0) -> Layer:
+               x_dtype: str = "bf16", name: str = "", group: int = 0,
+               refine: Optional[Tuple[int, int]] = None) -> Layer:
     bits = random_sign_words(_rng(seed, key, T_BITS), K, out, in_)
     rshape = (K, out, -(-in_ // group)) if group else (K, out)
     row = _as_dtype(np.abs(_rng(seed, key, T_ROW).standard_normal(rshape)) * 0.02, scale_dtype)
@@ -143,4 +153,21 @@ def make_layer(seed: int, key: Sequence[int], out: int, in_: int, K: int, scale_
         L.sal_scale = (cnorm[idx] * 0.02 / 42.0).astype(np.float32)
         L.col_scale = col.copy()
         L.col_scale[:, idx] = 0
+    if refine:
+        Ks, sp = refine
+        if not group:
+            raise ValueError("the salient refinement needs grouped row scales (group > 0)")
+        ng = -(-in_ // group)
+        rng = _rng(seed, key, T_REF)
+        cols = []
+        for j in range(ng):  # s salient columns per group, seeded (the pages choose them by a
+            lo, hi = j * group, min(in_, (j + 1) * group)  # Hessian score: data not available)
+            take = min(sp, hi - lo)
+            cols.extend(sorted(rng.choice(np.arange(lo, hi), size=take, replace=False).tolist()))
+        ref_idx = np.array(cols, dtype=np.int32)
+        L.ref_K = Ks
+        L.ref_idx = ref_idx
+        L.ref_bits = random_sign_words(rng, Ks, out, len(ref_idx))
+        L.ref_row_scale = _as_dtype(np.abs(rng.standard_normal((Ks, out, ng))) * 0.01, scale_dtype)
+        L.ref_col_scale = _as_dtype(np.abs(rng.standard_normal((Ks, len(ref_idx)))) * 0.02, scale_dtype)
     return L

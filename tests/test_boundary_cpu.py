@@ -91,3 +91,12 @@ def test_row_group_field_and_negative_group():
     assert declared[-1] == "row_group"
     L = bw.bisco_layer(out=10, in_=10, num_bases=0, row_group=-1)
     assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+
+
+def test_salient_refinement_is_refused_by_the_binding():
+    # no kernel runs FluxBin's refinement bases: the binding refuses such a layer instead of
+    # silently dropping a term
+    from synth import make_layer
+    L = make_layer(0, (55,), 64, 256, 2, "bf16", group=128, refine=(2, 8))
+    with pytest.raises(NotImplementedError):
+        bw.DeviceLayer(L)

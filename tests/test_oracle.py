@@ -556,3 +556,78 @@ def test_fluxbin_grouped_row_scales_use_the_group_of_each_column():
         blk = slice(j * g, min(cols, (j + 1) * g))
         Sj = oracle.fluxbin_sign_search(W[:, blk], r[:, :, j], c[:, blk])
         assert np.array_equal(S[:, :, blk], Sj)
+
+
+# ---- FluxBin binary salient refinement (Sec. 4, Kb-sS-gG) -----------------------
+
+def _refine_layer(rng, out, in_, g, idx, Ks, signs, r, c, K=0):
+    from synth.gen import Layer
+    L = Layer(out=out, in_=in_, K=K, scale_dtype="f32", bits=np.zeros((K, 1), np.uint32),
+              row_scale=np.zeros((K, out, -(-in_ // g)), np.float32), col_scale=np.zeros((K, in_), np.float32),
+              group=g)
+    L.ref_K = Ks
+    L.ref_idx = np.asarray(idx, np.int32)
+    L.ref_bits = np.stack([oracle.pack_bit_matrix(np.asarray(signs[k], np.int8)) for k in range(Ks)])
+    L.ref_row_scale = np.asarray(r, np.float32)
+    L.ref_col_scale = np.asarray(c, np.float32)
+    return L
+
+
+def test_refinement_all_plus_one_is_a_scaled_gathered_sum():
+    rng = np.random.default_rng(51)
+    out, in_, g, Ks = 5, 24, 8, 2
+    idx = [1, 6, 9, 15, 17, 23]   # two salient columns per group of 8
+    r = np.abs(rng.standard_normal((Ks, out, 3))).astype(np.float32)
+    c = np.abs(rng.standard_normal((Ks, len(idx)))).astype(np.float32)
+    L = _refine_layer(rng, out, in_, g, idx, Ks, [np.ones((out, len(idx)))] * Ks, r, c)
+    x = rng.standard_normal((1, in_)).astype(np.float32)
+    y = oracle.gemv(L, x, "f32")[0]
+    want = np.zeros(out)
+    for o in range(out):
+        for k in range(Ks):
+            for t, i in enumerate(idx):
+                want[o] += float(r[k, o, i // g]) * float(c[k, t]) * float(x[0, i])
+    assert np.allclose(y, want, rtol=1e-12, atol=0)
+
+
+def test_refinement_brute_force_over_every_sign_pattern():
+    import itertools
+    rng = np.random.default_rng(52)
+    out, in_, g, Ks = 2, 8, 4, 2
+    idx = [2, 5]                  # one salient column in each group of 4
+    r = np.abs(rng.standard_normal((Ks, out, 2))).astype(np.float32)
+    c = np.abs(rng.standard_normal((Ks, 2))).astype(np.float32)
+    for pat in itertools.product((-1, 1), repeat=Ks * out * 2):
+        signs = np.array(pat).reshape(Ks, out, 2)
+        L = _refine_layer(rng, out, in_, g, idx, Ks, signs, r, c)
+        W = oracle.reconstruct(L)
+        for o in range(out):
+            for i in range(in_):
+                want = 0.0
+                for k in range(Ks):
+                    for t, j in enumerate(idx):
+                        if j == i:
+                            want += float(r[k, o, j // g]) * float(c[k, t]) * signs[k, o, t]
+                assert W[o, i] == want
+
+
+def test_refinement_is_additive_on_the_global_bases():
+    # zero refinement column scales give exactly the grouped global layer
+    from synth import make_layer
+    L = make_layer(0, (53,), 40, 300, 2, "f32", group=128, refine=(2, 8))
+    W = oracle.reconstruct(L)
+    L0 = make_layer(0, (53,), 40, 300, 2, "f32", group=128)
+    assert not np.array_equal(W, oracle.reconstruct(L0))
+    L.ref_col_scale = np.zeros_like(L.ref_col_scale)
+    assert np.array_equal(oracle.reconstruct(L), oracle.reconstruct(L0))
+
+
+@pytest.mark.parametrize("g,s", [(128, 8), (128, 16), (64, 16)])
+def test_refinement_storage_matches_the_average_bit_width(g, s):
+    # the bits a generated 2b-sS-gG layer stores equal the Sec. C.2 accounting, which
+    # reproduces the page's 2.63 / 2.75 / 3.5 bits
+    from synth import make_layer
+    rows, cols = 64, 1024
+    L = make_layer(0, (54, g, s), rows, cols, 2, "bf16", group=g, refine=(2, s))
+    abw = oracle.fluxbin_storage_bits(L) / (rows * cols)
+    assert abw == oracle.fluxbin_average_bit_width(rows, cols, 2, 2, g, s)
