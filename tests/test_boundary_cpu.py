@@ -100,3 +100,21 @@ def test_salient_refinement_is_refused_by_the_binding():
     L = make_layer(0, (55,), 64, 256, 2, "bf16", group=128, refine=(2, 8))
     with pytest.raises(NotImplementedError):
         bw.DeviceLayer(L)
+
+
+def test_group_call_validates_before_touching_the_device():
+    # bisco_gemv_group: 1..3 layers of one input width; the workspace size is host arithmetic
+    import ctypes
+    a = bw.bisco_layer(out=64, in_=256, num_bases=0)
+    b = bw.bisco_layer(out=32, in_=256, num_bases=0, rank=0)
+    c = bw.bisco_layer(out=32, in_=384, num_bases=0)
+    arr = (bw.bisco_layer * 4)(a, b, a, b)
+    Y = (ctypes.c_void_p * 4)()
+    assert bw._lib.bisco_gemv_group(arr, 0, None, 0, 1, Y, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    assert bw._lib.bisco_gemv_group(arr, 4, None, 0, 1, Y, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    mixed = (bw.bisco_layer * 2)(a, c)
+    assert bw._lib.bisco_gemv_group(mixed, 2, None, 0, 1, Y, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert bw._lib.bisco_group_workspace_size(arr, 2, 1, ctypes.byref(n)) == bw.BISCO_OK
+    assert n.value >= 256  # the status region at least
+    assert bw._lib.bisco_group_workspace_size(mixed, 2, 1, ctypes.byref(n)) == bw.BISCO_ERR_INVALID_ARG
