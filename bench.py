@@ -6,12 +6,15 @@ graph holding S back-to-back GEMVs over S distinct weight copies whose total
 size exceeds 3x the L2 cache, so every GEMV streams its weights from HBM.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bisco|reference]
-                    [--workload attn4096|mlp_gate_up|mlp_down|lowrank5120|cfg1|decoder7b] [--M m]
+                    [--workload attn4096|mlp_gate_up|mlp_down|lowrank5120|cfg1|decoder7b|
+                                fluxbin4096_g128|fluxbin4096_s16] [--M m]
 
 Workload decoder7b is the 32-layer Llama-7B-shaped decoder weight stream (per layer
 q, k, v, o 4096x4096, gate and up 4096->11008, down 11008->4096; 2 bases and a
 rank-256 binary correction each): one step replays a graph of all 224 GEMVs, in
-layer order, over 1.71 GB of distinct weights.
+layer order, over 1.71 GB of distinct weights. Workloads fluxbin4096_* are the same
+4096x4096 projection in FluxBin's own configurations (2b-g128: grouped row scales; 2b-s16-g128:
+plus two binary refinement bases over 16 salient columns of every group).
 
 Metric: effective HBM GB/s of the M=1 binary GEMV (algorithmic bytes: packed
 sign bits, scales, correction signs and coefficients, salient payload, X read
@@ -36,7 +39,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth.configs import build  # noqa: E402
+from synth import make_activations, make_layer  # noqa: E402
+from synth.configs import SEED, build  # noqa: E402
 
 WORKLOADS = {
     # name: (config, spec index, default M, description)
@@ -47,7 +51,12 @@ WORKLOADS = {
     "cfg1": (1, 0, 1, "256x512, 1 base, fp32 scales, rank-8 correction"),
     "decoder7b": (5, None, 1, "32-layer Llama-7B decoder weight stream: q/k/v/o 4096^2, gate/up 4096->11008, "
                               "down 11008->4096, 2 bases + rank-256 binary correction each (224 GEMVs)"),
+    "fluxbin4096_g128": (2, 0, 1, "4096x4096 FluxBin 2b-g128: 2 bases, bf16 row scales per 128-column group"),
+    "fluxbin4096_s16": (2, 0, 1, "4096x4096 FluxBin 2b-s16-g128: 2 bases, bf16 row scales per 128-column group, "
+                                 "2 binary refinement bases over 16 salient columns per group"),
 }
+# FluxBin layers ("FluxBin", Sec. 4, Kb-sS-gG): workload -> (group size, (Ks, s) or None)
+FLUXBIN = {"fluxbin4096_g128": (128, None), "fluxbin4096_s16": (128, (2, 16))}
 DECODER_LAYERS = 32
 DECODER_MATRICES = 7  # q, k, v, o, gate, up, down
 
@@ -59,6 +68,10 @@ def base_matrices(workload, M):
     cfg, spec, _, _ = WORKLOADS[workload]
     if spec is None:
         return [build(cfg, i, M) for i in range(DECODER_MATRICES)]
+    if workload in FLUXBIN:
+        g, ref = FLUXBIN[workload]
+        L = make_layer(SEED, (870, 4096, 4096), 4096, 4096, 2, "bf16", group=g, refine=ref, name=workload)
+        return [(L, make_activations(SEED, (870, 4096, 1000 + M), M, 4096, "bf16"))]
     return [build(cfg, spec, M)]
 
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -183,7 +196,7 @@ def cpu_baseline(workload, M, budget_s=12.0):
     import oracle
     from threadpoolctl import threadpool_info
     cfg, spec, _, _ = WORKLOADS[workload]
-    L, X = build(cfg, spec if spec is not None else 0, M)  # decoder7b: its q projection
+    L, X = base_matrices(workload, M)[0] if spec is not None else build(cfg, 0, M)  # decoder7b: its q projection
     xdt = "f32" if cfg == 1 else "bf16"
     nbytes = oracle.algorithmic_bytes(L, M, xdt, "bf16")
     n, t0 = 0, time.perf_counter()
@@ -231,11 +244,17 @@ def algorithmic_bytes(L, M, x_bytes, y_bytes):
     """Bytes one GEMV must move (same accounting as the oracle's, restated for the
     product path so that the bench does not depend on the oracle)."""
     sb = 2 if L.scale_dtype == "bf16" else 4
-    n = L.K * L.out * L.in_ / 8.0 + L.K * (L.out + L.in_) * sb
+    g = getattr(L, "group", 0) or 0
+    ng = -(-L.in_ // g) if g else 1  # row scales per row
+    n = L.K * L.out * L.in_ / 8.0 + L.K * (L.out * ng + L.in_) * sb
     if L.rank:
         n += L.rank * (L.out + L.in_) / 8.0 + 4 * L.rank
     if L.n_sal:
         n += L.out * L.n_sal + 8 * L.n_sal
+    ks = getattr(L, "ref_K", 0) or 0
+    if ks:  # refinement signs, row scales per group, column scales, int32 indices
+        nr = len(L.ref_idx)
+        n += ks * L.out * nr / 8.0 + ks * (L.out * ng + nr) * sb + 4 * nr
     n += M * L.in_ * x_bytes + M * L.out * y_bytes
     return int(round(n))
 

@@ -26,7 +26,7 @@ BISCO_F32, BISCO_BF16 = 0, 1
 
 BISCO_PATH_AUTO, BISCO_PATH_LOOKUP_TABLE, BISCO_PATH_SMALL_BATCH_ONLY, BISCO_PATH_INTEGER_MMA = 0, 1, 2, 3
 (BISCO_KERNEL_LUT_WARP, BISCO_KERNEL_LUT_STREAM, BISCO_KERNEL_LUT_ROWS, BISCO_KERNEL_INTEGER_MMA,
- BISCO_KERNEL_TENSOR_CORE) = 1, 2, 3, 4, 5
+ BISCO_KERNEL_TENSOR_CORE, BISCO_KERNEL_REFINE) = 1, 2, 3, 4, 5, 6
 
 EXPORTED = [
     "bisco_packed_words", "bisco_pack", "bisco_unpack", "bisco_workspace_size", "bisco_workspace_init",
@@ -46,6 +46,8 @@ class bisco_layer(ctypes.Structure):
         ("n_sal", ctypes.c_int32), ("sal_stride", ctypes.c_int32),
         ("sal_idx", ctypes.c_void_p), ("sal_q", ctypes.c_void_p), ("sal_scale", ctypes.c_void_p),
         ("row_group", ctypes.c_int32),
+        ("ref_bases", ctypes.c_int32), ("n_ref", ctypes.c_int32), ("ref_idx", ctypes.c_void_p),
+        ("ref_bits", ctypes.c_void_p), ("ref_row_scale", ctypes.c_void_p), ("ref_col_scale", ctypes.c_void_p),
     ]
 
 
@@ -194,10 +196,6 @@ class DeviceLayer:
             return torch.from_numpy(a).to(device)
 
         self.host = host
-        if getattr(host, "ref_K", 0):
-            # FluxBin's binary salient refinement bases have no kernel (row-scale groups of s
-            # gathered columns); refuse rather than drop them
-            raise NotImplementedError("the binary salient refinement is not supported by libbisco")
         self.row_group = int(getattr(host, "group", 0) or 0)
         self.out, self.in_, self.K = host.out, host.in_, host.K
         self.rank, self.n_sal = host.rank, host.n_sal
@@ -213,6 +211,16 @@ class DeviceLayer:
         self.sal_idx = up(host.sal_idx)
         self.sal_q = up(host.sal_q)
         self.sal_scale = up(host.sal_scale)
+        self.ref_K = int(getattr(host, "ref_K", 0) or 0)
+        self.n_ref = len(host.ref_idx) if self.ref_K else 0
+        self.ref_idx = self.ref_bits = self.ref_row_scale = self.ref_col_scale = None
+        if self.ref_K:
+            self.ref_idx = up(np.asarray(host.ref_idx, dtype=np.int32))
+            self.ref_bits = up(host.ref_bits)
+            # host [Ks][out][groups] -> device [Ks][groups][out], like the global row scales
+            self.ref_row_scale = up(np.ascontiguousarray(
+                np.asarray(host.ref_row_scale).reshape(self.ref_K, host.out, -1).transpose(0, 2, 1)))
+            self.ref_col_scale = up(host.ref_col_scale)
         ptr = lambda t: (t.data_ptr() if t is not None else None)  # noqa: E731
         self.desc = bisco_layer(
             out=host.out, in_=host.in_, num_bases=host.K,
@@ -221,15 +229,18 @@ class DeviceLayer:
             rank=host.rank, v_bits=ptr(self.v_bits), ut_bits=ptr(self.ut_bits), alpha=ptr(self.alpha),
             n_sal=host.n_sal, sal_stride=host.sal_stride if host.n_sal else 0,
             sal_idx=ptr(self.sal_idx), sal_q=ptr(self.sal_q), sal_scale=ptr(self.sal_scale),
-            row_group=self.row_group)
+            row_group=self.row_group, ref_bases=self.ref_K, n_ref=self.n_ref, ref_idx=ptr(self.ref_idx),
+            ref_bits=ptr(self.ref_bits), ref_row_scale=ptr(self.ref_row_scale),
+            ref_col_scale=ptr(self.ref_col_scale))
 
     def clone(self):
         """Another device copy of the same layer (same values, separate device buffers)."""
         c = DeviceLayer.__new__(DeviceLayer)
         c.host = self.host
         c.out, c.in_, c.K, c.rank, c.n_sal = self.out, self.in_, self.K, self.rank, self.n_sal
-        c.row_group = self.row_group
-        for n in ("bits", "row_scale", "col_scale", "v_bits", "ut_bits", "alpha", "sal_idx", "sal_q", "sal_scale"):
+        c.row_group, c.ref_K, c.n_ref = self.row_group, self.ref_K, self.n_ref
+        for n in ("bits", "row_scale", "col_scale", "v_bits", "ut_bits", "alpha", "sal_idx", "sal_q", "sal_scale",
+                  "ref_idx", "ref_bits", "ref_row_scale", "ref_col_scale"):
             t = getattr(self, n)
             setattr(c, n, t.clone() if t is not None else None)
         ptr = lambda t: (t.data_ptr() if t is not None else None)  # noqa: E731
@@ -238,13 +249,16 @@ class DeviceLayer:
             out=d.out, in_=d.in_, num_bases=d.num_bases, bits=ptr(c.bits), row_scale=ptr(c.row_scale),
             col_scale=ptr(c.col_scale), scale_dtype=d.scale_dtype, rank=d.rank, v_bits=ptr(c.v_bits),
             ut_bits=ptr(c.ut_bits), alpha=ptr(c.alpha), n_sal=d.n_sal, sal_stride=d.sal_stride,
-            sal_idx=ptr(c.sal_idx), sal_q=ptr(c.sal_q), sal_scale=ptr(c.sal_scale), row_group=d.row_group)
+            sal_idx=ptr(c.sal_idx), sal_q=ptr(c.sal_q), sal_scale=ptr(c.sal_scale), row_group=d.row_group,
+            ref_bases=d.ref_bases, n_ref=d.n_ref, ref_idx=ptr(c.ref_idx), ref_bits=ptr(c.ref_bits),
+            ref_row_scale=ptr(c.ref_row_scale), ref_col_scale=ptr(c.ref_col_scale))
         return c
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
                    [self.bits, self.row_scale, self.col_scale, self.v_bits, self.ut_bits, self.alpha,
-                    self.sal_idx, self.sal_q, self.sal_scale] if t is not None)
+                    self.sal_idx, self.sal_q, self.sal_scale, self.ref_idx, self.ref_bits, self.ref_row_scale,
+                    self.ref_col_scale] if t is not None)
 
 
 def _desc(layer):

@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbisco.so")
-SOURCES = ["bisco_gemv.cu", "bisco_imma.cu", "bisco_tc.cu", "bisco_api.cpp", "bisco_noalloc.cu", "bisco_quant.cu"]
+SOURCES = ["bisco_gemv.cu", "bisco_imma.cu", "bisco_tc.cu", "bisco_api.cpp", "bisco_noalloc.cu", "bisco_quant.cu", "bisco_refine.cu"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

@@ -74,6 +74,12 @@ bisco_status validate_layer(const bisco_layer* L) {
     if (!L->sal_idx || !L->sal_q || !L->sal_scale || !aligned16(L->sal_q)) return BISCO_ERR_INVALID_ARG;
     if (L->sal_stride < L->n_sal || (L->sal_stride % 16) != 0) return BISCO_ERR_INVALID_ARG;
   }
+  if (L->ref_bases < 0 || L->ref_bases > kMaxBases) return BISCO_ERR_INVALID_ARG;
+  if (L->ref_bases > 0) {
+    if (L->row_group < 1 || L->n_ref < 1 || L->n_ref > L->in || !dtype_ok(L->scale_dtype)) return BISCO_ERR_INVALID_ARG;
+    if (!L->ref_idx || !L->ref_bits || !L->ref_row_scale || !L->ref_col_scale || !aligned16(L->ref_bits))
+      return BISCO_ERR_INVALID_ARG;
+  }
   return BISCO_OK;
 }
 
@@ -156,13 +162,18 @@ Layout cached_layout(const bisco_layer* L, int MB, int dev) {
   return cache->back().lo;
 }
 
-// Workspace bytes: the status word and, with a correction, z for one batch chunk.
+// Workspace bytes: the status word, with a correction z for one batch chunk, and with a
+// salient refinement that term for one 8-row chunk (after z of 8 rows).
 // ws_need is the minimum bisco_gemv accepts (chunks of 8 rows); ws_pref also lets the
 // tensor-core path take chunks of up to 128 rows for this batch size.
-size_t ws_need(const bisco_layer* L, int32_t) {
+size_t ref_offset(const bisco_layer* L) {
   return kStatusBytes + align256(L->rank > 0 ? static_cast<size_t>(kMaxBatchChunk) * L->rank * 4 : 0);
 }
+size_t ws_need(const bisco_layer* L, int32_t) {
+  return ref_offset(L) + align256(L->ref_bases > 0 ? static_cast<size_t>(kMaxBatchChunk) * L->out * 4 : 0);
+}
 size_t ws_pref(const bisco_layer* L, int32_t M) {
+  if (L->ref_bases > 0) return ws_need(L, M);  // refined layers run in 8-row integer chunks only
   // z rows of a tensor-core chunk (padded to 16; from 8 batch rows up a chunk may go to
   // the tensor cores when the integer plan does not fit)
   const int rows = M < kMaxBatchChunk ? kMaxBatchChunk : std::min<int>((M + 15) / 16 * 16, kTcMaxBatch);
@@ -369,11 +380,14 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
     tc_rows = static_cast<int>(std::min<size_t>(kTcMaxBatch, fit / 16 * 16));
   }
   const int policy = g_policy.load();
-  // grouped row scales: only the integer tensor-core kernel applies them, per 128-column unit
+  // grouped row scales: only the integer tensor-core kernel applies them, per 128-column
+  // unit; a salient refinement is added by the integer kernel only
   const bool grouped = L->num_bases > 0 && L->row_group > 0;
   if (grouped && L->row_group % 128 != 0) return BISCO_ERR_UNSUPPORTED;
+  const bool int_only = grouped || L->ref_bases > 0;
+  if (L->ref_bases > 0 && refine_smem_bytes(L, kMaxBatchChunk) > lim) return BISCO_ERR_UNSUPPORTED;
   const bool tc_ok = (L->num_bases == 0 || L->scale_dtype == BISCO_BF16) && tc_rows >= kTcMinBatch &&
-                     policy != BISCO_PATH_SMALL_BATCH_ONLY && !grouped;
+                     policy != BISCO_PATH_SMALL_BATCH_ONLY && !int_only;
   for (int m0 = 0; m0 < M;) {
     Chunk ch{};
     ch.m0 = m0;
@@ -389,10 +403,10 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
       // which are faster there; with a correction the one-launch integer kernel wins
       // (5120 x 5120, rank 512: 13.5 us against 16.4 us for the two lookup-table launches)
       const bool fusable = ch.lo.has_z && ch.lo.ifz.C > 0;
-      ch.imma = imma_fits(ch.lo) && (grouped || (policy != BISCO_PATH_LOOKUP_TABLE &&
+      ch.imma = imma_fits(ch.lo) && (int_only || (policy != BISCO_PATH_LOOKUP_TABLE &&
                 (batch_block(ch.Mc) >= 2 || policy == BISCO_PATH_INTEGER_MMA || fusable)));
       ch.fused = ch.imma && fusable;
-      if (grouped && !ch.imma) return BISCO_ERR_UNSUPPORTED;
+      if (int_only && !ch.imma) return BISCO_ERR_UNSUPPORTED;
       // a chunk of 8 rows whose integer plan does not fit (large K at 8 batch rows, e.g.
       // 4096 x 11008 with a rank-256 correction) is faster on the tensor cores, padded to
       // 16 columns, than on the lookup-table kernels (that layer: 97 us for a 16-row
@@ -498,14 +512,18 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
 
   int* status = reinterpret_cast<int*>(wsb);
   float* zbuf = reinterpret_cast<float*>(wsb + kStatusBytes);
+  float* rbuf = L->ref_bases > 0 ? reinterpret_cast<float*>(wsb + ref_offset(L)) : nullptr;
   const ImmaDebug dbg{g_dbg_skip_tile.load(), g_dbg_wait_ns.load()};
   for (const Chunk& ch : chunks) {
     const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(ch.m0) * L->in * xb;
     void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(ch.m0) * L->out * yb;
+    // the refinement term first; the integer launch that writes this chunk's Y adds it
+    if (rbuf && launch_refine(L, Xc, x_dtype, ch.Mc, rbuf, status, s) != cudaSuccess) return BISCO_ERR_CUDA;
     if (ch.fused) {
       PassParam pz{}, py{};
       pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);
       pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
+      py.rref = rbuf;
       PassParam both[2] = {pz, py};
       const int zsrc[2] = {-1, 0}, is_z[2] = {1, 0};
       if (run_imma(both, zsrc, is_z, 2, ch.lo.ifz, s, &dbg) != cudaSuccess) return BISCO_ERR_CUDA;
@@ -527,6 +545,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
     }
     PassParam py{};
     pass_y(L, py, Xc, x_dtype, ch.Mc, Yc, y_dtype, zbuf, status);
+    py.rref = rbuf;  // refined layers run on the integer kernel only
     cudaError_t e;
     if (ch.tc) {
       e = launch_tc(py, ch.ty, s, &dbg);
@@ -639,6 +658,8 @@ GroupPlan group_plan(const bisco_layer* Ls, int n, int MB, int dev) {
 // policy that allows the integer kernel.
 bool group_launch_ok(const bisco_layer* Ls, int n, int M, int dev) {
   if (n < 2 || M >= kTcMinBatch || g_policy.load() == BISCO_PATH_LOOKUP_TABLE) return false;
+  for (int j = 0; j < n; ++j)
+    if (Ls[j].ref_bases > 0) return false;  // a refined layer runs its own two launches
   for (int m0 = 0; m0 < M; m0 += kMaxBatchChunk) {
     const int Mc = std::min(kMaxBatchChunk, M - m0);
     if (group_plan(Ls, n, batch_block(Mc), dev).plan.C == 0) return false;
@@ -760,6 +781,7 @@ int32_t bisco_plan_kernels(const bisco_layer* L, int32_t M, int32_t x_dtype, siz
     ++n;
   };
   for (const Chunk& ch : chunks) {
+    if (L->ref_bases > 0) put(BISCO_KERNEL_REFINE);
     const int passes = L->rank > 0 && !ch.fused ? 2 : 1;
     for (int ps = 0; ps < passes; ++ps) {
       const bool is_z = L->rank > 0 && ps == 0;

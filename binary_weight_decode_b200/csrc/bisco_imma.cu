@@ -7,7 +7,9 @@
 // rs = r_k ("FluxBin", Sec. 3.1, decoupled row-column binary bases; the column scale is
 // folded into the activation as in Sec. 3.2, Stage 1), the correction's V with v = x and
 // rs = alpha, or its U^T with v = z ("BiLoCo", "The core idea": alpha * u * (v . x)).
-// A stored bit b means the sign (2b - 1) (FluxBin Sec. 3.2).
+// A stored bit b means the sign (2b - 1) (FluxBin Sec. 3.2). A layer with FluxBin's
+// binary salient refinement (Sec. 4) has that term computed by a small launch just
+// before this one into an fp32 buffer, which the owner of each output row adds last.
 //
 // Formulation. With bits b_i in {0, 1},
 //   sum_i (2 b_i - 1) v_i = 2 * sum_i b_i v_i - sum_i v_i,
@@ -750,6 +752,11 @@ __global__ void __launch_bounds__(kIT, 2)
           }
         }
       }
+    }
+    if (p.rref) {  // salient refinement term, written by the launch before this one
+#pragma unroll
+      for (int m = 0; m < MB; ++m)
+        if (m < p.Mc) sum[m] += __ldcg(p.rref + static_cast<long long>(m) * p.rows + o);
     }
 #pragma unroll
     for (int m = 0; m < MB; ++m) {

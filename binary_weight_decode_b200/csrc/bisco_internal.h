@@ -66,6 +66,7 @@ struct PassParam {
   // salient columns (added once per output row)
   int n_sal, sal_stride;
   const int* sal_idx; const int8_t* sal_q; const float* sal_scale;
+  const float* rref;     // [Mc][rows] salient refinement term to add (integer kernel), or nullptr
   int* status;           // device status word (workspace)
 };
 
@@ -143,6 +144,25 @@ struct ImmaRole {
 ImmaPlan make_imma_plan(const ImmaRole* roles, int nroles, int MB, size_t smem_limit);
 // L.pass[r] holds role r's pass with the plan's maxima filled in; L.rt its role table.
 cudaError_t launch_imma(const ImmaLaunch& L, const ImmaPlan& plan, cudaStream_t stream, bool pdl, const ImmaDebug* dbg);
+// One launch of the salient refinement kernel: rref[m][o] for the Mc batch rows of X
+// (grid: one CTA per 32-row tile of the output).
+struct RefineParam {
+  const uint32_t* bits;   // [Ks][packed words of out x n_ref]
+  const void* rrs;        // row scales [Ks][ngroups][out]
+  const void* rcs;        // column scales [Ks][n_ref]
+  int sdt;                // dtype of both scales
+  const int* idx;         // [n_ref] ascending input columns
+  int Ks, n_ref, in, out, g, ngroups, tiles;
+  const void* X; int xdt; int ldx;
+  int Mc;
+  float* rref;            // [Mc][out]
+  int* status;
+};
+// Shared memory of one refinement launch at batch block MB (0 for a layer without one).
+size_t refine_smem_bytes(const bisco_layer* L, int MB);
+// The salient refinement term of a layer for Mc batch rows of X into rref [Mc][out] (fp32).
+cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, int Mc, float* rref, int* status,
+                          cudaStream_t stream);
 cudaError_t imma_ensure_attrs();
 
 // Tensor-core path (16..128 batch rows per launch): one launch per pass.

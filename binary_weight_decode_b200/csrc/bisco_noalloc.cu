@@ -52,7 +52,7 @@ void* scratch_address(int dev, cudaError_t* err) {
 extern "C" bisco_status bisco_gemv_noalloc(const bisco_layer* layer, const void* X, int32_t x_dtype, int32_t M,
                                            void* Y, int32_t y_dtype, void* stream) {
   if (!layer) return BISCO_ERR_INVALID_ARG;
-  if (layer->rank > BISCO_NOALLOC_MAX_RANK) return BISCO_ERR_UNSUPPORTED;
+  if (layer->rank > BISCO_NOALLOC_MAX_RANK || layer->ref_bases > 0) return BISCO_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BISCO_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return BISCO_ERR_UNSUPPORTED;

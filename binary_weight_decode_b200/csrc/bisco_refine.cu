@@ -1,0 +1,227 @@
+// Binary salient refinement ("FluxBin: ...", Sec. 4 with the Kb-sS-gG configurations,
+// and Sec. 3.2 "Virtual Columnar Mapping (VCM) for Salient Phase"): Ks extra sign bases
+// over the s salient columns of every column group, stored as one dense packed sign matrix
+// over the gathered columns idx[0..n_ref). Row o of the term, for batch row m, is
+//
+//   rref[m][o] = sum_k sum_j rs_k[j][o] * sum_{t in group j} c_k[t] * (2 b_k(o, t) - 1) * x[m][idx[t]]
+//
+// where group j holds the gathered columns whose input column lies in [j*g, (j+1)*g)
+// (idx is ascending, so these are one contiguous run of t) and rs_k[j][o] is the
+// refinement's row scale of that group. The activations are gathered through idx once
+// per CTA (the translation layer of the mapping), the packed signs of the CTA's 32-row
+// tile and the column scales are staged in shared memory, and each warp takes every 8th
+// group of the tile's rows with one lane per row.
+//
+// The result goes to an fp32 workspace buffer; the integer GEMV launch that follows on the
+// stream adds it to the rest of the row before the output is rounded. Weight-side data
+// (signs, column scales, the first row scales, the group boundaries) is read before
+// griddepcontrol.wait, the activations only after it.
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+
+#include "bisco_internal.h"
+
+namespace bisco {
+namespace {
+
+constexpr int kRefWarps = 8;
+constexpr int kRefThreads = kRefWarps * 32;
+
+__device__ __forceinline__ float load_scale(const void* a, long long i, int dt) {
+  if (dt == BISCO_BF16)
+    return __uint_as_float(static_cast<unsigned>(__ldg(reinterpret_cast<const unsigned short*>(a) + i)) << 16);
+  return __ldg(reinterpret_cast<const float*>(a) + i);
+}
+
+__device__ __forceinline__ float load_act(const void* a, long long i, int dt) {
+  if (dt == BISCO_BF16)
+    return __uint_as_float(static_cast<unsigned>(reinterpret_cast<const unsigned short*>(a)[i]) << 16);
+  return reinterpret_cast<const float*>(a)[i];
+}
+
+// Shared memory of one CTA, in this order (4-byte words; sbits first, so that its 16-byte
+// stores are aligned whatever the other sizes):
+//   sbits [Ks][Qr][32][4]   the tile's packed refinement signs
+//   cs    [Ks][n_ref]       column scales c_k[t]
+//   xg    [MB][n_ref]       gathered activations x[m][idx[t]]
+//   sidx  [n_ref]           the gathered column indices
+//   gs    [ngroups + 1]     first gathered column of each group
+//   red   [kRefWarps][32][MB] per-warp partial sums of the tile's rows
+__host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, int MB) {
+  const size_t qr = (static_cast<size_t>(n_ref) + 127) / 128;
+  return 4 * (static_cast<size_t>(Ks) * n_ref + static_cast<size_t>(MB) * n_ref + n_ref + Ks * qr * 128 + ngroups +
+              1 + static_cast<size_t>(kRefWarps) * 32 * MB);
+}
+
+template <int MB>
+__global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_constant__ RefineParam p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int Ks = p.Ks, n = p.n_ref, ng = p.ngroups;
+  const int qr = (n + 127) / 128;
+  uint32_t* sbits = reinterpret_cast<uint32_t*>(smem);
+  float* cs = reinterpret_cast<float*>(sbits + static_cast<size_t>(Ks) * qr * 128);
+  float* xg = cs + static_cast<size_t>(Ks) * n;
+  int* sidx = reinterpret_cast<int*>(xg + static_cast<size_t>(MB) * n);
+  int* gs = sidx + n;
+  float* red = reinterpret_cast<float*>(gs + ng + 1);
+
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int tile = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int o = tile * 32 + lane;
+  const bool row_ok = o < p.out;
+
+  // the first group's row scales of this lane, in flight while the CTA stages its tables
+  float rs_cur[kMaxBases], rs_nxt[kMaxBases];
+#pragma unroll
+  for (int k = 0; k < kMaxBases; ++k) {
+    rs_cur[k] = 0.f;
+    if (k < Ks && warp < ng && row_ok) rs_cur[k] = load_scale(p.rrs, (static_cast<long long>(k) * ng + warp) * p.out + o, p.sdt);
+  }
+  for (int i = tid; i < Ks * n; i += kRefThreads) cs[i] = load_scale(p.rcs, i, p.sdt);
+  // the tile's words of base k are one contiguous run of qr * 128 words
+  const size_t words = static_cast<size_t>(p.tiles) * qr * 128;
+  for (int i = tid; i < Ks * qr * 32; i += kRefThreads) {
+    const int k = i / (qr * 32), w = i - k * qr * 32;
+    reinterpret_cast<uint4*>(sbits)[i] =
+        __ldg(reinterpret_cast<const uint4*>(p.bits + k * words + static_cast<size_t>(tile) * qr * 128) + w);
+  }
+  // group j starts at the first gathered column whose input column is >= j * g: every
+  // column t whose group differs from that of column t-1 starts the groups in between (one
+  // pass over idx instead of a dependent search per group). Entries stay n for groups after
+  // the last column, and every entry is a valid position whatever idx holds.
+  for (int j = tid; j <= ng; j += kRefThreads) gs[j] = n;
+  __syncthreads();
+  for (int t = tid; t < n; t += kRefThreads) {
+    const int c = __ldg(p.idx + t);
+    sidx[t] = c;
+    const int jt = min(max(c, 0) / p.g, ng - 1);
+    const int jp = t == 0 ? -1 : min(max(__ldg(p.idx + t - 1), 0) / p.g, ng - 1);
+    for (int j = jp + 1; j <= jt; ++j) gs[j] = t;
+  }
+
+  __syncthreads();  // sidx complete
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int i = tid; i < MB * n; i += kRefThreads) {
+    const int m = i / n, t = i - m * n;
+    float v = 0.f;
+    if (m < p.Mc) {
+      const int c = sidx[t];
+      if (c < 0 || c >= p.in) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+      else v = load_act(p.X, static_cast<long long>(m) * p.ldx + c, p.xdt);
+    }
+    xg[i] = v;
+  }
+  __syncthreads();
+
+  float acc[MB];
+#pragma unroll
+  for (int m = 0; m < MB; ++m) acc[m] = 0.f;
+  for (int j = warp; j < ng; j += kRefWarps) {
+    const int jn = j + kRefWarps;
+#pragma unroll
+    for (int k = 0; k < kMaxBases; ++k) {
+      rs_nxt[k] = 0.f;
+      if (k < Ks && jn < ng && row_ok) rs_nxt[k] = load_scale(p.rrs, (static_cast<long long>(k) * ng + jn) * p.out + o, p.sdt);
+    }
+    const int t0 = gs[j], t1 = gs[j + 1];  // t0 > t1 only for indices out of order: no columns
+    for (int k = 0; k < Ks; ++k) {
+      float part[MB];
+#pragma unroll
+      for (int m = 0; m < MB; ++m) part[m] = 0.f;
+      const uint32_t* kb = sbits + static_cast<size_t>(k) * qr * 128;
+      uint32_t word = 0;
+      for (int t = t0; t < t1; ++t) {
+        if (t == t0 || (t & 31) == 0) word = kb[((t >> 7) * 32 + lane) * 4 + ((t >> 5) & 3)];
+        const float c = cs[k * n + t];
+        const float sc = ((word >> (t & 31)) & 1u) ? c : -c;
+#pragma unroll
+        for (int m = 0; m < MB; ++m) part[m] = fmaf(sc, xg[m * n + t], part[m]);
+      }
+      float r = 0.f;
+#pragma unroll
+      for (int q = 0; q < kMaxBases; ++q)
+        if (q == k) r = rs_cur[q];
+#pragma unroll
+      for (int m = 0; m < MB; ++m) acc[m] = fmaf(r, part[m], acc[m]);
+    }
+#pragma unroll
+    for (int k = 0; k < kMaxBases; ++k) rs_cur[k] = rs_nxt[k];
+  }
+#pragma unroll
+  for (int m = 0; m < MB; ++m) red[(warp * 32 + lane) * MB + m] = acc[m];
+  __syncthreads();
+  // the 8 warps' partials of a row, summed in warp order
+  for (int i = tid; i < 32 * MB; i += kRefThreads) {
+    const int r = i / MB, m = i - r * MB, oo = tile * 32 + r;
+    if (oo >= p.out || m >= p.Mc) continue;
+    float s = 0.f;
+    for (int w = 0; w < kRefWarps; ++w) s += red[(w * 32 + r) * MB + m];
+    p.rref[static_cast<size_t>(m) * p.out + oo] = s;
+  }
+}
+
+template <int MB>
+cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t stream) {
+  static std::atomic<size_t> allowed{48 * 1024};  // dynamic shared memory this kernel is opted in to
+  if (smem > allowed.load()) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(refine_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    allowed.store(smem);
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.tiles);
+  cfg.blockDim = dim3(kRefThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, refine_kernel<MB>, p);
+}
+
+}  // namespace
+
+size_t refine_smem_bytes(const bisco_layer* L, int MB) {
+  if (L->ref_bases <= 0 || L->row_group <= 0) return 0;
+  const int ng = static_cast<int>((static_cast<long long>(L->in) + L->row_group - 1) / L->row_group);
+  return refine_smem(L->ref_bases, L->n_ref, ng, MB);
+}
+
+cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, int Mc, float* rref, int* status,
+                          cudaStream_t stream) {
+  RefineParam p{};
+  p.bits = L->ref_bits;
+  p.rrs = L->ref_row_scale;
+  p.rcs = L->ref_col_scale;
+  p.sdt = L->scale_dtype;
+  p.idx = L->ref_idx;
+  p.Ks = L->ref_bases;
+  p.n_ref = L->n_ref;
+  p.in = L->in;
+  p.out = L->out;
+  p.g = L->row_group;
+  p.ngroups = static_cast<int>((static_cast<long long>(L->in) + L->row_group - 1) / L->row_group);
+  p.tiles = (L->out + 31) / 32;
+  p.X = X;
+  p.xdt = x_dtype;
+  p.ldx = L->in;
+  p.Mc = Mc;
+  p.rref = rref;
+  p.status = status;
+  const int MB = Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8;
+  const size_t smem = refine_smem(p.Ks, p.n_ref, p.ngroups, MB);
+  switch (MB) {
+    case 1: return launch_refine_mb<1>(p, smem, stream);
+    case 2: return launch_refine_mb<2>(p, smem, stream);
+    case 4: return launch_refine_mb<4>(p, smem, stream);
+    default: return launch_refine_mb<8>(p, smem, stream);
+  }
+}
+
+}  // namespace bisco

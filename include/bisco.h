@@ -110,6 +110,18 @@ typedef struct {
                                The kernels take g a multiple of 128 (else
                                BISCO_ERR_UNSUPPORTED); grouped layers run on the
                                integer tensor-core kernel in chunks of up to 8 rows */
+  /* Binary salient refinement ("FluxBin", Sec. 4, Kb-sS-gG; stored as one dense sign
+     matrix over the gathered salient columns, Sec. 3.2 Virtual Columnar Mapping), added to
+     the rest of W: entry (o, ref_idx[t]) gains
+     sum_k ref_row_scale[k][ref_idx[t] / row_group][o] * ref_col_scale[k][t] * (2b - 1),
+     b = bit (o, t) of refinement base k. Needs row_group > 0 (the refinement's row scales
+     are grouped like the global ones). */
+  int32_t ref_bases;        /* Ks in 0..4; 0 = none                                    */
+  int32_t n_ref;            /* salient columns of the refinement, >= 1 when Ks > 0     */
+  const int32_t* ref_idx;   /* [n_ref] strictly ascending column indices in [0, in)    */
+  const uint32_t* ref_bits; /* [Ks][bisco_packed_words(out, n_ref)] packed signs       */
+  const void* ref_row_scale; /* [Ks][ceil(in/row_group)][out], dtype scale_dtype       */
+  const void* ref_col_scale; /* [Ks][n_ref], dtype scale_dtype                         */
 } bisco_layer;
 
 /*
@@ -121,7 +133,8 @@ bisco_status bisco_workspace_size(const bisco_layer* layer, int32_t M, size_t* b
 /*
  * Prepare a workspace for first use: zero-fills ws_bytes bytes on `stream`.
  * The workspace holds the device status word, counters that a launch computing z and
- * y together uses to hand z over (each such launch returns them to zero), and z.
+ * y together uses to hand z over (each such launch returns them to zero), z, and for a
+ * layer with a salient refinement that term of one 8-row batch chunk (fp32).
  * Every bisco_gemv call leaves the workspace ready for the next call, so this is
  * needed once per buffer (and again after a call reported an error).
  */
@@ -149,8 +162,9 @@ bisco_status bisco_gemv(const bisco_layer* layer, const void* X, int32_t x_dtype
  * below 16 rows each chunk of up to 8 rows runs as ONE integer tensor-core launch whose
  * clusters are split between the layers (and, for a layer with a correction, between its
  * z pass and its output pass, as in bisco_gemv), so the dependent chain of a launch is paid
- * once for the group. Larger batches, or groups whose launch does not fit, run layer by
- * layer exactly as bisco_gemv (same results within the documented tolerance either way).
+ * once for the group. Larger batches, groups whose launch does not fit and groups with a
+ * salient-refined layer run layer by layer exactly as bisco_gemv (same results within the
+ * documented tolerance either way).
  *  layers: host array of n layers.   X: device [M][in].   Y: host array of n device
  *  pointers, Y[j] [M][layers[j].out].   ws: at least bisco_group_workspace_size bytes,
  *  prepared by bisco_workspace_init. Errors as bisco_gemv; BISCO_ERR_INVALID_ARG for n
@@ -183,6 +197,11 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  *    tcgen05 kernel).
  *  BISCO_PATH_INTEGER_MMA: as AUTO, but chunks of up to 8 rows, single rows included,
  *    take the integer tensor-core kernel whenever its plan fits.
+ * Layers with grouped row scales or a salient refinement run every batch chunk (8 rows
+ * at most) on the integer tensor-core kernel under every policy; a refined chunk is
+ * preceded by one refinement launch (BISCO_KERNEL_REFINE). BISCO_ERR_UNSUPPORTED when
+ * the integer plan, or the refinement's shared-memory tables (about
+ * 4 * (Ks + 9) * n_ref + 512 * Ks * ceil(n_ref / 128) bytes), do not fit.
  * Every path computes the same product within the documented tolerance.
  * Returns BISCO_ERR_INVALID_ARG for an unknown policy.
  */
@@ -196,7 +215,9 @@ enum {
   BISCO_KERNEL_LUT_ROWS = 3,      /* lookup tables, warps own row tiles, 4 or 8 rows     */
   BISCO_KERNEL_INTEGER_MMA = 4,   /* int8 tensor cores (mma.sync), <= 8 rows; with a
                                      correction, z and y in one launch                   */
-  BISCO_KERNEL_TENSOR_CORE = 5    /* tcgen05 tensor cores, 16..128 rows                  */
+  BISCO_KERNEL_TENSOR_CORE = 5,   /* tcgen05 tensor cores, 16..128 rows                  */
+  BISCO_KERNEL_REFINE = 6         /* salient refinement term into the workspace (CUDA
+                                     cores), ahead of the integer launch that adds it     */
 };
 
 /*
@@ -238,7 +259,8 @@ bisco_status bisco_debug_set_wait_test(int32_t skip_tile, uint64_t wait_ns);
  * that loads the library keeps it until the process exits. This call allocates nothing.
  *
  * Arguments and results are those of bisco_gemv, minus the workspace. Layers with
- * rank > BISCO_NOALLOC_MAX_RANK are rejected with BISCO_ERR_UNSUPPORTED.
+ * rank > BISCO_NOALLOC_MAX_RANK, and layers with a salient refinement (ref_bases > 0,
+ * whose term needs out * 32 bytes of scratch), are rejected with BISCO_ERR_UNSUPPORTED.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress);
  * make that first call before any stream capture starts. A failed lookup is not cached
  * (the next call retries); a device reset invalidates the cached address.

@@ -346,14 +346,21 @@ def _dtype_bytes(dtype):
 
 
 def algorithmic_bytes(layer, M, x_dtype, y_dtype="f32"):
-    """Bytes one GEMV must move at minimum: unpadded sign bits, scales, correction
-    signs and coefficients, salient payload, X read and Y written."""
+    """Bytes one GEMV must move at minimum: unpadded sign bits, scales (grouped row scales
+    counted per group), correction signs and coefficients, salient payload, refinement
+    signs, scales and indices, X read and Y written."""
     sb = _dtype_bytes(layer.scale_dtype)
+    g = getattr(layer, "group", 0) or 0
+    ng = -(-layer.in_ // g) if g else 1  # row scales per row (FluxBin Sec. 3.1 groups)
     n = layer.K * layer.out * layer.in_ / 8.0
-    n += layer.K * (layer.out + layer.in_) * sb
+    n += layer.K * (layer.out * ng + layer.in_) * sb
     if layer.rank:
         n += layer.rank * (layer.out + layer.in_) / 8.0 + 4 * layer.rank
     if layer.n_sal:
         n += layer.out * layer.n_sal + 4 * layer.n_sal + 4 * layer.n_sal
+    ks = getattr(layer, "ref_K", 0) or 0
+    if ks:  # FluxBin Sec. 4 refinement: signs, per-group row scales, column scales, int32 indices
+        nr = len(layer.ref_idx)
+        n += ks * layer.out * nr / 8.0 + ks * (layer.out * ng + nr) * sb + 4 * nr
     n += M * layer.in_ * _dtype_bytes(x_dtype) + M * layer.out * _dtype_bytes(y_dtype)
     return int(round(n))

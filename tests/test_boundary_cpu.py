@@ -80,26 +80,76 @@ def test_gemv_rejects_bad_arguments_before_touching_the_device():
     assert bw.bisco_status_string(bw.BISCO_ERR_WORKSPACE) == "BISCO_ERR_WORKSPACE"
 
 
-def test_row_group_field_and_negative_group():
-    # bisco_layer ends with row_group (0 = one row scale per row); a negative group is
-    # refused before anything touches the device
+def test_binding_constants_match_the_header():
+    # every enumerator the header declares (status codes, dtypes, policies, kernel kinds)
+    # exists in the binding with the same value
+    hdr = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "bisco.h")).read(), flags=re.S)
+    found = 0
+    for body in re.findall(r"(?:typedef\s+)?enum\s*\w*\s*\{(.*?)\}", hdr, flags=re.S):
+        nxt = 0
+        for item in [i.strip() for i in body.split(",") if i.strip()]:
+            name, _, val = item.partition("=")
+            name = name.strip()
+            nxt = int(val.strip(), 0) if val.strip() else nxt
+            assert getattr(bw, name) == nxt, name
+            found += 1
+            nxt += 1
+    assert found >= 18 and bw.BISCO_KERNEL_REFINE == 6
+
+
+def test_layer_fields_and_negative_group():
+    # the binding's struct mirrors bisco_layer field by field (row_group, then the salient
+    # refinement's six fields last); a negative group is refused before anything touches
+    # the device
     hdr = open(os.path.join(ROOT, "include", "bisco.h")).read()
     body = hdr[hdr.index("typedef struct {", hdr.index("One layer.")):hdr.index("} bisco_layer;")]
     body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)  # drop comments
     declared = re.findall(r"(\w+)\s*;", body)  # field names in declaration order
     assert [n.rstrip("_") for n, _ in bw.bisco_layer._fields_] == declared
-    assert declared[-1] == "row_group"
+    assert declared[-7:] == ["row_group", "ref_bases", "n_ref", "ref_idx", "ref_bits", "ref_row_scale",
+                             "ref_col_scale"]
     L = bw.bisco_layer(out=10, in_=10, num_bases=0, row_group=-1)
     assert bw._lib.bisco_gemv(L, None, 0, 1, None, 0, None, 0, None) == bw.BISCO_ERR_INVALID_ARG
 
 
-def test_salient_refinement_is_refused_by_the_binding():
-    # no kernel runs FluxBin's refinement bases: the binding refuses such a layer instead of
-    # silently dropping a term
-    from synth import make_layer
-    L = make_layer(0, (55,), 64, 256, 2, "bf16", group=128, refine=(2, 8))
-    with pytest.raises(NotImplementedError):
-        bw.DeviceLayer(L)
+def _refined_desc(**kw):
+    # a descriptor with placeholder (never dereferenced) 16-byte aligned addresses: the
+    # calls below only validate and size
+    import ctypes
+    f = dict(out=96, in_=512, num_bases=1, bits=0x1000, row_scale=0x2000, col_scale=0x3000,
+             scale_dtype=bw.BISCO_BF16, row_group=128, ref_bases=2, n_ref=32, ref_idx=0x4000,
+             ref_bits=0x5000, ref_row_scale=0x6000, ref_col_scale=0x7000)
+    f.update(kw)
+    return (bw.bisco_layer * 1)(bw.bisco_layer(**f)), ctypes
+
+
+def test_salient_refinement_fields_are_validated():
+    # FluxBin's refinement (Sec. 4, Kb-sS-gG) needs the group size of its row scales, 1..4
+    # bases, 1..in gathered columns, every array, and 16-byte aligned packed signs
+    ok, ctypes = _refined_desc()
+    n = ctypes.c_size_t(0)
+    assert bw._lib.bisco_group_workspace_size(ok, 1, 1, ctypes.byref(n)) == bw.BISCO_OK
+    # status region, no z, then the refinement term of one 8-row chunk: 8 * 96 fp32
+    assert n.value == 256 + 8 * 96 * 4
+    okz, _ = _refined_desc(rank=64, v_bits=0x8000, ut_bits=0x9000, alpha=0xA000)
+    assert bw._lib.bisco_group_workspace_size(okz, 1, 40, ctypes.byref(n)) == bw.BISCO_OK
+    assert n.value == 256 + 8 * 64 * 4 + 8 * 96 * 4  # refined layers never take 16-row chunks
+    bad = [dict(row_group=0), dict(ref_bases=5), dict(ref_bases=-1), dict(n_ref=0), dict(n_ref=513),
+           dict(ref_idx=None), dict(ref_bits=None), dict(ref_row_scale=None), dict(ref_col_scale=None),
+           dict(ref_bits=0x5004), dict(scale_dtype=7)]
+    for kw in bad:
+        d, _ = _refined_desc(**kw)
+        assert bw._lib.bisco_group_workspace_size(d, 1, 1, ctypes.byref(n)) == bw.BISCO_ERR_INVALID_ARG, kw
+    # without refinement bases the other refinement fields are ignored
+    d, _ = _refined_desc(ref_bases=0, n_ref=0, ref_idx=None, ref_bits=None)
+    assert bw._lib.bisco_group_workspace_size(d, 1, 1, ctypes.byref(n)) == bw.BISCO_OK
+    assert n.value == 256
+
+
+def test_no_alloc_entry_refuses_a_refined_layer():
+    # the fixed scratch array has no room for the refinement term
+    ok, _ = _refined_desc()
+    assert bw._lib.bisco_gemv_noalloc(ok, None, 0, 1, None, 0, None) == bw.BISCO_ERR_UNSUPPORTED
 
 
 def test_group_call_validates_before_touching_the_device():

@@ -465,6 +465,23 @@ def test_algorithmic_bytes_salient_term():
     assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 11_818_360 + 4096 + 8
 
 
+def test_algorithmic_bytes_grouped_and_refined():
+    # FluxBin 2b-g128 and 2b-s16-g128 on 4096 x 4096 (Sec. 4 configurations), batch 1, bf16
+    # x and y, counted by hand: signs 2*4096*4096/8 = 4,194,304; grouped row scales
+    # 2*4096*32*2 = 524,288; column scales 2*4096*2 = 16,384; x 8,192; y 8,192 -> 4,751,360
+    from synth import make_layer
+    L = make_layer(0, (56,), 4096, 4096, 2, "bf16", group=128)
+    assert oracle.algorithmic_bytes(L, 1, "bf16", "bf16") == 4_751_360
+    # refinement over 16 salient columns of each of the 32 groups (n_ref = 512): signs
+    # 2*4096*512/8 = 524,288; row scales 2*4096*32*2 = 524,288; column scales 2*512*2 = 2,048;
+    # int32 indices 512*4 = 2,048 -> 1,052,672 more
+    L = make_layer(0, (56,), 4096, 4096, 2, "bf16", group=128, refine=(2, 16))
+    n = oracle.algorithmic_bytes(L, 1, "bf16", "bf16")
+    assert n == 4_751_360 + 1_052_672
+    # the weight bytes are the Sec. C.2 storage, but for int32 instead of 16-bit indices
+    assert n - 8_192 - 8_192 - 2 * 512 == oracle.fluxbin_storage_bits(L) // 8
+
+
 @pytest.mark.parametrize("rows,cols", [(70, 300), (33, 129), (1, 5)])
 def test_row_decoder_matches_independent_packer(rows, cols):
     S = np.random.default_rng(7 * rows + cols).choice(np.array([-1, 1], np.int8), size=(rows, cols))
