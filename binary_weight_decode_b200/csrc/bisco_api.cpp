@@ -399,6 +399,12 @@ bisco_status plan_chunks(const bisco_layer* L, int M, int32_t x_dtype, size_t ws
     if (!ch.tc) {
       ch.Mc = std::min(kMaxBatchChunk, rem);
       ch.lo = cached_layout(L, batch_block(ch.Mc), dev);
+      // grouped or refined layers have no other kernel: where the integer plan of 8 rows
+      // does not fit (e.g. 11008 input columns), the chunk takes 4, 2 or 1 rows instead
+      while (int_only && !imma_fits(ch.lo) && ch.Mc > 1) {
+        ch.Mc = batch_block(ch.Mc) / 2;
+        ch.lo = cached_layout(L, batch_block(ch.Mc), dev);
+      }
       // single rows of a layer without a correction stay on the lookup-table kernels,
       // which are faster there; with a correction the one-launch integer kernel wins
       // (5120 x 5120, rank 512: 13.5 us against 16.4 us for the two lookup-table launches)

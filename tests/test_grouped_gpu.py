@@ -55,6 +55,18 @@ def test_grouped_layer_llama_shape_sampled():
     check(Y[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
 
 
+def test_grouped_down_projection_at_eight_rows():
+    # 4096 x 11008 (the down projection), g = 128, 8 batch rows: the integer plan of 8 rows
+    # does not fit shared memory, so the chunk runs as smaller integer launches
+    X = make_activations(0, (834,), 8, 11008, "bf16")
+    L = make_layer(0, (834,), 4096, 11008, 2, "bf16", group=128)
+    ks = kinds(L, 8)
+    assert set(ks) == {bw.BISCO_KERNEL_INTEGER_MMA} and len(ks) >= 1
+    Y = run(L, X, "bf16", "f32")
+    rows = sample_rows(L.out, 128, 10)
+    check(Y[:, rows], oracle.gemv_rows(L, X, "bf16", rows), X, "bf16", "f32")
+
+
 def test_grouped_layers_take_the_integer_kernel_under_every_policy():
     L = make_layer(0, (832,), 256, 512, 2, "bf16", group=128)
     try:
