@@ -9,13 +9,14 @@
 // (idx is ascending, so these are one contiguous run of t) and rs_k[j][o] is the
 // refinement's row scale of that group. The activations are gathered through idx once
 // per CTA (the translation layer of the mapping), the packed signs of the CTA's 32-row
-// tile and the column scales are staged in shared memory, and each warp takes every 8th
-// group of the tile's rows with one lane per row.
+// tile, their row scales and the column scales are staged in shared memory, and each warp
+// takes every 8th group of the tile's rows with one lane per row.
 //
 // The result goes to an fp32 workspace buffer; the integer GEMV launch that follows on the
 // stream adds it to the rest of the row before the output is rounded. Weight-side data
-// (signs, column scales, the first row scales, the group boundaries) is read before
-// griddepcontrol.wait, the activations only after it.
+// (signs, row and column scales, the group boundaries) is read before griddepcontrol.wait,
+// the activations only after it; each staging round issues all of its loads before it
+// stores any, so the kernel pays a handful of memory latencies, not one per element.
 
 #include <cuda_runtime.h>
 
@@ -45,6 +46,7 @@ __device__ __forceinline__ float load_act(const void* a, long long i, int dt) {
 // Shared memory of one CTA, in this order (4-byte words; sbits first, so that its 16-byte
 // stores are aligned whatever the other sizes):
 //   sbits [Ks][Qr][32][4]   the tile's packed refinement signs
+//   srs   [Ks][ngroups][32] the tile's refinement row scales
 //   cs    [Ks][n_ref]       column scales c_k[t]
 //   xg    [MB][n_ref]       gathered activations x[m][idx[t]]
 //   sidx  [n_ref]           the gathered column indices
@@ -52,9 +54,14 @@ __device__ __forceinline__ float load_act(const void* a, long long i, int dt) {
 //   red   [kRefWarps][32][MB] per-warp partial sums of the tile's rows
 __host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, int MB) {
   const size_t qr = (static_cast<size_t>(n_ref) + 127) / 128;
-  return 4 * (static_cast<size_t>(Ks) * n_ref + static_cast<size_t>(MB) * n_ref + n_ref + Ks * qr * 128 + ngroups +
-              1 + static_cast<size_t>(kRefWarps) * 32 * MB);
+  return 4 * (static_cast<size_t>(Ks) * qr * 128 + static_cast<size_t>(Ks) * ngroups * 32 +
+              static_cast<size_t>(Ks) * n_ref + static_cast<size_t>(MB) * n_ref + n_ref + ngroups + 1 +
+              static_cast<size_t>(kRefWarps) * 32 * MB);
 }
+
+// Loads in flight per thread in one staging round: every load of a round is issued before
+// the first of its values is stored, so a round costs one memory latency.
+constexpr int kBatch = 4;
 
 template <int MB>
 __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_constant__ RefineParam p) {
@@ -62,7 +69,8 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
   const int Ks = p.Ks, n = p.n_ref, ng = p.ngroups;
   const int qr = (n + 127) / 128;
   uint32_t* sbits = reinterpret_cast<uint32_t*>(smem);
-  float* cs = reinterpret_cast<float*>(sbits + static_cast<size_t>(Ks) * qr * 128);
+  float* srs = reinterpret_cast<float*>(sbits + static_cast<size_t>(Ks) * qr * 128);
+  float* cs = srs + static_cast<size_t>(Ks) * ng * 32;
   float* xg = cs + static_cast<size_t>(Ks) * n;
   int* sidx = reinterpret_cast<int*>(xg + static_cast<size_t>(MB) * n);
   int* gs = sidx + n;
@@ -70,49 +78,80 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
 
   asm volatile("griddepcontrol.launch_dependents;");
   const int tile = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int o = tile * 32 + lane;
-  const bool row_ok = o < p.out;
 
-  // the first group's row scales of this lane, in flight while the CTA stages its tables
-  float rs_cur[kMaxBases], rs_nxt[kMaxBases];
-#pragma unroll
-  for (int k = 0; k < kMaxBases; ++k) {
-    rs_cur[k] = 0.f;
-    if (k < Ks && warp < ng && row_ok) rs_cur[k] = load_scale(p.rrs, (static_cast<long long>(k) * ng + warp) * p.out + o, p.sdt);
-  }
-  for (int i = tid; i < Ks * n; i += kRefThreads) cs[i] = load_scale(p.rcs, i, p.sdt);
-  // the tile's words of base k are one contiguous run of qr * 128 words
-  const size_t words = static_cast<size_t>(p.tiles) * qr * 128;
-  for (int i = tid; i < Ks * qr * 32; i += kRefThreads) {
-    const int k = i / (qr * 32), w = i - k * qr * 32;
-    reinterpret_cast<uint4*>(sbits)[i] =
-        __ldg(reinterpret_cast<const uint4*>(p.bits + k * words + static_cast<size_t>(tile) * qr * 128) + w);
-  }
   // group j starts at the first gathered column whose input column is >= j * g: every
   // column t whose group differs from that of column t-1 starts the groups in between (one
   // pass over idx instead of a dependent search per group). Entries stay n for groups after
   // the last column, and every entry is a valid position whatever idx holds.
   for (int j = tid; j <= ng; j += kRefThreads) gs[j] = n;
   __syncthreads();
-  for (int t = tid; t < n; t += kRefThreads) {
-    const int c = __ldg(p.idx + t);
-    sidx[t] = c;
-    const int jt = min(max(c, 0) / p.g, ng - 1);
-    const int jp = t == 0 ? -1 : min(max(__ldg(p.idx + t - 1), 0) / p.g, ng - 1);
-    for (int j = jp + 1; j <= jt; ++j) gs[j] = t;
-  }
 
-  __syncthreads();  // sidx complete
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  for (int i = tid; i < MB * n; i += kRefThreads) {
-    const int m = i / n, t = i - m * n;
-    float v = 0.f;
-    if (m < p.Mc) {
-      const int c = sidx[t];
-      if (c < 0 || c >= p.in) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
-      else v = load_act(p.X, static_cast<long long>(m) * p.ldx + c, p.xdt);
+  // Weight-side staging, all before the dependency wait: signs of the tile (base k's words
+  // are one contiguous run of qr * 128 words), row scales of the tile's rows (item
+  // (k * ng + j) * 32 + r, so a warp reads 32 consecutive rows), column scales, indices.
+  const size_t words = static_cast<size_t>(p.tiles) * qr * 128;
+  const int n_bw = Ks * qr * 32, n_rs = Ks * ng * 32, n_cs = Ks * n;
+  const int n_items = max(max(n_bw, n_rs), max(n_cs, n));
+  for (int base = 0; base < n_items; base += kBatch * kRefThreads) {
+    uint4 bv[kBatch];
+    float rv[kBatch], cv[kBatch];
+    int iv[kBatch], ipv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * kRefThreads + tid;
+      if (i < n_bw) {
+        const int k = i / (qr * 32), w = i - k * qr * 32;
+        bv[u] = __ldg(reinterpret_cast<const uint4*>(p.bits + k * words + static_cast<size_t>(tile) * qr * 128) + w);
+      }
+      rv[u] = 0.f;
+      if (i < n_rs) {
+        const int kj = i >> 5, o = tile * 32 + (i & 31);
+        if (o < p.out) rv[u] = load_scale(p.rrs, static_cast<long long>(kj) * p.out + o, p.sdt);
+      }
+      if (i < n_cs) cv[u] = load_scale(p.rcs, i, p.sdt);
+      if (i < n) {
+        iv[u] = __ldg(p.idx + i);
+        ipv[u] = i > 0 ? __ldg(p.idx + i - 1) : 0;
+      }
     }
-    xg[i] = v;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * kRefThreads + tid;
+      if (i < n_bw) reinterpret_cast<uint4*>(sbits)[i] = bv[u];
+      if (i < n_rs) srs[i] = rv[u];
+      if (i < n_cs) cs[i] = cv[u];
+      if (i < n) {
+        sidx[i] = iv[u];
+        const int jt = min(max(iv[u], 0) / p.g, ng - 1);
+        const int jp = i == 0 ? -1 : min(max(ipv[u], 0) / p.g, ng - 1);
+        for (int j = jp + 1; j <= jt; ++j) gs[j] = i;
+      }
+    }
+  }
+  __syncthreads();
+
+  // activations, gathered through the index list once per CTA
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  for (int base = 0; base < MB * n; base += kBatch * kRefThreads) {
+    float xv[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * kRefThreads + tid;
+      xv[u] = 0.f;
+      if (i < MB * n) {
+        const int m = i / n, t = i - m * n;
+        const int c = sidx[t];
+        if (m < p.Mc) {
+          if (c < 0 || c >= p.in) atomicExch(p.status, static_cast<int>(BISCO_ERR_INVALID_ARG));
+          else xv[u] = load_act(p.X, static_cast<long long>(m) * p.ldx + c, p.xdt);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = base + u * kRefThreads + tid;
+      if (i < MB * n) xg[i] = xv[u];
+    }
   }
   __syncthreads();
 
@@ -120,12 +159,6 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
 #pragma unroll
   for (int m = 0; m < MB; ++m) acc[m] = 0.f;
   for (int j = warp; j < ng; j += kRefWarps) {
-    const int jn = j + kRefWarps;
-#pragma unroll
-    for (int k = 0; k < kMaxBases; ++k) {
-      rs_nxt[k] = 0.f;
-      if (k < Ks && jn < ng && row_ok) rs_nxt[k] = load_scale(p.rrs, (static_cast<long long>(k) * ng + jn) * p.out + o, p.sdt);
-    }
     const int t0 = gs[j], t1 = gs[j + 1];  // t0 > t1 only for indices out of order: no columns
     for (int k = 0; k < Ks; ++k) {
       float part[MB];
@@ -140,15 +173,10 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
 #pragma unroll
         for (int m = 0; m < MB; ++m) part[m] = fmaf(sc, xg[m * n + t], part[m]);
       }
-      float r = 0.f;
-#pragma unroll
-      for (int q = 0; q < kMaxBases; ++q)
-        if (q == k) r = rs_cur[q];
+      const float r = srs[(k * ng + j) * 32 + lane];
 #pragma unroll
       for (int m = 0; m < MB; ++m) acc[m] = fmaf(r, part[m], acc[m]);
     }
-#pragma unroll
-    for (int k = 0; k < kMaxBases; ++k) rs_cur[k] = rs_nxt[k];
   }
 #pragma unroll
   for (int m = 0; m < MB; ++m) red[(warp * 32 + lane) * MB + m] = acc[m];

@@ -198,10 +198,12 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  *  BISCO_PATH_INTEGER_MMA: as AUTO, but chunks of up to 8 rows, single rows included,
  *    take the integer tensor-core kernel whenever its plan fits.
  * Layers with grouped row scales or a salient refinement run every batch chunk (8 rows
- * at most) on the integer tensor-core kernel under every policy; a refined chunk is
+ * at most; 4, 2 or 1 where the 8-row plan does not fit shared memory, e.g. 11008 input
+ * columns) on the integer tensor-core kernel under every policy; a refined chunk is
  * preceded by one refinement launch (BISCO_KERNEL_REFINE). BISCO_ERR_UNSUPPORTED when
- * the integer plan, or the refinement's shared-memory tables (about
- * 4 * (Ks + 9) * n_ref + 512 * Ks * ceil(n_ref / 128) bytes), do not fit.
+ * the integer plan of one row, or the refinement's shared-memory tables (about
+ * 4 * (Ks + 9) * n_ref + 512 * Ks * ceil(n_ref / 128) + 128 * Ks * ceil(in / g) bytes),
+ * do not fit.
  * Every path computes the same product within the documented tolerance.
  * Returns BISCO_ERR_INVALID_ARG for an unknown policy.
  */
