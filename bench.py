@@ -115,14 +115,18 @@ def algorithmic_flops(L, M):
 
 
 def traffic_for(workload, M):
-    """dram bytes per launch of the dominant kernel from a committed ncu capture,
-    or None if there is none for this workload or the kernel sources changed."""
+    """dram bytes per launch of the dominant kernel from a committed ncu capture (plus the
+    refinement launch of the same GEMV where the workload has one), or None if there is
+    none for this workload or the kernel sources changed."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        e = t.get(f"{workload}_M{M}")
+        e, r = t.get(f"{workload}_M{M}"), t.get(f"{workload}_M{M}_refine")
         if e and e.get("sources") == sources_digest():
-            return e["dram_bytes_per_launch"]
+            if r is None:
+                return e["dram_bytes_per_launch"]
+            if r.get("sources") == e["sources"]:
+                return e["dram_bytes_per_launch"] + r["dram_bytes_per_launch"]
     except Exception:
         pass
     return None
