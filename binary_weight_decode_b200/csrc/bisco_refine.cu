@@ -10,7 +10,7 @@
 // refinement's row scale of that group. The activations are gathered through idx once
 // per CTA (the translation layer of the mapping), the packed signs of the CTA's 32-row
 // tile, their row scales and the column scales are staged in shared memory, and each warp
-// takes every 8th group of the tile's rows with one lane per row.
+// takes every 16th group of the tile's rows with one lane per row.
 //
 // The result goes to an fp32 workspace buffer; the integer GEMV launch that follows on the
 // stream adds it to the rest of the row before the output is rounded. Weight-side data
@@ -28,7 +28,7 @@
 namespace bisco {
 namespace {
 
-constexpr int kRefWarps = 8;
+constexpr int kRefWarps = 16;  // 512 threads, <= 64 registers: 32K registers, so a CTA of the integer kernel (256 x 128) fits beside it
 constexpr int kRefThreads = kRefWarps * 32;
 
 __device__ __forceinline__ float load_scale(const void* a, long long i, int dt) {
@@ -64,7 +64,7 @@ __host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, in
 constexpr int kBatch = 4;
 
 template <int MB>
-__global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_constant__ RefineParam p) {
+__global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_constant__ RefineParam p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Ks = p.Ks, n = p.n_ref, ng = p.ngroups;
   const int qr = (n + 127) / 128;
@@ -165,13 +165,18 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
 #pragma unroll
       for (int m = 0; m < MB; ++m) part[m] = 0.f;
       const uint32_t* kb = sbits + static_cast<size_t>(k) * qr * 128;
-      uint32_t word = 0;
-      for (int t = t0; t < t1; ++t) {
-        if (t == t0 || (t & 31) == 0) word = kb[((t >> 7) * 32 + lane) * 4 + ((t >> 5) & 3)];
-        const float c = cs[k * n + t];
-        const float sc = ((word >> (t & 31)) & 1u) ? c : -c;
+      const float* ck = cs + static_cast<size_t>(k) * n;
+      for (int ta = t0; ta < t1;) {  // one 32-column sign word at a time
+        const int tb = min(t1, (ta | 31) + 1);
+        const uint32_t word = kb[((ta >> 7) * 32 + lane) * 4 + ((ta >> 5) & 3)];
+#pragma unroll 4
+        for (int t = ta; t < tb; ++t) {
+          const float c = ck[t];
+          const float sc = ((word >> (t & 31)) & 1u) ? c : -c;
 #pragma unroll
-        for (int m = 0; m < MB; ++m) part[m] = fmaf(sc, xg[m * n + t], part[m]);
+          for (int m = 0; m < MB; ++m) part[m] = fmaf(sc, xg[m * n + t], part[m]);
+        }
+        ta = tb;
       }
       const float r = srs[(k * ng + j) * 32 + lane];
 #pragma unroll
@@ -181,7 +186,7 @@ __global__ void __launch_bounds__(kRefThreads) refine_kernel(const __grid_consta
 #pragma unroll
   for (int m = 0; m < MB; ++m) red[(warp * 32 + lane) * MB + m] = acc[m];
   __syncthreads();
-  // the 8 warps' partials of a row, summed in warp order
+  // the warps' partials of a row, summed in warp order
   for (int i = tid; i < 32 * MB; i += kRefThreads) {
     const int r = i / MB, m = i - r * MB, oo = tile * 32 + r;
     if (oo >= p.out || m >= p.Mc) continue;
