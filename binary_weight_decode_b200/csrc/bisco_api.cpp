@@ -524,8 +524,7 @@ bisco_status bisco_gemv(const bisco_layer* L, const void* X, int32_t x_dtype, in
     const void* Xc = static_cast<const unsigned char*>(X) + static_cast<size_t>(ch.m0) * L->in * xb;
     void* Yc = static_cast<unsigned char*>(Y) + static_cast<size_t>(ch.m0) * L->out * yb;
     // the refinement term first; the integer launch that writes this chunk's Y adds it
-    if (rbuf && launch_refine(L, Xc, x_dtype, ch.Mc, rbuf, status, cached_smem_limit(dev), s) != cudaSuccess)
-      return BISCO_ERR_CUDA;
+    if (rbuf && launch_refine(L, Xc, x_dtype, ch.Mc, rbuf, status, s) != cudaSuccess) return BISCO_ERR_CUDA;
     if (ch.fused) {
       PassParam pz{}, py{};
       pass_z(L, pz, Xc, x_dtype, ch.Mc, zbuf, status);

@@ -161,9 +161,8 @@ struct RefineParam {
 // Shared memory of one refinement launch at batch block MB (0 for a layer without one).
 size_t refine_smem_bytes(const bisco_layer* L, int MB);
 // The salient refinement term of a layer for Mc batch rows of X into rref [Mc][out] (fp32).
-// smem_limit: opt-in shared memory per CTA (the dense form is used when it fits).
 cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, int Mc, float* rref, int* status,
-                          size_t smem_limit, cudaStream_t stream);
+                          cudaStream_t stream);
 cudaError_t imma_ensure_attrs();
 
 // Tensor-core path (16..128 batch rows per launch): one launch per pass.

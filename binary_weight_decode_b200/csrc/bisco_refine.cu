@@ -52,23 +52,18 @@ __device__ __forceinline__ float load_act(const void* a, long long i, int dt) {
 //   sidx  [n_ref]           the gathered column indices
 //   gs    [ngroups + 1]     first gathered column of each group
 //   red   [kRefWarps][32][MB] per-warp partial sums of the tile's rows
-//   wd    [n_ref][32]       dense form only: the tile's refinement weights
-__host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, int MB, bool dense) {
+__host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, int MB) {
   const size_t qr = (static_cast<size_t>(n_ref) + 127) / 128;
   return 4 * (static_cast<size_t>(Ks) * qr * 128 + static_cast<size_t>(Ks) * ngroups * 32 +
               static_cast<size_t>(Ks) * n_ref + static_cast<size_t>(MB) * n_ref + n_ref + ngroups + 1 +
-              static_cast<size_t>(kRefWarps) * 32 * MB + (dense ? static_cast<size_t>(n_ref) * 32 : 0));
+              static_cast<size_t>(kRefWarps) * 32 * MB);
 }
 
 // Loads in flight per thread in one staging round: every load of a round is issued before
 // the first of its values is stored, so a round costs one memory latency.
 constexpr int kBatch = 4;
 
-// DENSE: the tile's weights W[t][r] = sum_k r_k[group of t][r] c_k[t] (2b - 1) are formed in
-// shared memory before the dependency wait, so that after it only the gather and one dot
-// product of n_ref / 16 columns per warp remain (used when they fit in shared memory);
-// otherwise each warp walks its groups bit by bit after the wait.
-template <int MB, bool DENSE>
+template <int MB>
 __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_constant__ RefineParam p) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int Ks = p.Ks, n = p.n_ref, ng = p.ngroups;
@@ -80,7 +75,6 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   int* sidx = reinterpret_cast<int*>(xg + static_cast<size_t>(MB) * n);
   int* gs = sidx + n;
   float* red = reinterpret_cast<float*>(gs + ng + 1);
-  float* wd = red + kRefWarps * 32 * MB;
 
   asm volatile("griddepcontrol.launch_dependents;");
   const int tile = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -136,21 +130,6 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   }
   __syncthreads();
 
-  if constexpr (DENSE) {
-    // item i = t * 32 + r: lane r of every warp owns row r (kRefThreads is a multiple of 32)
-    for (int i = tid; i < n * 32; i += kRefThreads) {
-      const int t = i >> 5, r = i & 31;
-      const int j = min(max(sidx[t], 0) / p.g, ng - 1);
-      float w = 0.f;
-      for (int k = 0; k < Ks; ++k) {
-        const uint32_t word = sbits[static_cast<size_t>(k) * qr * 128 + ((t >> 7) * 32 + r) * 4 + ((t >> 5) & 3)];
-        const float c = cs[k * n + t] * srs[(k * ng + j) * 32 + r];
-        w += ((word >> (t & 31)) & 1u) ? c : -c;
-      }
-      wd[i] = w;
-    }
-  }
-
   // activations, gathered through the index list once per CTA
   asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int base = 0; base < MB * n; base += kBatch * kRefThreads) {
@@ -179,17 +158,7 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   float acc[MB];
 #pragma unroll
   for (int m = 0; m < MB; ++m) acc[m] = 0.f;
-  if constexpr (DENSE) {
-    const int cw = (n + kRefWarps - 1) / kRefWarps;
-    const int ta = warp * cw, tb = min(n, ta + cw);
-#pragma unroll 4
-    for (int t = ta; t < tb; ++t) {
-      const float w = wd[t * 32 + lane];
-#pragma unroll
-      for (int m = 0; m < MB; ++m) acc[m] = fmaf(w, xg[m * n + t], acc[m]);
-    }
-  }
-  for (int j = warp; !DENSE && j < ng; j += kRefWarps) {
+  for (int j = warp; j < ng; j += kRefWarps) {
     const int t0 = gs[j], t1 = gs[j + 1];  // t0 > t1 only for indices out of order: no columns
     for (int k = 0; k < Ks; ++k) {
       float part[MB];
@@ -227,12 +196,12 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   }
 }
 
-template <int MB, bool DENSE>
+template <int MB>
 cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t stream) {
   static std::atomic<size_t> allowed{48 * 1024};  // dynamic shared memory this kernel is opted in to
   if (smem > allowed.load()) {
     const cudaError_t e =
-        cudaFuncSetAttribute(refine_kernel<MB, DENSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaFuncSetAttribute(refine_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     allowed.store(smem);
   }
@@ -246,7 +215,7 @@ cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t str
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, refine_kernel<MB, DENSE>, p);
+  return cudaLaunchKernelEx(&cfg, refine_kernel<MB>, p);
 }
 
 }  // namespace
@@ -254,11 +223,11 @@ cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t str
 size_t refine_smem_bytes(const bisco_layer* L, int MB) {
   if (L->ref_bases <= 0 || L->row_group <= 0) return 0;
   const int ng = static_cast<int>((static_cast<long long>(L->in) + L->row_group - 1) / L->row_group);
-  return refine_smem(L->ref_bases, L->n_ref, ng, MB, false);
+  return refine_smem(L->ref_bases, L->n_ref, ng, MB);
 }
 
 cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, int Mc, float* rref, int* status,
-                          size_t smem_limit, cudaStream_t stream) {
+                          cudaStream_t stream) {
   RefineParam p{};
   p.bits = L->ref_bits;
   p.rrs = L->ref_row_scale;
@@ -279,21 +248,12 @@ cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, 
   p.rref = rref;
   p.status = status;
   const int MB = Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8;
-  const size_t dense = refine_smem(p.Ks, p.n_ref, p.ngroups, MB, true);
-  if (dense <= smem_limit) {
-    switch (MB) {
-      case 1: return launch_refine_mb<1, true>(p, dense, stream);
-      case 2: return launch_refine_mb<2, true>(p, dense, stream);
-      case 4: return launch_refine_mb<4, true>(p, dense, stream);
-      default: return launch_refine_mb<8, true>(p, dense, stream);
-    }
-  }
-  const size_t smem = refine_smem(p.Ks, p.n_ref, p.ngroups, MB, false);
+  const size_t smem = refine_smem(p.Ks, p.n_ref, p.ngroups, MB);
   switch (MB) {
-    case 1: return launch_refine_mb<1, false>(p, smem, stream);
-    case 2: return launch_refine_mb<2, false>(p, smem, stream);
-    case 4: return launch_refine_mb<4, false>(p, smem, stream);
-    default: return launch_refine_mb<8, false>(p, smem, stream);
+    case 1: return launch_refine_mb<1>(p, smem, stream);
+    case 2: return launch_refine_mb<2>(p, smem, stream);
+    case 4: return launch_refine_mb<4>(p, smem, stream);
+    default: return launch_refine_mb<8>(p, smem, stream);
   }
 }
 

@@ -4,9 +4,8 @@ columns of every column group, stored densely over the gathered columns, with on
 scale per (base, row, group) and one column scale per (base, gathered column):
 W[o][idx_t] += sum_k r_k[o][idx_t // g] c_k[t] (2b - 1).
 
-The library computes the term in its own launch (BISCO_KERNEL_REFINE; a dense form when the
-tile's refinement weights fit in shared memory, a bit-walking form otherwise) and the
-integer tensor-core launch after it adds the term before rounding the output. Bars are those of
+The library computes the term in its own launch (BISCO_KERNEL_REFINE) and the integer
+tensor-core launch after it adds the term before rounding the output. Bars are those of
 tests/test_gemv_gpu.py; the main cases also check the device's refinement term alone (Y
 minus the same layer run without it) against the oracle's term, so a dropped, mis-signed or
 mis-grouped term cannot hide inside the bar when the rest of Y is much larger.
@@ -70,8 +69,8 @@ CASES = [
     (64, 128, 1, 0, 0.0, 128, "f32", (2, 128)),      # every column salient (n_ref = in)
     (96, 600, 2, 0, 0.0, 128, "bf16", (2, 1)),       # one salient column per group
     (40, 200, 1, 0, 0.0, 1024, "f32", (3, 5)),       # one group wider than the row
-    (96, 4096, 2, 8, 0.0, 128, "bf16", (2, 64)),     # n_ref = 2048: the tile's dense weights do not
-]                                                    # fit shared memory, the bit-walking form runs
+    (96, 4096, 2, 8, 0.0, 128, "bf16", (2, 64)),     # n_ref = 2048: 16 sign words per row
+]
 IDS = ["ragged", "g256_s16", "g384_f32", "ks4_many_groups", "all_salient", "s1", "g_wide", "half_salient"]
 
 
