@@ -28,8 +28,10 @@
 namespace bisco {
 namespace {
 
-constexpr int kRefWarps = 16;  // 512 threads, <= 64 registers: 32K registers, so a CTA of the integer kernel (256 x 128) fits beside it
-constexpr int kRefThreads = kRefWarps * 32;
+// Warps per CTA (one 32-row tile): 16 for batch blocks of up to 4 rows, 32 for 8 rows, where
+// each warp's chain of groups is the longest (measured on 2b-s16-g128 at 4096 x 4096: 32
+// warps are slower at one row, faster at eight).
+__host__ __device__ constexpr int ref_warps(int MB) { return MB >= 8 ? 32 : 16; }
 
 __device__ __forceinline__ float load_scale(const void* a, long long i, int dt) {
   if (dt == BISCO_BF16)
@@ -51,22 +53,26 @@ __device__ __forceinline__ float load_act(const void* a, long long i, int dt) {
 //   xg    [MB][n_ref]       gathered activations x[m][idx[t]]
 //   sidx  [n_ref]           the gathered column indices
 //   gs    [ngroups + 1]     first gathered column of each group
-//   red   [kRefWarps][32][MB] per-warp partial sums of the tile's rows
+//   red   [warps][32][MB]   per-warp partial sums of the tile's rows
 __host__ __device__ inline size_t refine_smem(int Ks, int n_ref, int ngroups, int MB) {
   const size_t qr = (static_cast<size_t>(n_ref) + 127) / 128;
   return 4 * (static_cast<size_t>(Ks) * qr * 128 + static_cast<size_t>(Ks) * ngroups * 32 +
               static_cast<size_t>(Ks) * n_ref + static_cast<size_t>(MB) * n_ref + n_ref + ngroups + 1 +
-              static_cast<size_t>(kRefWarps) * 32 * MB);
+              static_cast<size_t>(ref_warps(MB)) * 32 * MB);
 }
 
 // Loads in flight per thread in one staging round: every load of a round is issued before
 // the first of its values is stored, so a round costs one memory latency.
 constexpr int kBatch = 4;
 
-template <int MB>
-__global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_constant__ RefineParam p) {
+// KS: refinement bases (1..4), a template parameter so that the per-base partial sums of a
+// group stay in registers and each gathered activation is read once for all bases.
+template <int MB, int KS>
+__global__ void __launch_bounds__(ref_warps(MB) * 32, MB >= 8 ? 1 : 2) refine_kernel(const __grid_constant__ RefineParam p) {
+  constexpr int kRefWarps = ref_warps(MB), kRefThreads = kRefWarps * 32;
   extern __shared__ __align__(16) unsigned char smem[];
-  const int Ks = p.Ks, n = p.n_ref, ng = p.ngroups;
+  constexpr int Ks = KS;
+  const int n = p.n_ref, ng = p.ngroups;
   const int qr = (n + 127) / 128;
   uint32_t* sbits = reinterpret_cast<uint32_t*>(smem);
   float* srs = reinterpret_cast<float*>(sbits + static_cast<size_t>(Ks) * qr * 128);
@@ -160,27 +166,37 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   for (int m = 0; m < MB; ++m) acc[m] = 0.f;
   for (int j = warp; j < ng; j += kRefWarps) {
     const int t0 = gs[j], t1 = gs[j + 1];  // t0 > t1 only for indices out of order: no columns
-    for (int k = 0; k < Ks; ++k) {
-      float part[MB];
+    float part[KS][MB];
 #pragma unroll
-      for (int m = 0; m < MB; ++m) part[m] = 0.f;
-      const uint32_t* kb = sbits + static_cast<size_t>(k) * qr * 128;
-      const float* ck = cs + static_cast<size_t>(k) * n;
-      for (int ta = t0; ta < t1;) {  // one 32-column sign word at a time
-        const int tb = min(t1, (ta | 31) + 1);
-        const uint32_t word = kb[((ta >> 7) * 32 + lane) * 4 + ((ta >> 5) & 3)];
-#pragma unroll 4
-        for (int t = ta; t < tb; ++t) {
-          const float c = ck[t];
-          const float sc = ((word >> (t & 31)) & 1u) ? c : -c;
+    for (int k = 0; k < KS; ++k)
 #pragma unroll
-          for (int m = 0; m < MB; ++m) part[m] = fmaf(sc, xg[m * n + t], part[m]);
+      for (int m = 0; m < MB; ++m) part[k][m] = 0.f;
+    for (int ta = t0; ta < t1;) {  // one 32-column sign word (per base) at a time
+      const int tb = min(t1, (ta | 31) + 1);
+      uint32_t word[KS];
+#pragma unroll
+      for (int k = 0; k < KS; ++k)
+        word[k] = sbits[static_cast<size_t>(k) * qr * 128 + ((ta >> 7) * 32 + lane) * 4 + ((ta >> 5) & 3)];
+#pragma unroll 2
+      for (int t = ta; t < tb; ++t) {
+        float xv[MB];
+#pragma unroll
+        for (int m = 0; m < MB; ++m) xv[m] = xg[m * n + t];
+#pragma unroll
+        for (int k = 0; k < KS; ++k) {
+          const float c = cs[k * n + t];
+          const float sc = ((word[k] >> (t & 31)) & 1u) ? c : -c;
+#pragma unroll
+          for (int m = 0; m < MB; ++m) part[k][m] = fmaf(sc, xv[m], part[k][m]);
         }
-        ta = tb;
       }
+      ta = tb;
+    }
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
       const float r = srs[(k * ng + j) * 32 + lane];
 #pragma unroll
-      for (int m = 0; m < MB; ++m) acc[m] = fmaf(r, part[m], acc[m]);
+      for (int m = 0; m < MB; ++m) acc[m] = fmaf(r, part[k][m], acc[m]);
     }
   }
 #pragma unroll
@@ -196,18 +212,18 @@ __global__ void __launch_bounds__(kRefThreads, 2) refine_kernel(const __grid_con
   }
 }
 
-template <int MB>
+template <int MB, int KS>
 cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t stream) {
   static std::atomic<size_t> allowed{48 * 1024};  // dynamic shared memory this kernel is opted in to
   if (smem > allowed.load()) {
     const cudaError_t e =
-        cudaFuncSetAttribute(refine_kernel<MB>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaFuncSetAttribute(refine_kernel<MB, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     allowed.store(smem);
   }
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(p.tiles);
-  cfg.blockDim = dim3(kRefThreads);
+  cfg.blockDim = dim3(ref_warps(MB) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -215,7 +231,17 @@ cudaError_t launch_refine_mb(const RefineParam& p, size_t smem, cudaStream_t str
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, refine_kernel<MB>, p);
+  return cudaLaunchKernelEx(&cfg, refine_kernel<MB, KS>, p);
+}
+
+template <int MB>
+cudaError_t launch_refine_ks(const RefineParam& p, size_t smem, cudaStream_t stream) {
+  switch (p.Ks) {
+    case 1: return launch_refine_mb<MB, 1>(p, smem, stream);
+    case 2: return launch_refine_mb<MB, 2>(p, smem, stream);
+    case 3: return launch_refine_mb<MB, 3>(p, smem, stream);
+    default: return launch_refine_mb<MB, 4>(p, smem, stream);
+  }
 }
 
 }  // namespace
@@ -250,10 +276,10 @@ cudaError_t launch_refine(const bisco_layer* L, const void* X, int32_t x_dtype, 
   const int MB = Mc <= 1 ? 1 : Mc <= 2 ? 2 : Mc <= 4 ? 4 : 8;
   const size_t smem = refine_smem(p.Ks, p.n_ref, p.ngroups, MB);
   switch (MB) {
-    case 1: return launch_refine_mb<1>(p, smem, stream);
-    case 2: return launch_refine_mb<2>(p, smem, stream);
-    case 4: return launch_refine_mb<4>(p, smem, stream);
-    default: return launch_refine_mb<8>(p, smem, stream);
+    case 1: return launch_refine_ks<1>(p, smem, stream);
+    case 2: return launch_refine_ks<2>(p, smem, stream);
+    case 4: return launch_refine_ks<4>(p, smem, stream);
+    default: return launch_refine_ks<8>(p, smem, stream);
   }
 }
 

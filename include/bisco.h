@@ -202,8 +202,8 @@ bisco_status bisco_sync_status(void* stream, const void* ws);
  * columns) on the integer tensor-core kernel under every policy; a refined chunk is
  * preceded by one refinement launch (BISCO_KERNEL_REFINE). BISCO_ERR_UNSUPPORTED when
  * the integer plan of one row, or the refinement's shared-memory tables (about
- * 4 * (Ks + 9) * n_ref + 512 * Ks * ceil(n_ref / 128) + 128 * Ks * ceil(in / g) bytes),
- * do not fit.
+ * 4 * (Ks + 9) * n_ref + 512 * Ks * ceil(n_ref / 128) + 128 * Ks * ceil(in / g) + 32768
+ * bytes), do not fit.
  * Every path computes the same product within the documented tolerance.
  * Returns BISCO_ERR_INVALID_ARG for an unknown policy.
  */
