@@ -614,8 +614,10 @@ __global__ void __launch_bounds__(kIT, 2)
               }
             }
             // drain: D = sum_b (acc_b >> b) per slot, times the slot weight, summed over the
-            // slots of each batch row (the four lanes of a quad), times the row scale; the run
-            // that starts the CTA's range of the segment also subtracts r * sum_i v_i
+            // slots of each batch row held by this lane, times the row scale (the same for the
+            // four lanes of a quad, so the sum over the quad's slots waits until the block is
+            // done); the run that starts the CTA's range of the segment also subtracts
+            // r * sum_i v_i, once per quad
             float wlo[NG][2];
 #pragma unroll
             for (int g = 0; g < NG; ++g) {
@@ -654,9 +656,7 @@ __global__ void __launch_bounds__(kIT, 2)
 #pragma unroll
                 for (int mm = 0; mm < MB; ++mm) {
                   float v = cv[r][mm];
-                  v += __shfl_xor_sync(0xffffffffu, v, 1);
-                  v += __shfl_xor_sync(0xffffffffu, v, 2);
-                  if (first_run) v -= S.ssf[ls * MB + mm];
+                  if (first_run && tq == 0) v -= S.ssf[ls * MB + mm];
                   pacc[h][r][mm] = fmaf(v, rs, pacc[h][r][mm]);
                 }
               }
@@ -664,6 +664,18 @@ __global__ void __launch_bounds__(kIT, 2)
           }
           ur = ue;
         }
+        // the sums over the slots of each batch row (the four lanes of a quad)
+#pragma unroll
+        for (int h = 0; h < RH; ++h)
+#pragma unroll
+          for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int mm = 0; mm < MB; ++mm) {
+              float v = pacc[h][r][mm];
+              v += __shfl_xor_sync(0xffffffffu, v, 1);
+              v += __shfl_xor_sync(0xffffffffu, v, 2);
+              pacc[h][r][mm] = v;
+            }
         // push the block's row partial sums to the CTA that owns the rows, one store per
         // lane: after the quad reduction every lane of a quad holds the same sums, so lane
         // tq takes one (half, row) pair (32-row blocks) or one row and half the batch rows
