@@ -75,6 +75,46 @@ def test_decoder_stream_matrices():
     assert total == 1_714_176_000
 
 
+def test_fluxbin_workloads_and_their_bytes():
+    # FluxBin 2b-g128 and 2b-s16-g128 on 4096 x 4096 ("FluxBin", Sec. 4 configurations):
+    # grouped row scales of 128 columns; 16 salient columns in each of the 32 groups for the
+    # refined one. The bench's byte accounting (restated so that the bench does not import
+    # the oracle) agrees with the oracle's.
+    import oracle
+    b = _bench()
+    (Lg, Xg), = b.base_matrices("fluxbin4096_g128", 1)
+    (Ls, Xs), = b.base_matrices("fluxbin4096_s16", 8)
+    assert Lg.group == Ls.group == 128 and Lg.K == Ls.K == 2 and getattr(Lg, "ref_K", 0) == 0
+    assert Ls.ref_K == 2 and len(Ls.ref_idx) == 512 and Xs.shape == (8, 4096)
+    assert all(((Ls.ref_idx >= 128 * j) & (Ls.ref_idx < 128 * (j + 1))).sum() == 16 for j in range(32))
+    for L, M in ((Lg, 1), (Ls, 1), (Ls, 8)):
+        assert b.algorithmic_bytes(L, M, 2, 2) == oracle.algorithmic_bytes(L, M, "bf16", "bf16")
+    assert b.algorithmic_bytes(Ls, 1, 2, 2) - b.algorithmic_bytes(Lg, 1, 2, 2) == 1_052_672
+
+
+def test_traffic_record_sums_the_refinement_launch_and_checks_the_sources(tmp_path):
+    # roofline.traffic is the DRAM bytes of one GEMV from committed captures: the dominant
+    # launch plus, for a refined layer, its refinement launch; null when either capture was
+    # taken from other kernel sources
+    import json
+    b = _bench()
+    dig = b.sources_digest()
+    rec = {"fluxbin4096_s16_M1": {"sources": dig, "dram_bytes_per_launch": 4_800_000},
+           "fluxbin4096_s16_M1_refine": {"sources": dig, "dram_bytes_per_launch": 1_100_000},
+           "attn4096_M1": {"sources": dig, "dram_bytes_per_launch": 4_276_000},
+           "attn4096_M2": {"sources": "0000000000000000", "dram_bytes_per_launch": 4_300_000},
+           "lowrank5120_M1": {"sources": dig, "dram_bytes_per_launch": 7_300_000},
+           "lowrank5120_M1_refine": {"sources": "0000000000000000", "dram_bytes_per_launch": 1}}
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps(rec))
+    b.TRAFFIC_FILE = str(f)
+    assert b.traffic_for("fluxbin4096_s16", 1) == 5_900_000
+    assert b.traffic_for("attn4096", 1) == 4_276_000
+    assert b.traffic_for("attn4096", 2) is None        # captured from other sources
+    assert b.traffic_for("lowrank5120", 1) is None     # its second launch was
+    assert b.traffic_for("fluxbin4096_g128", 1) is None  # never captured
+
+
 def test_reference_arm_prints_one_contract_line():
     # bench.py --impl reference times the oracle on the host cores (no GPU needed) and
     # prints one JSON line with the base contract's keys, the same metric and config as
