@@ -26,6 +26,8 @@ PINS = [
     P.test_grouped_all_plus_one_is_a_sum_of_group_sums,
     P.test_biloco_decomposition_reproduces_the_page_toy,
     lambda: P.test_grouped_brute_force_all_sign_patterns(2, 4, 1, 2),
+    P.test_refinement_all_plus_one_is_a_scaled_gathered_sum,
+    P.test_refinement_brute_force_over_every_sign_pattern,
 ]
 
 
@@ -158,6 +160,27 @@ def _salient_wrong_column(layer, rows):
     return W
 
 
+def _refinement_variant(layer, rows, *, drop=False, group_of_position=False, col_scale_base0=False,
+                        invert=False, column_t=False):
+    W = np.zeros((len(rows), layer.in_), dtype=np.float64)
+    Ks = getattr(layer, "ref_K", 0)
+    if not Ks or drop:
+        return W
+    g = layer.group
+    idx = np.asarray(layer.ref_idx, dtype=np.int64)
+    n = len(idx)
+    R = O.decode_values(layer.ref_row_scale, layer.scale_dtype).reshape(Ks, layer.out, -1)
+    C = O.decode_values(layer.ref_col_scale, layer.scale_dtype).reshape(Ks, n)
+    bits = np.asarray(layer.ref_bits).reshape(Ks, -1)
+    grp = (np.arange(n) // g) if group_of_position else (idx // g)
+    cols = np.arange(n) if column_t else idx
+    for k in range(Ks):
+        S = O.unpack_bit_rows(bits[k], layer.out, n, rows) * (-1 if invert else 1)
+        ck = C[0] if col_scale_base0 else C[k]
+        W[:, cols] += R[k][rows][:, grp] * S * ck[None, :]
+    return W
+
+
 def _gemv_untransposed(layer, X, x_dtype, rows):
     Xd = O.decode_values(X, x_dtype).reshape(-1, layer.in_)
     return Xd @ O.reconstruct_rows(layer, rows)
@@ -183,6 +206,14 @@ MUTATIONS = {
     "salient term dropped": ("_salient_part_rows", _salient_dropped),
     "salient column index ignored": ("_salient_part_rows", _salient_wrong_column),
     "W not transposed": ("gemv_rows", _gemv_untransposed),
+    "refinement dropped": ("_refinement_part_rows", lambda L, r: _refinement_variant(L, r, drop=True)),
+    "refinement row-scale group taken from the gathered position":
+        ("_refinement_part_rows", lambda L, r: _refinement_variant(L, r, group_of_position=True)),
+    "refinement column scale of base 0 reused":
+        ("_refinement_part_rows", lambda L, r: _refinement_variant(L, r, col_scale_base0=True)),
+    "refinement signs inverted": ("_refinement_part_rows", lambda L, r: _refinement_variant(L, r, invert=True)),
+    "refinement added at column t instead of idx_t":
+        ("_refinement_part_rows", lambda L, r: _refinement_variant(L, r, column_t=True)),
     "decomposition coefficient over rows only": ("biloco_decompose", _decompose_alpha_over_rows),
     "decomposition refit skipped": ("biloco_decompose", _decompose_refit_skipped),
     "bf16 widened with wrong shift": ("decode_values", _bf16_wrong_shift),
