@@ -2,8 +2,9 @@
 
 The product Y = X W^T splits by output rows without any exchange inside the GEMV: a rank
 holding rows [r0, r1) of every sign matrix B_k, of U^T (the correction's first factor,
-stored transposed), of the row scales and of the salient block computes Y[:, r0:r1] with
-bisco_gemv on its own GPU; X, the column scales, V, alpha and the salient indices are
+stored transposed), of the row scales, of the salient block and of the salient refinement's
+signs and row scales computes Y[:, r0:r1] with bisco_gemv on its own GPU; X, the column
+scales, V, alpha, the salient indices and the refinement's indices and column scales are
 replicated (V x is recomputed on every rank: it is R x in, tiny next to the weights). One
 all-gather of the slices rebuilds Y where a consumer needs every row.
 
@@ -57,6 +58,13 @@ def shard_rows(layer, rank, world):
         kw["ut_bits"] = _tile_slice(layer.ut_bits, layer.out, layer.rank, t0, t1)
     if layer.n_sal:
         kw["sal_q"] = np.ascontiguousarray(np.asarray(layer.sal_q)[r0:r1])
+    ks = getattr(layer, "ref_K", 0) or 0
+    if ks:  # salient refinement: its signs (out x n_ref) and row scales [Ks][out][groups] by rows
+        n_ref = len(layer.ref_idx)
+        rb = np.asarray(layer.ref_bits).reshape(ks, -1)
+        kw["ref_bits"] = np.stack([_tile_slice(rb[k], layer.out, n_ref, t0, t1) for k in range(ks)])
+        rr = np.asarray(layer.ref_row_scale).reshape(ks, layer.out, -1)
+        kw["ref_row_scale"] = np.ascontiguousarray(rr[:, r0:r1])
     return dataclasses.replace(layer, **kw)
 
 

@@ -155,6 +155,18 @@ def test_refined_layer_in_a_group_call():
         check(Yd.cpu().numpy().astype(np.float64), oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
 
 
+@pytest.mark.parametrize("world,M", [(3, 1), (2, 8)])
+def test_refined_layer_row_shards_on_the_device(world, M):
+    # row shards of a refined layer (its signs and row scales cut by rows, indices and
+    # column scales replicated) run one after another on one GPU; side by side they meet the
+    # bar against the whole layer's oracle product
+    from binary_weight_decode_b200 import shard
+    X = make_activations(0, (858, M), M, 700, "bf16")
+    L = make_layer(0, (858,), 200, 700, 2, "bf16", rank=8, group=128, refine=(2, 8))
+    parts = [run(shard.shard_rows(L, r, world), X, "bf16") for r in range(world)]
+    check(np.concatenate(parts, axis=1), oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
+
+
 def test_out_of_range_refinement_index_is_reported_not_read():
     # a gathered column outside [0, in) is recorded as BISCO_ERR_INVALID_ARG by the kernel,
     # which reads zero in its place

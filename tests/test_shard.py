@@ -17,7 +17,7 @@ import torch.multiprocessing as mp  # noqa: E402
 
 import oracle  # noqa: E402
 from binary_weight_decode_b200 import shard  # noqa: E402
-from synth import make_activations, make_layer  # noqa: E402
+from synth import make_activations, make_layer, packed_words  # noqa: E402
 
 
 @pytest.mark.parametrize("out,world", [(200, 1), (200, 2), (200, 3), (200, 7), (64, 4), (33, 2), (4096, 8)])
@@ -61,6 +61,24 @@ def test_grouped_layers_shard_by_rows(world):
     for rank, (r0, r1) in enumerate(shard.shard_bounds(L.out, world)):
         S = shard.shard_rows(L, rank, world)
         assert np.array_equal(oracle.reconstruct(S), W[r0:r1])
+
+
+@pytest.mark.parametrize("world", [2, 3, 5])
+def test_refined_layers_shard_by_rows(world):
+    # the salient refinement's signs (out x n_ref, tiled) and row scales [Ks][out][groups]
+    # are cut along the rows; its indices and column scales are replicated
+    L = make_layer(0, (612,), 150, 700, 2, "bf16", rank=8, group=128, refine=(2, 8))
+    X = make_activations(0, (612,), 3, 700, "bf16")
+    W = oracle.reconstruct(L)
+    Y = oracle.gemv(L, X, "bf16")
+    for rank, (r0, r1) in enumerate(shard.shard_bounds(L.out, world)):
+        S = shard.shard_rows(L, rank, world)
+        if S.out == 0:
+            continue
+        assert np.array_equal(S.ref_idx, L.ref_idx) and np.array_equal(S.ref_col_scale, L.ref_col_scale)
+        assert np.asarray(S.ref_bits).reshape(2, -1).shape[1] == packed_words(S.out, len(L.ref_idx))
+        assert np.array_equal(oracle.reconstruct(S), W[r0:r1])
+        assert np.allclose(oracle.gemv(S, X, "bf16"), Y[:, r0:r1], rtol=1e-12, atol=0)
 
 
 def _free_port():
