@@ -118,7 +118,11 @@ typedef struct {
      are grouped like the global ones). */
   int32_t ref_bases;        /* Ks in 0..4; 0 = none                                    */
   int32_t n_ref;            /* salient columns of the refinement, >= 1 when Ks > 0     */
-  const int32_t* ref_idx;   /* [n_ref] strictly ascending column indices in [0, in)    */
+  const int32_t* ref_idx;   /* [n_ref] strictly ascending column indices in [0, in); an
+                               index outside that range is read as a zero activation and
+                               recorded as BISCO_ERR_INVALID_ARG in the workspace status;
+                               indices out of order give wrong groups (never an
+                               out-of-bounds access)                                    */
   const uint32_t* ref_bits; /* [Ks][bisco_packed_words(out, n_ref)] packed signs       */
   const void* ref_row_scale; /* [Ks][ceil(in/row_group)][out], dtype scale_dtype       */
   const void* ref_col_scale; /* [Ks][n_ref], dtype scale_dtype                         */
