@@ -155,6 +155,26 @@ def test_refined_layer_in_a_group_call():
         check(Yd.cpu().numpy().astype(np.float64), oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
 
 
+@pytest.mark.parametrize("keep", [0, 1, 2])
+@pytest.mark.parametrize("M", [1, 8])
+def test_refinement_with_empty_groups(keep, M):
+    # only the groups j with j % 3 == keep hold salient columns: the first, last or inner
+    # groups have none (the group boundaries of an empty group coincide)
+    X = make_activations(0, (859, M), M, 1100, "bf16")
+    L = make_layer(0, (859,), 170, 1100, 2, "bf16", rank=8, group=128, refine=(2, 8))
+    idx = np.asarray(L.ref_idx)
+    sel = (idx // 128) % 3 == keep
+    n = int(sel.sum())
+    S = np.stack([oracle.unpack_bit_matrix(np.asarray(L.ref_bits)[k], L.out, len(idx)) for k in range(2)])
+    L.ref_idx = np.ascontiguousarray(idx[sel]).astype(np.int32)
+    L.ref_bits = np.stack([oracle.pack_bit_matrix(S[k][:, sel]) for k in range(2)])
+    L.ref_col_scale = np.ascontiguousarray(np.asarray(L.ref_col_scale)[:, sel])
+    assert 0 < n < len(idx)
+    Y = run(L, X, "bf16", "f32")
+    check(Y, oracle.gemv(L, X, "bf16"), X, "bf16", "f32")
+    check_term(L, X, "bf16", Y)
+
+
 @pytest.mark.parametrize("world,M", [(3, 1), (2, 8)])
 def test_refined_layer_row_shards_on_the_device(world, M):
     # row shards of a refined layer (its signs and row scales cut by rows, indices and
